@@ -1,0 +1,156 @@
+"""Seeded synthetic inputs for the DF-SSM scaffold linear (inputs only).
+
+This module draws the tensors the layer consumes; it contains none of the
+layer's arithmetic. Both the CPU oracle and the CUDA path read the bytes it
+writes. The C side (``synth.c``) defines the generator: SplitMix64 in counter
+mode, keyed by ``(seed, stream_id)``.
+
+Shapes follow Mamba-2 1.3B (d_model 2048, 48 layers): in_proj 2048 -> 8512
+(2*4096 z/x + 2*128 B/C + 64 dt heads), out_proj 4096 -> 2048, LoRA rank 16
+("Density Field State Space Models", gist.science technical summary, §2.B:
+rank-16 int8 LoRA on every in_proj and out_proj of all 48 layers).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "synth.c")
+_LIB_PATH = os.path.join(_HERE, "libdfssm_synth.so")
+
+MASTER_SEED = 0x20260610
+RANK = 16
+D_MODEL = 2048
+IN_PROJ = (2048, 8512)    # (d_in, d_out)
+OUT_PROJ = (4096, 2048)
+N_LAYERS = 48
+
+# tensor ids inside a stream
+T_X, T_COLS, T_SIGN, T_ALPHA, T_WA, T_SA, T_WB, T_SB = range(8)
+KIND_WEIGHTS, KIND_ACT = 1, 2
+
+
+def build(force: bool = False) -> str:
+    """Compile synth.c into libdfssm_synth.so next to it (gcc, OpenMP)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-std=c11",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+_lib = None
+
+
+def _L():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        u64, i64, i32, vp, dbl = (ctypes.c_uint64, ctypes.c_int64, ctypes.c_int,
+                                  ctypes.c_void_p, ctypes.c_double)
+        lib.dfssm_synth_key.restype = u64
+        lib.dfssm_synth_key.argtypes = [u64, u64]
+        lib.dfssm_synth_raw.argtypes = [u64, u64, i64, vp]
+        lib.dfssm_synth_outlier_cols.argtypes = [u64, i32, i32, vp]
+        lib.dfssm_synth_x.argtypes = [u64, u64, i32, i32, vp]
+        lib.dfssm_synth_bits.argtypes = [u64, i64, vp]
+        lib.dfssm_synth_uniform_f32.argtypes = [u64, i64, dbl, dbl, vp]
+        lib.dfssm_synth_int8_sym127.argtypes = [u64, i64, vp]
+        lib.dfssm_synth_f64_to_bf16.restype = ctypes.c_uint16
+        lib.dfssm_synth_f64_to_bf16.argtypes = [dbl]
+        _lib = lib
+    return _lib
+
+
+def stream_id(kind: int, cfg: int, m: int, index: int, tensor: int) -> int:
+    assert 0 <= m < (1 << 20) and 0 <= index < (1 << 24) and 0 <= tensor < 256
+    return (kind << 60) | (cfg << 52) | (m << 32) | (index << 8) | tensor
+
+
+def key(seed: int, sid: int) -> int:
+    return int(_L().dfssm_synth_key(seed & (2**64 - 1), sid))
+
+
+def _ptr(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data
+
+
+def raw(seed: int, sid: int, start: int, n: int) -> np.ndarray:
+    out = np.empty(n, dtype=np.uint64)
+    _L().dfssm_synth_raw(key(seed, sid), start, n, _ptr(out))
+    return out
+
+
+def outlier_cols(seed: int, cfg: int, m: int, index: int, d_in: int) -> np.ndarray:
+    n_out = int(np.floor(0.01 * d_in + 0.5))
+    out = np.empty(n_out, dtype=np.int32)
+    if n_out:
+        _L().dfssm_synth_outlier_cols(key(seed, stream_id(KIND_ACT, cfg, m, index, T_COLS)),
+                                      d_in, n_out, _ptr(out))
+    return out
+
+
+def activations(seed: int, cfg: int, index: int, m: int, d_in: int, out: np.ndarray | None = None):
+    """x for one linear: m x d_in bf16, returned as its uint16 bit patterns."""
+    if out is None:
+        out = np.empty((m, d_in), dtype=np.uint16)
+    assert out.dtype == np.uint16 and out.shape == (m, d_in)
+    kx = key(seed, stream_id(KIND_ACT, cfg, m, index, T_X))
+    kc = key(seed, stream_id(KIND_ACT, cfg, m, index, T_COLS))
+    _L().dfssm_synth_x(kx, kc, m, d_in, _ptr(out))
+    return out
+
+
+def linear_weights(seed: int, cfg: int, index: int, d_in: int, d_out: int, rank: int = RANK,
+                   out: dict | None = None) -> dict:
+    """Weights of one linear. ``sign`` is packed (d_out x d_in/8 bytes)."""
+    assert d_in % 8 == 0
+    shapes = {
+        "sign": ((d_out, d_in // 8), np.uint8), "alpha": ((d_out,), np.float32),
+        "wa": ((d_out, rank), np.int8), "sa": ((d_out,), np.float32),
+        "wb": ((rank, d_in), np.int8), "sb": ((rank,), np.float32),
+    }
+    if out is None:
+        out = {k: np.empty(s, dtype=t) for k, (s, t) in shapes.items()}
+    for k, (s, t) in shapes.items():
+        assert out[k].shape == s and out[k].dtype == t, (k, out[k].shape, s)
+    L = _L()
+
+    def k_(t):
+        return key(seed, stream_id(KIND_WEIGHTS, cfg, 0, index, t))
+
+    L.dfssm_synth_bits(k_(T_SIGN), out["sign"].size, _ptr(out["sign"]))
+    L.dfssm_synth_uniform_f32(k_(T_ALPHA), d_out, 0.005, 0.05, _ptr(out["alpha"]))
+    L.dfssm_synth_int8_sym127(k_(T_WA), out["wa"].size, _ptr(out["wa"]))
+    L.dfssm_synth_uniform_f32(k_(T_SA), d_out, 1e-4, 1e-3, _ptr(out["sa"]))
+    L.dfssm_synth_int8_sym127(k_(T_WB), out["wb"].size, _ptr(out["wb"]))
+    L.dfssm_synth_uniform_f32(k_(T_SB), rank, 1e-4, 1e-3, _ptr(out["sb"]))
+    return out
+
+
+def stack_shapes(n_layers: int = N_LAYERS):
+    """(d_in, d_out) of the 2*n_layers linears in stack order: in_proj, out_proj per layer."""
+    return [IN_PROJ if i % 2 == 0 else OUT_PROJ for i in range(2 * n_layers)]
+
+
+# Named workloads (sizes of the Mamba-2-1.3B scaffold-linear stack).
+WORKLOADS = {
+    "out_proj_m1": dict(cfg=0, shapes=[OUT_PROJ], m=1),
+    "in_proj_m1": dict(cfg=1, shapes=[IN_PROJ], m=1),
+    "stack48_m1": dict(cfg=2, shapes=stack_shapes(), m=1),
+    "stack48_m4": dict(cfg=3, shapes=stack_shapes(), m=4),
+    "stack48_m16": dict(cfg=3, shapes=stack_shapes(), m=16),
+    "stack48_m64": dict(cfg=3, shapes=stack_shapes(), m=64),
+    "stack48_m2048": dict(cfg=4, shapes=stack_shapes(), m=2048),
+}
+
+# Stack workloads draw their weights from one stream family (the M=1 stack's),
+# so every stack workload runs on identical weights.
+def weight_cfg(cfg: int) -> int:
+    return 2 if cfg in (2, 3, 4) else cfg

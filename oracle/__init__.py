@@ -1,0 +1,146 @@
+"""CPU oracle for the DF-SSM 1-bit scaffold + int8 LoRA linear (TEST INFRASTRUCTURE).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package. The library (``bit_gemv_gemm_dfssm_b200``)
+never imports it, and the two share no code. ``dfssm_oracle.cpp`` holds the
+arithmetic, written as plain loops; this file only loads it and marshals numpy
+arrays.
+
+Every function is pinned by ``tests/test_oracle_pins.py`` against brute force,
+closed forms, invariants and hand-computed fixtures; no function here is
+"parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dfssm_oracle.cpp")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with g++ (no fast-math, no FMA contraction, OpenMP)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["g++", "-O2", "-fPIC", "-shared", "-fopenmp", "-std=c++17",
+                               "-ffp-contract=off", "-fno-fast-math", "-o", tmp, _SRC])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+_lib = None
+
+
+def _L():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        vp, i32, i64, dbl = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
+        lib.dfssm_oracle_f64_to_bf16.restype = ctypes.c_uint16
+        lib.dfssm_oracle_f64_to_bf16.argtypes = [dbl]
+        lib.dfssm_oracle_f64_to_bf16_array.argtypes = [vp, i64, vp]
+        lib.dfssm_oracle_unpack_sign.argtypes = [vp, i32, i32, vp]
+        lib.dfssm_oracle_pack_sign_f32.argtypes = [vp, i32, i32, vp]
+        lib.dfssm_oracle_pack_sign_i8.argtypes = [vp, i32, i32, vp]
+        lib.dfssm_oracle_quantize.argtypes = [vp, i32, i32, vp, vp]
+        lib.dfssm_oracle_linear.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp,
+                                            vp, vp, vp, vp, vp, i32]
+        lib.dfssm_oracle_linear_sampled.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp,
+                                                    vp, vp, i64, vp, vp]
+        lib.dfssm_oracle_weight_bytes.argtypes = [i32, i32, i32, vp, vp, vp]
+        _lib = lib
+    return _lib
+
+
+def _c(a, dtype):
+    a = np.ascontiguousarray(a, dtype=dtype)
+    return a, a.ctypes.data
+
+
+def f64_to_bf16(v) -> np.ndarray:
+    """Round float64 values to bf16 (nearest, ties to even); returns uint16 bit patterns."""
+    v, pv = _c(v, np.float64)
+    out = np.empty(v.shape, dtype=np.uint16)
+    _L().dfssm_oracle_f64_to_bf16_array(pv, v.size, out.ctypes.data)
+    return out
+
+
+def bf16_bits_to_f64(b) -> np.ndarray:
+    """Exact widening of bf16 bit patterns (numpy only)."""
+    b = np.ascontiguousarray(b, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def unpack_sign(packed, d_out: int, d_in: int) -> np.ndarray:
+    p, pp = _c(packed, np.uint8)
+    assert p.size == d_out * d_in // 8
+    w = np.empty((d_out, d_in), dtype=np.int8)
+    _L().dfssm_oracle_unpack_sign(pp, d_out, d_in, w.ctypes.data)
+    return w
+
+
+def pack_sign(src, d_out: int, d_in: int) -> np.ndarray:
+    """Pack a frozen scaffold (fp32 or int8): value >= 0 -> bit 1 (+1), value < 0 -> bit 0."""
+    src = np.asarray(src)
+    out = np.empty((d_out, d_in // 8), dtype=np.uint8)
+    if src.dtype == np.float32:
+        s, ps = _c(src, np.float32)
+        rc = _L().dfssm_oracle_pack_sign_f32(ps, d_out, d_in, out.ctypes.data)
+    elif src.dtype == np.int8:
+        s, ps = _c(src, np.int8)
+        rc = _L().dfssm_oracle_pack_sign_i8(ps, d_out, d_in, out.ctypes.data)
+    else:
+        raise TypeError(src.dtype)
+    if rc:
+        raise ValueError("NaN in the scaffold source")
+    return out
+
+
+def quantize(x_bf16_bits, m: int, d_in: int):
+    """Per-token symmetric absmax int8 quantiser. Returns (q int8 m x d_in, s_x fp32 m)."""
+    x, px = _c(x_bf16_bits, np.uint16)
+    q = np.empty((m, d_in), dtype=np.int8)
+    sx = np.empty(m, dtype=np.float32)
+    _L().dfssm_oracle_quantize(px, m, d_in, q.ctypes.data, sx.ctypes.data)
+    return q, sx
+
+
+def linear(x_bf16_bits, w: dict, m: int, d_in: int, d_out: int, rank: int = 16, threads: int = 0):
+    """The whole layer. Returns dict(q, sx, acc, h, y) with y in float64."""
+    x, px = _c(x_bf16_bits, np.uint16)
+    keep = [_c(w["sign"], np.uint8), _c(w["alpha"], np.float32), _c(w["wa"], np.int8),
+            _c(w["sa"], np.float32), _c(w["wb"], np.int8), _c(w["sb"], np.float32)]
+    out = dict(q=np.empty((m, d_in), np.int8), sx=np.empty(m, np.float32),
+               acc=np.empty((m, d_out), np.int32), h=np.empty((m, rank), np.int32),
+               y=np.empty((m, d_out), np.float64))
+    _L().dfssm_oracle_linear(px, m, d_in, d_out, rank, *[p for _, p in keep],
+                             out["q"].ctypes.data, out["sx"].ctypes.data, out["acc"].ctypes.data,
+                             out["h"].ctypes.data, out["y"].ctypes.data, threads)
+    return out
+
+
+def linear_sampled(x_bf16_bits, w: dict, m: int, d_in: int, d_out: int, t_idx, o_idx, rank: int = 16):
+    """y (float64) and acc (int32) at the pairs (t_idx[i], o_idx[i]) only."""
+    x, px = _c(x_bf16_bits, np.uint16)
+    keep = [_c(w["sign"], np.uint8), _c(w["alpha"], np.float32), _c(w["wa"], np.int8),
+            _c(w["sa"], np.float32), _c(w["wb"], np.int8), _c(w["sb"], np.float32)]
+    t, pt = _c(t_idx, np.int32)
+    o, po = _c(o_idx, np.int32)
+    n = t.size
+    acc = np.empty(n, np.int32)
+    y = np.empty(n, np.float64)
+    _L().dfssm_oracle_linear_sampled(px, m, d_in, d_out, rank, *[p for _, p in keep], pt, po, n,
+                                     acc.ctypes.data, y.ctypes.data)
+    return dict(acc=acc, y=y)
+
+
+def weight_bytes(d_in: int, d_out: int, rank: int = 16):
+    """(sign, lora, scale) bytes of one linear as stored."""
+    a, b, c = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    _L().dfssm_oracle_weight_bytes(d_in, d_out, rank, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c))
+    return a.value, b.value, c.value
