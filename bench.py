@@ -1,0 +1,466 @@
+"""Benchmark of the DF-SSM scaffold + LoRA linear stack on B200.
+
+One step = one pass of the whole path over the 48-layer Mamba-2-1.3B
+in_proj/out_proj stack (96 linears, one dfssm_linear_stack_fwd call):
+activation quantisation + LoRA down-projection, scaffold contraction, LoRA
+up-projection and dequantisation, for every linear.
+
+Default workload: the stack at M = 1 token (metric: effective HBM GB/s and
+tokens/s). The same line carries the M = 2048 prefill pass (int8 tensor-core
+TOPS) under "prefill". Inputs are seeded synthetic tensors with the shapes and
+distributions of the Mamba-2-1.3B stack; two independent weight sets are
+alternated so that consecutive steps never find their weights in L2.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+Multi-GPU (launched by torchrun): every rank runs an independent replica on its
+own data (the layer has no exchange step); value = all ranks' work / max time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import dfssm_synth as synth  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+INT8_PER_BF16 = 2.0          # nominal dense int8 : bf16 tensor throughput (4.5 : 2.25 PFLOP/s)
+
+
+# --------------------------------------------------------------------------- work accounting
+
+def stack_bytes(shapes, m):
+    """Algorithmic bytes of one stack pass: 1-bit signs, int8 LoRA, fp32 scales, bf16 x in, bf16 y out."""
+    sign = sum(d_out * d_in // 8 for d_in, d_out in shapes)
+    lora = sum(16 * (d_out + d_in) for d_in, d_out in shapes)
+    scales = sum(4 * (2 * d_out + 16) for d_in, d_out in shapes)
+    act = sum(2 * m * (d_in + d_out) for d_in, d_out in shapes)
+    return sign + lora + scales + act
+
+
+def stack_ops(shapes, m):
+    """Integer ops of one pass: 2*M*d_in*d_out scaffold + 2*M*16*(d_in + d_out) LoRA."""
+    return sum(2 * m * d_in * d_out + 2 * m * 16 * (d_in + d_out) for d_in, d_out in shapes)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return dict(hbm=float(j["hbm_gbs"]), bf16=float(j["bf16_tflops"]),
+                    bf16_sustained=float(j.get("bf16_tflops_sustained", j["bf16_tflops"])), src="measured")
+    return dict(hbm=FALLBACK_HBM_GBS, bf16=FALLBACK_BF16_TFLOPS, bf16_sustained=1400.0, src="fallback")
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_gemv_gemm_dfssm_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per call from the committed ncu summary, if taken on the current kernels."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    rec = j.get(workload)
+    if not rec or rec.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_call")
+
+
+# --------------------------------------------------------------------------- distributed helpers
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def max_over_ranks(value: float, dist, device=None) -> float:
+    """Max of a per-rank float over the process group (identity without one)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, dist, device=None) -> float:
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def replica_seed(rank: int) -> int:
+    """Each replica draws its own inputs: the master seed offset by the rank."""
+    return synth.MASTER_SEED + 1000003 * rank
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle"}
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._th = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._th = threading.Thread(target=self._run, daemon=True)
+            self._th.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._th is not None:
+            self._th.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- CPU oracle (baseline arms)
+
+def oracle_stack_pass(shapes, m, seed, cfg, linear_ids, threads=0):
+    """Run the oracle over the given linears of the stack; returns (seconds, bytes, threads)."""
+    import oracle
+    inputs = []
+    for i in linear_ids:
+        d_in, d_out = shapes[i]
+        inputs.append((synth.linear_weights(seed, synth.weight_cfg(cfg), i, d_in, d_out),
+                       synth.activations(seed, cfg, i, m, d_in), d_in, d_out))
+    t0 = time.perf_counter()
+    for w, x, d_in, d_out in inputs:
+        oracle.linear(x, w, m, d_in, d_out, threads=threads)
+    dt = time.perf_counter() - t0
+    nbytes = stack_bytes([shapes[i] for i in linear_ids], m)
+    return dt, nbytes
+
+
+def oracle_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, wl_name):
+    """The oracle as it stands, timed on the host cores: one bounded sample per step."""
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    wl = synth.WORKLOADS[wl_name]
+    shapes, m, cfg = wl["shapes"], wl["m"], wl["cfg"]
+    sample_ids = [0, 1, 2, 3] if m <= 64 else [0, 1]
+    m_s = m if m <= 64 else 4
+    cores = oracle_threads()
+    for _ in range(args.warmup):
+        oracle_stack_pass(shapes, m_s, synth.MASTER_SEED, cfg, sample_ids)
+    tot_t, tot_b = 0.0, 0
+    for _ in range(args.steps):
+        dt, nb = oracle_stack_pass(shapes, m_s, synth.MASTER_SEED, cfg, sample_ids)
+        tot_t += dt
+        tot_b += nb
+    gbs = tot_b / tot_t / 1e9
+    sample = f"{len(sample_ids)} of {len(shapes)} linears (in_proj/out_proj pairs), M={m_s}, per step"
+    line = {
+        "impl": "reference", "metric": metric_name(), "value": gbs, "unit": "GB/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / max(args.steps, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8/int32/f64",
+        "data": "synthetic (seeded)", "config": {"workload": wl_name, "m": m, "linears": len(shapes)},
+        "cpu_baseline": {"kind": "oracle", "value": gbs, "unit": "GB/s", "cores": cores, "sample": sample},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def metric_name():
+    return "effective HBM GB/s and tokens/s for 48-layer in/out_proj stack at M=1; TOPS at M=2048"
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+class StackRunner:
+    """Device buffers, plan and stack entries for one workload, two weight sets."""
+
+    def __init__(self, shapes, m, cfg, seed, n_sets=2):
+        import torch
+        import bit_gemv_gemm_dfssm_b200 as dfssm
+        self.torch, self.dfssm = torch, dfssm
+        self.shapes, self.m, self.cfg = shapes, m, cfg
+        n = len(shapes)
+        self.plan = dfssm.dfssm_linear_plan([(d_in, d_out, m, dfssm.DFSSM_BF16) for d_in, d_out in shapes])
+        # contiguous activation buffers (one H2D and one D2H copy per step end to end)
+        self.x_off, self.y_off = [], []
+        xo = yo = 0
+        for d_in, d_out in shapes:
+            self.x_off.append(xo)
+            self.y_off.append(yo)
+            xo += m * d_in
+            yo += m * d_out
+        self.x_elems, self.y_elems = xo, yo
+        self.x_host = torch.empty(xo, dtype=torch.int16).pin_memory()
+        xh = self.x_host.numpy().view(np.uint16)
+        for i, (d_in, d_out) in enumerate(shapes):
+            synth.activations(seed, cfg, i, m, d_in, out=xh[self.x_off[i]:self.x_off[i] + m * d_in].reshape(m, d_in))
+        self.x = self.x_host.cuda()
+        self.y = torch.empty(yo, dtype=torch.bfloat16, device="cuda")
+        self.y_host = torch.empty(yo, dtype=torch.int16).pin_memory()
+        self.sets = []
+        for s in range(n_sets):
+            ws = []
+            for i, (d_in, d_out) in enumerate(shapes):
+                w = synth.linear_weights(seed + 7919 * s, synth.weight_cfg(cfg), i, d_in, d_out)
+                ws.append({k: torch.from_numpy(v).cuda() for k, v in w.items()})
+            ents = []
+            for i, w in enumerate(ws):
+                ents.append(dfssm.StackEntry(
+                    dfssm.weights_struct(w["sign"], w["alpha"], w["wa"], w["sa"], w["wb"], w["sb"]),
+                    self.x.data_ptr() + 2 * self.x_off[i], self.y.data_ptr() + 2 * self.y_off[i],
+                    dfssm.Debug(0, 0, 0, 0), i, 0))
+            raw = dfssm.stack_entries_bytes(ents)
+            edev = torch.frombuffer(bytearray(raw), dtype=torch.uint8).cuda()
+            self.sets.append((ws, edev))
+        self.n = n
+        torch.cuda.synchronize()
+
+    def weights_of(self, s):
+        return self.sets[s][0]
+
+    def call(self, s, stream):
+        self.dfssm.dfssm_linear_stack_fwd(self.plan, self.sets[s][1].data_ptr(), self.n, self.m, stream)
+
+    def graphs(self):
+        """One CUDA graph per weight set (each = one step)."""
+        torch = self.torch
+        gs = []
+        side = torch.cuda.Stream()
+        for s in range(len(self.sets)):
+            g = torch.cuda.CUDAGraph()
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.graph(g, stream=side):
+                self.call(s, torch.cuda.current_stream().cuda_stream)
+            gs.append(g)
+        torch.cuda.synchronize()
+        return gs
+
+    def check(self):
+        st, bits = self.dfssm.dfssm_plan_check(self.plan)
+        if st != self.dfssm.DFSSM_OK:
+            raise RuntimeError(f"device error word set: {bits:#x}")
+
+    def close(self):
+        self.dfssm.dfssm_plan_destroy(self.plan)
+
+
+def timed_device(torch, run_step, steps, warmup, dist, dev):
+    for i in range(warmup):
+        run_step(i)
+    torch.cuda.synchronize()
+    if dist is not None and dist.is_initialized():
+        dist.barrier()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        run_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None and dist.is_initialized():
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    return max_over_ranks(ms, dist, dev)
+
+
+def run_gpu(args, wl_name):
+    import torch
+    ws, rank, local = dist_env()
+    dist = None
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist_mod
+        dist = dist_mod
+        backend = os.environ.get("DFSSM_BENCH_BACKEND", "nccl")
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    wl = synth.WORKLOADS[wl_name]
+    shapes, m, cfg = wl["shapes"], wl["m"], wl["cfg"]
+    seed = replica_seed(rank)
+
+    r = StackRunner(shapes, m, cfg, seed)
+    graphs = r.graphs()
+    nb = stack_bytes(shapes, m)
+    nops = stack_ops(shapes, m)
+
+    def step(i):
+        graphs[i % 2].replay()
+
+    with ClockSampler(local) as clk:
+        ms = timed_device(torch, step, args.steps, args.warmup, dist, dev)
+    r.check()
+    ms_step = ms / args.steps
+    total_units = sum_over_ranks(float(m * args.steps), dist, dev)      # tokens, all ranks
+    total_bytes = sum_over_ranks(float(nb * args.steps), dist, dev)
+    value_gbs = total_bytes / (ms * 1e-3) / 1e9
+    tok_s = total_units / (ms * 1e-3)
+    achieved = nb / (ms_step * 1e-3) / 1e9
+
+    # end to end through the C ABI: pinned host x -> device, stack call, y -> pinned host
+    stream = torch.cuda.current_stream()
+
+    def e2e_step(i):
+        r.x.copy_(r.x_host, non_blocking=True)
+        r.call(i % 2, stream.cuda_stream)
+        r.y_host.copy_(r.y.view(torch.int16), non_blocking=True)
+
+    e2e_ms = timed_device(torch, e2e_step, args.steps, args.warmup, dist, dev)
+    e2e_gbs = sum_over_ranks(float(nb * args.steps), dist, dev) / (e2e_ms * 1e-3) / 1e9
+    h2d = r.x_elems * 2
+    d2h = r.y_elems * 2
+    r.check()
+    r.close()
+    del graphs
+
+    # prefill pass (M = 2048): int8 tensor-core TOPS
+    prefill = None
+    if not args.no_prefill:
+        pwl = synth.WORKLOADS["stack48_m2048"]
+        pr = StackRunner(pwl["shapes"], pwl["m"], pwl["cfg"], seed)
+        psteps = args.prefill_steps
+        pgraphs = pr.graphs()
+        with ClockSampler(local) as pclk:
+            pms = timed_device(torch, lambda i: pgraphs[i % 2].replay(), psteps, max(3, args.warmup // 10), dist, dev)
+        pr.check()
+        pops = stack_ops(pwl["shapes"], pwl["m"])
+        tops = sum_over_ranks(float(pops * psteps), dist, dev) / (pms * 1e-3) / 1e12
+        peak_i8 = peaks["bf16"] * INT8_PER_BF16
+        ach = pops / (pms / psteps * 1e-3) / 1e12
+        prefill = {
+            "workload": "stack48_m2048", "m": pwl["m"], "steps": psteps, "ms_per_step": pms / psteps,
+            "value": tops, "unit": "TOPS", "tokens_per_s": sum_over_ranks(float(pwl["m"] * psteps), dist, dev)
+            / (pms * 1e-3),
+            "roofline": {"bound": "tensor", "achieved": ach, "peak": peak_i8, "unit": "TOPS",
+                         "frac": ach / peak_i8, "traffic": recorded_traffic("stack48_m2048"),
+                         "peak_source": f"int8 = {INT8_PER_BF16:g} x {peaks['src']} bf16 burst"},
+            "clocks": pclk.summary(),
+        }
+        pr.close()
+        del pgraphs
+
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return 0
+
+    cpu = None
+    if ws == 1 and not args.no_cpu_baseline:
+        ids = list(range(len(shapes))) if m == 1 else [0, 1, 2, 3]
+        dt, cb = oracle_stack_pass(shapes, m, seed, cfg, ids)
+        cpu = {"kind": "oracle", "value": cb / dt / 1e9, "unit": "GB/s", "cores": oracle_threads(),
+               "sample": f"{len(ids)} of {len(shapes)} linears at M={m}, one pass, OpenMP over rows"}
+
+    line = {
+        "metric": metric_name(), "value": value_gbs, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8 x 1-bit -> int32, fp32 epilogue, bf16 out",
+        "data": "synthetic (seeded; Mamba-2-1.3B shapes, random weights)",
+        "config": {"workload": wl_name, "m": m, "linears": len(shapes), "layers": len(shapes) // 2,
+                   "d_model": 2048, "rank": 16, "parallelism": f"replicas x{ws}",
+                   "l2": "two weight sets alternated per step (2 x 171.8 MB > 126 MB L2)",
+                   "bytes_per_step": nb, "graph": "one CUDA graph per step"},
+        "tokens_per_s": tok_s,
+        "tops": sum_over_ranks(float(nops * args.steps), dist, dev) / (ms * 1e-3) / 1e12,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm"], "traffic": recorded_traffic(wl_name),
+                     "peak_source": f"{peaks['src']} copy bandwidth",
+                     "timed": "quant_kernel + decode_kernel per call (PDL-overlapped)"},
+        "e2e": {"value": e2e_gbs, "unit": "GB/s", "ms_per_step": e2e_ms / args.steps,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+        "cpu_baseline": cpu,
+        "prefill": prefill,
+    }
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="dfssm", choices=["dfssm", "reference"])
+    ap.add_argument("--workload", default="stack48_m1", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--prefill-steps", type=int, default=30)
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args, args.workload)
+    return run_gpu(args, args.workload)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,104 @@
+// Internal definitions shared by the libdfssm kernels (not part of the ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "../../include/dfssm.h"
+
+namespace dfssm {
+
+constexpr int kRank = 16;
+constexpr int kMaxDIn = 8192;
+constexpr int kMaxM = 65536;
+
+// Per-linear shape and workspace offsets, resident in device memory.
+struct DevDesc {
+    int32_t d_in;
+    int32_t d_out;
+    int32_t y_dtype;
+    int32_t max_m;
+    int64_t q_off;      // byte offset of this linear's int8 activations in the q workspace
+    int64_t st_off;     // index of its first TokStats record
+    int32_t blk_begin;  // first 64-row decode block of this linear in the flattened stack order
+    int32_t rt_begin;   // first 128-row prefill tile row of this linear in the same order
+};
+
+// Per-token values the main kernels need after quantisation.
+//   sx   : s_x = amax / 127 (fp32)
+//   sumq : sum_j q[t,j] (int32). The scaffold kernels count sum_{bit=1} q and
+//          form acc = 2 * that - sumq (exact integer identity for +-1 weights).
+//   u[k] : s_B[k] * h[t,k] in fp32 (the LoRA bottleneck, not re-quantised)
+struct alignas(16) TokStats {
+    float sx;
+    int32_t sumq;
+    int32_t pad0, pad1;
+    float u[kRank];
+};
+static_assert(sizeof(TokStats) == 80, "TokStats layout");
+static_assert(sizeof(dfssm_stack_entry) == 104, "dfssm_stack_entry layout");
+
+// Activation layout in the q workspace ("permuted int8"): rows of d_in bytes,
+// one per token; inside every 32-column group, byte position 4*p + i holds
+// column 8*i + p (p = 0..7, i = 0..3). With this order, the 4 bytes selected by
+// the mask 0x01010101 << p from one 32-bit word of sign bits line up with 4
+// consecutive q bytes, so bit expansion needs no shuffling.
+__host__ __device__ inline int perm_pos(int col) {
+    int g = col >> 5, c = col & 31;
+    int i = c >> 3, p = c & 7;
+    return (g << 5) | (p << 2) | i;
+}
+
+// ---- launch wrappers implemented in the .cu files ---------------------------------
+
+struct LaunchCtx {
+    const dfssm_stack_entry* entries;  // device array, or nullptr for `single`
+    dfssm_stack_entry single;          // used when entries == nullptr (n == 1)
+    int n;                             // number of linears
+    int m;                             // tokens per linear
+    const DevDesc* desc;               // device descriptor table (n entries, index = position)
+    const DevDesc* host_desc;          // host copy (same content)
+    int8_t* q_ws;
+    TokStats* st_ws;
+    uint32_t* err;
+    const void* tmaps;                 // device array of CUtensorMap (prefill), one per desc
+    int max_d_in;                      // largest d_in among the n linears
+    int64_t total_rows;                // sum of d_out over the n linears
+    int sm_count;
+    cudaStream_t stream;
+};
+
+cudaError_t launch_pack_sign(const void* src, int src_dtype, int d_out, int d_in, uint8_t* packed,
+                             cudaStream_t s);
+cudaError_t launch_quant(const LaunchCtx& c);
+cudaError_t launch_decode(const LaunchCtx& c);
+cudaError_t launch_prefill(const LaunchCtx& c);
+
+// ---- small device helpers -----------------------------------------------------------
+
+__device__ __forceinline__ const dfssm_stack_entry& entry_at(const dfssm_stack_entry* entries,
+                                                            const dfssm_stack_entry& single, int i) {
+    return entries ? entries[i] : single;
+}
+
+__device__ __forceinline__ bool ptr_ok(const void* p) {
+    return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+__device__ __forceinline__ bool opt_ptr_ok(const void* p) {
+    return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+// Every pointer of an entry is non-NULL (debug ones may be NULL) and 16-byte aligned.
+// Entries of a stack call live in device memory, so the host cannot check them.
+__device__ __forceinline__ bool entry_ptrs_ok(const dfssm_stack_entry& e) {
+    return ptr_ok(e.w.sign) && ptr_ok(e.w.alpha) && ptr_ok(e.w.wa) && ptr_ok(e.w.sa) && ptr_ok(e.w.wb) &&
+           ptr_ok(e.w.sb) && ptr_ok(e.x) && ptr_ok(e.y) && opt_ptr_ok(e.dbg.q) && opt_ptr_ok(e.dbg.sx) &&
+           opt_ptr_ok(e.dbg.acc) && opt_ptr_ok(e.dbg.h);
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t b16) {
+    return __uint_as_float(b16 << 16);
+}
+
+}  // namespace dfssm

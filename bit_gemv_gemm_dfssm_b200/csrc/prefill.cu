@@ -1,0 +1,335 @@
+// Prefill path (many tokens): the scaffold contraction as a dense int8 GEMM on
+// the 5th-generation tensor cores (tcgen05, accumulators in TMEM), with the
+// LoRA up-projection and both dequantisation epilogues fused.
+//
+// "Density Field State Space Models" (gist.science technical summary), §2.C:
+// packed 1-bit scaffold weights are expanded on the fly to int8 and multiplied
+// on INT8 tensor cores. With many tokens the contraction is a dense GEMM
+// (2 * d_in ops per token per output row), so here the expansion happens in
+// shared memory, once per 128-row x 128-column weight block, and the block is
+// reused by 256 tokens:
+//
+//   D[o, t] = sum_k b[o, k] * q[t, k]    (b = sign bit as 0/1, int32 in TMEM)
+//   acc     = 2 * D - sum_k q[t, k]       (a +-1 weight is 2b - 1)
+//
+// Persistent kernel, one CTA per SM, 12 warps with fixed roles:
+//   warp 0      TMA producer: 256-token x 128-byte tiles of the int8
+//               activations (permuted column order, 128B swizzle), no multicast
+//   warp 1      TMEM owner and MMA issuer: tcgen05.mma.kind::i8, M=128 rows,
+//               N=256 tokens, K=32 per instruction, 4 per 128-column block
+//   warps 4-7   bit expansion: each thread owns one weight row of the tile,
+//               loads 16 bytes of sign bits per k-block and writes 128 0/1 bytes
+//               into the K-major SWIZZLE_128B layout the MMA reads
+//   warps 8-11  epilogue: tcgen05.ld of its 32 TMEM lanes (= output rows),
+//               acc = 2D - sum q, LoRA up-projection and dequantisation,
+//               coalesced stores of y along the output dimension
+// 4-stage shared-memory ring (mbarriers), two TMEM accumulator buffers of 256
+// columns so the epilogue of one tile overlaps the main loop of the next.
+// Every mbarrier wait is bounded; a timeout sets the plan's error word.
+#include <cuda.h>
+
+#include "dfssm_internal.cuh"
+#include "ptx.cuh"
+
+namespace dfssm {
+
+namespace {
+
+constexpr int BM = 128;            // output rows per tile (MMA M, TMEM lanes)
+constexpr int BN = 256;            // tokens per tile (MMA N, TMEM columns)
+constexpr int BK = 128;            // k (bytes) per stage
+constexpr int STAGES = 4;
+constexpr int A_STAGE = BM * BK;   // 16 KB
+constexpr int B_STAGE = BN * BK;   // 32 KB
+constexpr int NUM_THREADS = 12 * 32;
+constexpr int SMEM_BYTES = STAGES * (A_STAGE + B_STAGE) + 256 + 1024;
+constexpr uint32_t TMEM_COLS = 512;
+
+struct PrefillArgs {
+    const dfssm_stack_entry* entries;
+    dfssm_stack_entry single;
+    const DevDesc* desc;          // desc[0] is the first linear of this launch
+    const CUtensorMap* tmaps;     // tmaps[l] maps linear l's q rows (same indexing as desc)
+    int n;
+    int m;
+    int n_tiles;
+    const TokStats* st_ws;
+    uint32_t* err;
+};
+
+// K-major, 128-byte swizzle shared-memory matrix descriptor: 8-row x 128-byte
+// atoms stacked every 1024 bytes (SBO), leading offset 1 (unused for this
+// layout), descriptor version 1, layout type 2 (SWIZZLE_128B).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// kind::i8 instruction descriptor: D s32, A s8, B s8, both K-major, N = BN, M = BM.
+constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                            ((uint32_t)(BM >> 4) << 24);
+
+struct TileCoord {
+    int lin, row0, tok0;
+};
+
+__device__ __forceinline__ TileCoord tile_coord(const DevDesc* desc, int n, int n_tt, int tile) {
+    const int rt = tile / n_tt;                 // global 128-row tile index
+    const int tt = tile - rt * n_tt;
+    const int base = desc[0].rt_begin;
+    int lo = 0, hi = n - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (desc[mid].rt_begin - base <= rt) lo = mid; else hi = mid - 1;
+    }
+    TileCoord c;
+    c.lin = lo;
+    c.row0 = (rt - (desc[lo].rt_begin - base)) * BM;
+    c.tok0 = tt * BN;
+    return c;
+}
+
+__device__ __forceinline__ void set_err(uint32_t* err, uint32_t bit) { atomicOr(err, bit); }
+
+__global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_constant__ PrefillArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + STAGES * A_STAGE;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE);
+    uint64_t* full_a = bars;               // [STAGES], 128 arrivals (expansion threads)
+    uint64_t* full_b = bars + STAGES;      // [STAGES], TMA transaction bytes
+    uint64_t* empty = bars + 2 * STAGES;   // [STAGES], MMA commit
+    uint64_t* acc_full = bars + 3 * STAGES;       // [2], MMA commit
+    uint64_t* acc_empty = bars + 3 * STAGES + 2;  // [2], 128 epilogue arrivals
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 4);
+    volatile uint32_t* abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_tt = (a.m + BN - 1) / BN;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            ptx::mbar_init(&full_a[s], 128);
+            ptx::mbar_init(&full_b[s], 1);
+            ptx::mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(&acc_full[b], 1);
+            ptx::mbar_init(&acc_empty[b], 128);
+        }
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (activations)
+        if (lane == 0) {
+            ptx::pdl_wait();
+            int it = 0;
+            for (int tile = blockIdx.x; tile < a.n_tiles && !*abort_flag; tile += gridDim.x) {
+                const TileCoord tc = tile_coord(a.desc, a.n, n_tt, tile);
+                const CUtensorMap* tm = a.tmaps + tc.lin;
+                const int nkb = a.desc[tc.lin].d_in / BK;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+                    if (!ptx::mbar_wait(&empty[s], ph ^ 1u)) { set_err(a.err, DFSSM_DEVERR_TIMEOUT); *abort_flag = 1; break; }
+                    ptx::mbar_arrive_expect_tx(&full_b[s], B_STAGE);
+                    ptx::tma_load_2d(sB + s * B_STAGE, tm, kb * BK, tc.tok0, &full_b[s]);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int it = 0, tcount = 0;
+            for (int tile = blockIdx.x; tile < a.n_tiles && !*abort_flag; tile += gridDim.x, ++tcount) {
+                const TileCoord tc = tile_coord(a.desc, a.n, n_tt, tile);
+                const int nkb = a.desc[tc.lin].d_in / BK;
+                const int buf = tcount & 1;
+                const uint32_t acc_ph = (uint32_t)(tcount >> 1) & 1u;
+                if (!ptx::mbar_wait(&acc_empty[buf], acc_ph ^ 1u)) { set_err(a.err, DFSSM_DEVERR_TIMEOUT); *abort_flag = 1; break; }
+                ptx::tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
+                bool ok = true;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+                    if (!ptx::mbar_wait(&full_a[s], ph) || !ptx::mbar_wait(&full_b[s], ph)) {
+                        set_err(a.err, DFSSM_DEVERR_TIMEOUT); *abort_flag = 1; ok = false; break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint64_t adesc = sw128_desc(ptx::smem_u32(sA + s * A_STAGE));
+                    const uint64_t bdesc = sw128_desc(ptx::smem_u32(sB + s * B_STAGE));
+#pragma unroll
+                    for (int kk = 0; kk < BK / 32; ++kk)   // +32 bytes along K = +2 in the 16-byte address field
+                        ptx::mma_i8(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, kIdesc, (kb | kk) != 0);
+                    ptx::mma_commit(&empty[s]);
+                }
+                if (!ok) break;
+                ptx::mma_commit(&acc_full[buf]);
+            }
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------ bit expansion (one weight row per thread)
+        const int r = threadIdx.x - 128;
+        int it = 0;
+        for (int tile = blockIdx.x; tile < a.n_tiles && !*abort_flag; tile += gridDim.x) {
+            const TileCoord tc = tile_coord(a.desc, a.n, n_tt, tile);
+            const DevDesc d = a.desc[tc.lin];
+            const dfssm_stack_entry& e = entry_at(a.entries, a.single, tc.lin);
+            const int nkb = d.d_in / BK;
+            const int o = tc.row0 + r;
+            const bool valid = o < d.d_out && entry_ptrs_ok(e);
+            const uint4* src = reinterpret_cast<const uint4*>(e.w.sign + (int64_t)(valid ? o : 0) * (d.d_in >> 3));
+            // rolling prefetch of the next 4 k-blocks of this row's bits
+            uint4 pf[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                pf[u] = (valid && u < nkb) ? __ldg(src + u) : make_uint4(0, 0, 0, 0);
+            // swizzled destination of this row: atom (r/8), row-in-atom (r%8)
+            const uint32_t rrow = (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u;
+            const uint32_t xr = (uint32_t)(r & 7);
+            bool ok = true;
+            for (int kb0 = 0; kb0 < nkb && ok; kb0 += 4) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int kb = kb0 + u;
+                    if (kb >= nkb) break;
+                    const uint4 bits = pf[u];
+                    pf[u] = (valid && kb + 4 < nkb) ? __ldg(src + kb + 4) : make_uint4(0, 0, 0, 0);
+                    const int s = it % STAGES;
+                    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+                    ++it;
+                    if (!ptx::mbar_wait(&empty[s], ph ^ 1u)) { set_err(a.err, DFSSM_DEVERR_TIMEOUT); *abort_flag = 1; ok = false; break; }
+                    uint8_t* dst = sA + s * A_STAGE + rrow;
+                    const uint32_t wv[4] = {bits.x, bits.y, bits.z, bits.w};
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        uint32_t e4[8];
+#pragma unroll
+                        for (int p = 0; p < 8; ++p) e4[p] = (wv[w] >> p) & 0x01010101u;
+                        const uint32_t c0 = (uint32_t)(2 * w), c1 = c0 + 1;
+                        *reinterpret_cast<uint4*>(dst + ((c0 ^ xr) << 4)) = make_uint4(e4[0], e4[1], e4[2], e4[3]);
+                        *reinterpret_cast<uint4*>(dst + ((c1 ^ xr) << 4)) = make_uint4(e4[4], e4[5], e4[6], e4[7]);
+                    }
+                    ptx::fence_proxy_async_smem();
+                    ptx::mbar_arrive(&full_a[s]);
+                }
+            }
+            if (!ok) break;
+        }
+    } else if (warp >= 8) {
+        // ------------------------------------------------ epilogue (TMEM lanes 32*(warp%4) ..)
+        ptx::pdl_wait();
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;
+        int tcount = 0;
+        for (int tile = blockIdx.x; tile < a.n_tiles && !*abort_flag; tile += gridDim.x, ++tcount) {
+            const TileCoord tc = tile_coord(a.desc, a.n, n_tt, tile);
+            const DevDesc d = a.desc[tc.lin];
+            const dfssm_stack_entry& e = entry_at(a.entries, a.single, tc.lin);
+            const int o = tc.row0 + r;
+            const bool valid = o < d.d_out && entry_ptrs_ok(e);
+            float alpha = 0.f, sa = 0.f, wa[kRank];
+            if (valid) {
+                alpha = e.w.alpha[o];
+                sa = e.w.sa[o];
+                const int4 w4 = *reinterpret_cast<const int4*>(e.w.wa + (int64_t)o * kRank);
+                const int8_t* wb = reinterpret_cast<const int8_t*>(&w4);
+#pragma unroll
+                for (int k = 0; k < kRank; ++k) wa[k] = (float)wb[k];
+            } else {
+#pragma unroll
+                for (int k = 0; k < kRank; ++k) wa[k] = 0.f;
+            }
+            const int buf = tcount & 1;
+            const uint32_t acc_ph = (uint32_t)(tcount >> 1) & 1u;
+            const bool got = __all_sync(0xffffffffu, ptx::mbar_wait(&acc_full[buf], acc_ph));
+            if (!got) {
+                if (lane == 0) { set_err(a.err, DFSSM_DEVERR_TIMEOUT); *abort_flag = 1; }
+                break;
+            }
+            ptx::tc_fence_after();
+            const TokStats* st = a.st_ws + d.st_off;
+            const uint32_t taddr = tmem_base + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(buf * BN);
+            for (int cb = 0; cb < BN; cb += 16) {
+                uint32_t v[16];
+                ptx::tmem_ld_32x32b_x16(taddr + (uint32_t)cb, v);
+                ptx::tmem_ld_wait();
+                if (tc.tok0 + cb >= a.m) continue;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int t = tc.tok0 + cb + j;
+                    if (t >= a.m) break;
+                    const TokStats& s = st[t];
+                    const int acc = 2 * (int)v[j] - s.sumq;
+                    float dot = 0.0f;
+#pragma unroll
+                    for (int k = 0; k < kRank; ++k) dot = __fmaf_rn(wa[k], s.u[k], dot);
+                    const float y = __fmul_rn(s.sx, __fmaf_rn(alpha, (float)acc, __fmul_rn(sa, dot)));
+                    if (valid) {
+                        const int64_t idx = (int64_t)t * d.d_out + o;
+                        if (d.y_dtype == DFSSM_BF16)
+                            reinterpret_cast<__nv_bfloat16*>(e.y)[idx] = __float2bfloat16_rn(y);
+                        else
+                            reinterpret_cast<float*>(e.y)[idx] = y;
+                        if (e.dbg.acc) e.dbg.acc[idx] = acc;
+                    }
+                }
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&acc_empty[buf]);
+        }
+    }
+
+    // ------------------------------------------------ teardown
+    __syncwarp();
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const LaunchCtx& c) {
+    int row_tiles = 0;
+    for (int i = 0; i < c.n; ++i) row_tiles += (c.host_desc[i].d_out + BM - 1) / BM;
+    const int n_tt = (c.m + BN - 1) / BN;
+    PrefillArgs a{c.entries, c.single, c.desc, reinterpret_cast<const CUtensorMap*>(c.tmaps), c.n, c.m,
+                  row_tiles * n_tt, c.st_ws, c.err};
+    const int grid = c.sm_count < a.n_tiles ? c.sm_count : a.n_tiles;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = c.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, prefill_kernel, a);
+}
+
+void set_prefill_attr(int max_dyn_smem) {
+    cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         max_dyn_smem < SMEM_BYTES ? max_dyn_smem : SMEM_BYTES);
+}
+
+int prefill_box_tokens() { return BN; }
+int prefill_box_bytes() { return BK; }
+
+}  // namespace dfssm

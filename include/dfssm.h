@@ -1,0 +1,176 @@
+/*
+ * dfssm.h - C ABI of libdfssm: the DF-SSM 1-bit scaffold + int8 LoRA linear on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer ("Density Field State Space Models", gist.science technical
+ * summary, §2.B "frozen scaffold with LoRA correction" and §2.C "optimised
+ * inference pipeline"; arXiv 2606.10932 abstract): every Mamba-2 in_proj and
+ * out_proj is a frozen 1-bit sign matrix plus a rank-16 int8 LoRA correction,
+ * applied to int8-quantised activations. For token t and output row o:
+ *
+ *   q, s_x   : per-token symmetric absmax int8 quantisation of x (below)
+ *   acc[t,o] = sum_j w[o,j] * q[t,j]        w[o,j] in {-1,+1}, int32
+ *   h[t,k]   = sum_j W_B[k,j] * q[t,j]      k < 16, int32
+ *   y[t,o]   = s_x[t] * ( alpha[o] * acc[t,o]
+ *                         + s_A[o] * sum_k W_A[o,k] * (s_B[k] * h[t,k]) )
+ *
+ * Conventions the pages leave open, fixed here (and identical in the oracle):
+ *   - sign bits: row-major, d_in/8 bytes per output row, no padding; column j
+ *     of row o is bit (j % 8) of byte o*(d_in/8) + j/8 (LSB first);
+ *     bit 1 -> +1, bit 0 -> -1.
+ *   - quantiser, in IEEE fp32 with round-to-nearest: amax = max_j |x[t,j]|;
+ *     amax == 0 -> q = 0, s_x = 0; otherwise inv = 127/amax,
+ *     q = clamp(round_half_even(x * inv), -127, 127), s_x = amax/127.
+ *   - alpha, s_A: one fp32 per output row; s_B: one fp32 per LoRA row.
+ *   - s_x multiplies both terms; s_B * h stays in fp32 (not re-quantised).
+ *
+ * Memory: every tensor pointer is a DEVICE pointer owned by the caller; the
+ * library never frees it. Tensor pointers must be 16-byte aligned. A plan owns
+ * its workspace (device memory allocated by dfssm_linear_plan, freed by
+ * dfssm_plan_destroy) and is tied to the device current at plan time.
+ *
+ * Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ * stream). Calls only enqueue work; they never synchronise, except
+ * dfssm_plan_check. Caller buffers must stay valid until the stream has run
+ * the work. x and y must not overlap. A plan's workspace is reused by every
+ * call, so calls on one plan must be ordered (same stream, or synchronised);
+ * a plan is not thread-safe.
+ *
+ * Errors: argument errors are returned synchronously and nothing is enqueued.
+ * A failed launch returns DFSSM_ERR_CUDA. Conditions only the device can see
+ * (a stack entry whose desc_index does not match its position or whose
+ * pointers are NULL or misaligned, a non-finite amax, a bounded wait that gave
+ * up) set the plan's device error word instead of trapping; read it with
+ * dfssm_plan_check.
+ */
+#ifndef DFSSM_H
+#define DFSSM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DFSSM_OK = 0,
+    DFSSM_ERR_INVALID_ARG = 1,       /* NULL / misaligned pointer, bad enum, m out of range */
+    DFSSM_ERR_UNSUPPORTED_SHAPE = 2, /* d_in % 128 != 0, d_in > 8192, rank != 16, ... */
+    DFSSM_ERR_CUDA = 3,              /* a CUDA runtime call or launch failed */
+    DFSSM_ERR_NO_MEMORY = 4,         /* workspace allocation failed */
+    DFSSM_ERR_DEVICE_CHECK = 5       /* the device error word was set (dfssm_plan_check) */
+} dfssm_status;
+
+typedef enum { DFSSM_BF16 = 0, DFSSM_F32 = 1, DFSSM_I8 = 2 } dfssm_dtype;
+
+/* Device error word bits (dfssm_plan_check). */
+#define DFSSM_DEVERR_ENTRY_DESC 0x1u   /* stack entry i has desc_index != i */
+#define DFSSM_DEVERR_NONFINITE  0x2u   /* a token's amax was Inf or NaN (output undefined) */
+#define DFSSM_DEVERR_TIMEOUT    0x4u   /* a bounded in-kernel wait gave up (output undefined) */
+#define DFSSM_DEVERR_ENTRY_PTR  0x8u   /* a stack entry holds a NULL or misaligned pointer (entry skipped) */
+
+/* Shape of one linear. d_in % 128 == 0, 128 <= d_in <= 8192; 1 <= d_out <= 2^20;
+ * rank == 16; 1 <= max_m <= 65536; y_dtype DFSSM_BF16 or DFSSM_F32; flags = 0. */
+typedef struct {
+    int32_t d_in;
+    int32_t d_out;
+    int32_t rank;
+    int32_t max_m;
+    int32_t y_dtype;
+    uint32_t flags;
+} dfssm_linear_desc;
+
+/* Weights of one linear (device pointers, caller-owned, 16-byte aligned).
+ *   sign  : d_out x (d_in/8) bytes, packed as above (see dfssm_pack_sign)
+ *   alpha : d_out fp32 scaffold scale per output row
+ *   wa    : d_out x 16 int8, row-major (LoRA up-projection W_A)
+ *   sa    : d_out fp32 (per-row scale of W_A)
+ *   wb    : 16 x d_in int8, row-major (LoRA down-projection W_B)
+ *   sb    : 16 fp32 (per-row scale of W_B)
+ * ("Density Field State Space Models", technical summary §2.B: W_A in
+ * R^{d_out x r}, W_B in R^{r x d_in}, r = 16, int8 with per-channel/row scales.) */
+typedef struct {
+    const uint8_t* sign;
+    const float* alpha;
+    const int8_t* wa;
+    const float* sa;
+    const int8_t* wb;
+    const float* sb;
+} dfssm_linear_weights;
+
+/* Optional exports for bit-exact checks (device pointers; any may be NULL):
+ *   q   : m x d_in int8 (natural column order), sx : m fp32,
+ *   acc : m x d_out int32 (scaffold sums), h : m x 16 int32 (LoRA down sums). */
+typedef struct {
+    int8_t* q;
+    float* sx;
+    int32_t* acc;
+    int32_t* h;
+} dfssm_debug;
+
+/* One linear of a stack (this struct lives in DEVICE memory for
+ * dfssm_linear_stack_fwd). x: m x d_in bf16 row-major; y: m x d_out of the
+ * desc's y_dtype, row-major. desc_index must equal the entry's position. */
+typedef struct {
+    dfssm_linear_weights w;
+    const void* x;
+    void* y;
+    dfssm_debug dbg;
+    int32_t desc_index;
+    int32_t reserved;
+} dfssm_stack_entry;
+
+typedef struct dfssm_plan_s* dfssm_plan;
+
+/* Create a plan for n_descs linears on the current device. For a stack, desc i
+ * describes stack entry i (48 Mamba-2 layers = 96 descs: in_proj, out_proj,
+ * ...). Allocates the workspace (int8 activations and per-token scales for
+ * max_m tokens per linear, the prefill tensor maps and the error word).
+ * On success *out receives the plan; on failure *out is NULL and nothing is
+ * left allocated. */
+dfssm_status dfssm_linear_plan(const dfssm_linear_desc* descs, int n_descs, dfssm_plan* out);
+
+/* Free a plan and its workspace. Waits for the device to finish using it
+ * (device synchronise). NULL is accepted. */
+dfssm_status dfssm_plan_destroy(dfssm_plan plan);
+
+/* Pack a frozen scaffold into sign bits (technical summary §2.B: the scaffold
+ * is frozen at its rounded values; §2.C / §3: stored at 1 bit per weight).
+ * src: d_out x d_in device tensor, row-major, of src_dtype DFSSM_I8 or
+ * DFSSM_F32; value >= 0 (including -0.0) -> +1 -> bit 1, value < 0 -> bit 0.
+ * A NaN in an fp32 source is outside the contract (its bit is unspecified).
+ * packed: d_out x d_in/8 bytes, device. d_in % 128 == 0. */
+dfssm_status dfssm_pack_sign(const void* src, int32_t src_dtype, int32_t d_out, int32_t d_in,
+                             uint8_t* packed, void* stream);
+
+/* y = layer(x) for one linear (the formula at the top of this file).
+ * desc_index selects the shape; w is a HOST struct of device pointers;
+ * x: m x d_in bf16 (device); y: m x d_out of the desc's y_dtype (device);
+ * 1 <= m <= max_m. dbg may be NULL. */
+dfssm_status dfssm_linear_fwd(dfssm_plan plan, int32_t desc_index, const dfssm_linear_weights* w,
+                              const void* x, int32_t m, void* y, const dfssm_debug* dbg,
+                              void* stream);
+
+/* The layer for n_entries independent linears, in one pass (the pages capture
+ * the whole 48-layer forward as one CUDA graph, technical summary §2.C).
+ * entries_dev: DEVICE array of n_entries dfssm_stack_entry, entry i planned by
+ * desc i; 1 <= n_entries <= n_descs; every entry uses the same m. */
+dfssm_status dfssm_linear_stack_fwd(dfssm_plan plan, const dfssm_stack_entry* entries_dev,
+                                    int32_t n_entries, int32_t m, void* stream);
+
+/* Synchronise the plan's device, read and clear its error word.
+ * Returns DFSSM_OK or DFSSM_ERR_DEVICE_CHECK (*bits, if not NULL, gets the word). */
+dfssm_status dfssm_plan_check(dfssm_plan plan, uint32_t* bits);
+
+/* Bytes of device workspace the plan holds. */
+dfssm_status dfssm_plan_workspace_bytes(dfssm_plan plan, size_t* bytes);
+
+/* Static description of a status code. */
+const char* dfssm_status_string(dfssm_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DFSSM_H */
