@@ -342,6 +342,8 @@ def run_gpu(args, wl_name):
     peaks = load_peaks()
     wl = synth.WORKLOADS[wl_name]
     shapes, m, cfg = wl["shapes"], wl["m"], wl["cfg"]
+    if args.layers:
+        shapes = shapes[:2 * args.layers]
     seed = replica_seed(rank)
 
     r = StackRunner(shapes, m, cfg, seed)
@@ -370,10 +372,12 @@ def run_gpu(args, wl_name):
         r.call(i % 2, stream.cuda_stream)
         r.y_host.copy_(r.y.view(torch.int16), non_blocking=True)
 
-    e2e_ms = timed_device(torch, e2e_step, args.steps, args.warmup, dist, dev)
-    e2e_gbs = sum_over_ranks(float(nb * args.steps), dist, dev) / (e2e_ms * 1e-3) / 1e9
-    h2d = r.x_elems * 2
-    d2h = r.y_elems * 2
+    e2e = None
+    if not args.no_e2e:
+        e2e_ms = timed_device(torch, e2e_step, args.steps, args.warmup, dist, dev)
+        e2e = {"value": sum_over_ranks(float(nb * args.steps), dist, dev) / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "ms_per_step": e2e_ms / args.steps, "h2d_bytes_per_step": r.x_elems * 2,
+               "d2h_bytes_per_step": r.y_elems * 2}
     r.check()
     r.close()
     del graphs
@@ -382,13 +386,14 @@ def run_gpu(args, wl_name):
     prefill = None
     if not args.no_prefill:
         pwl = synth.WORKLOADS["stack48_m2048"]
-        pr = StackRunner(pwl["shapes"], pwl["m"], pwl["cfg"], seed)
+        pshapes = pwl["shapes"][:2 * args.layers] if args.layers else pwl["shapes"]
+        pr = StackRunner(pshapes, pwl["m"], pwl["cfg"], seed)
         psteps = args.prefill_steps
         pgraphs = pr.graphs()
         with ClockSampler(local) as pclk:
             pms = timed_device(torch, lambda i: pgraphs[i % 2].replay(), psteps, max(3, args.warmup // 10), dist, dev)
         pr.check()
-        pops = stack_ops(pwl["shapes"], pwl["m"])
+        pops = stack_ops(pshapes, pwl["m"])
         tops = sum_over_ranks(float(pops * psteps), dist, dev) / (pms * 1e-3) / 1e12
         peak_i8 = peaks["bf16"] * INT8_PER_BF16
         ach = pops / (pms / psteps * 1e-3) / 1e12
@@ -421,7 +426,8 @@ def run_gpu(args, wl_name):
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8 x 1-bit -> int32, fp32 epilogue, bf16 out",
         "data": "synthetic (seeded; Mamba-2-1.3B shapes, random weights)",
-        "config": {"workload": wl_name, "m": m, "linears": len(shapes), "layers": len(shapes) // 2,
+        "config": {"workload": wl_name if not args.layers else f"{wl_name} (first {args.layers} layers)",
+                   "m": m, "linears": len(shapes), "layers": len(shapes) // 2,
                    "d_model": 2048, "rank": 16, "parallelism": f"replicas x{ws}",
                    "l2": "two weight sets alternated per step (2 x 171.8 MB > 126 MB L2)",
                    "bytes_per_step": nb, "graph": "one CUDA graph per step"},
@@ -431,8 +437,7 @@ def run_gpu(args, wl_name):
                      "frac": achieved / peaks["hbm"], "traffic": recorded_traffic(wl_name),
                      "peak_source": f"{peaks['src']} copy bandwidth",
                      "timed": "quant_kernel + decode_kernel per call (PDL-overlapped)"},
-        "e2e": {"value": e2e_gbs, "unit": "GB/s", "ms_per_step": e2e_ms / args.steps,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": e2e,
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
         "cpu_baseline": cpu,
@@ -454,6 +459,9 @@ def main(argv=None):
     ap.add_argument("--prefill-steps", type=int, default=30)
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="use only the first L layers of the stack (small cases for profiling)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

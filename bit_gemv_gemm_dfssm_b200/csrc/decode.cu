@@ -4,270 +4,483 @@
 // "Density Field State Space Models" (gist.science technical summary), §2.C:
 // the 1-bit scaffold weights are expanded on the fly to int8 and fed to int8
 // tensor cores, which cuts weight traffic 8x against int8 weights; at batch 1
-// the layer is bound by that weight stream. Here the bits never leave
-// registers as bytes in memory:
+// the layer is bound by that weight stream. Here the bits never exist as int8
+// bytes in memory:
 //
-//  * A CTA owns 64 output rows of one linear. Its rows are brought into shared
-//    memory by the TMA bulk-copy engine (one cp.async.bulk per row, padded row
-//    stride so the fragment reads below are bank-conflict free), completion
-//    tracked by one mbarrier. No multicast.
+//  * Work: blocks of R = 64 * RT output rows (4 warps, RT 16-row tiles per
+//    warp), flattened over all linears of the call. Each CTA is persistent and
+//    owns a contiguous range of blocks holding an equal share of the sign bytes.
+//  * Streaming: a block is consumed in k-chunks of 1024 columns (128 bytes per
+//    row). A ring of kStages shared-memory slots is filled with 16-byte
+//    cp.async; in slot row r, 16-byte chunk j sits at (j + r) mod 8, so the
+//    ldmatrix reads of 8 rows hit 8 different bank groups. The last k-chunk of
+//    a block also brings its alpha, s_A and W_A.
+//  * Activations: when a CTA reaches a new linear it quantises that linear's
+//    x itself (same fp32 arithmetic as the quantisation kernel, so the same
+//    bits) into shared memory, while its weight chunks are already in flight.
+//    Only the LoRA vector u = s_B * h comes from the quantisation kernel, and
+//    the CTA waits for that kernel (programmatic dependent launch) just before
+//    its first epilogue.
 //  * Expansion: for a 32-bit word of sign bits w and bit position p,
-//    w & (0x01010101 << p) is four bytes that are each 0 or 2^p: the bits of
-//    columns 8i + p (i = 0..3) scaled by 2^p. One LOP3 expands four weights.
-//  * These bytes are the u8 A operand of the legacy warp MMA
-//    m16n8k32 (u8 x s8 -> s32); the int8 activations, stored in the matching
-//    permuted column order (byte 4p + i of a 32-column group = column 8i + p),
-//    are the s8 B operand, with the tokens as the N = 8 columns.
-//  * One accumulator set per bit position p, so each sums 2^p * S_p exactly;
+//    w & (0x01010101 << p) is four bytes, each 0 or 2^p: the bits of columns
+//    8i + p (i = 0..3) scaled by 2^p. One LOP3 expands four weights.
+//  * These bytes are the u8 A operand of the warp MMA m16n8k32 (u8 x s8 -> s32),
+//    loaded with ldmatrix.x4 straight from the staged bits; the int8
+//    activations in the matching permuted column order (byte 4p + i of a
+//    32-column group = column 8i + p) are the s8 B operand, tokens = N.
+//  * One accumulator set per p, so set p sums 2^p * S_p exactly;
 //    S1 = sum_p D_p / 2^p = sum_{bit = 1} q, and acc = 2 * S1 - sum_j q
 //    (a +-1 weight is 2b - 1).
-//  * Epilogue per (token t, row o), in fp32 in this fixed order:
-//      dot = sum_{k=0..15} W_A[o,k] * u[t,k]   (fmaf, k ascending)
-//      y   = s_x[t] * fmaf(alpha[o], acc, s_A[o] * dot)
-//    the same order as the prefill path, so the two paths agree bit for bit.
-//
-// The kernel is launched with programmatic dependent launch: it issues its
-// weight copies first and only then waits for the quantisation kernel that
-// produces q, s_x, sum q and u.
+//  * Epilogue (epilogue.cuh): lane i of a warp takes output row i, gathers its
+//    sums with warp shuffles, and applies the LoRA up-projection and the
+//    dequantisation in the same fp32 order as the prefill path.
 #include "dfssm_internal.cuh"
+#include "epilogue.cuh"
 #include "ptx.cuh"
 
 namespace dfssm {
 
 namespace {
 
-constexpr int kRowsPerCta = 64;
 constexpr int kWarps = 4;
-constexpr int kRowPad = 32;      // bytes added to each staged sign row
-constexpr int kTokPad = 64;      // bytes added to each staged q row
+constexpr int kThreads = kWarps * 32;
+constexpr int kChunkBytes = 128;   // sign bytes per row per k-chunk (1024 columns)
+constexpr int kTokPad = 16;        // q row stride = d_in + 16 (= 16 mod 128: conflict-free B reads)
+constexpr int kStages = 3;
+constexpr int kMaxTok = 16;
 
 struct DecodeArgs {
     const dfssm_stack_entry* entries;
     dfssm_stack_entry single;
-    const DevDesc* desc;   // desc[0] is the first linear of this launch
+    const DevDesc* desc;     // desc[0] is the first linear of this launch
     int n;
     int m;
-    const int8_t* q_ws;
     const TokStats* st_ws;
-    uint32_t* err;
+    int64_t total_bytes;     // sign bytes of the n linears
+    int slot_bytes;          // bytes of one ring slot
+    int q_region;            // bytes of the staged-q region
 };
 
-__device__ __forceinline__ int find_linear(const DevDesc* desc, int n, int blk) {
-    // largest l with desc[l].blk_begin - desc[0].blk_begin <= blk
-    const int base = desc[0].blk_begin;
-    int lo = 0, hi = n - 1;
-    while (lo < hi) {
-        int mid = (lo + hi + 1) >> 1;
-        if (desc[mid].blk_begin - base <= blk) lo = mid; else hi = mid - 1;
-    }
-    return lo;
+// Fields of one linear, cached in registers while a cursor is on it.
+struct Lin {
+    int d_in, d_out, rb, nchunks, nblocks, y_dtype;
+    int64_t byte_rel;        // first sign byte relative to desc[0]
+    int64_t st_off;
+    const uint8_t* sign;
+    const float* alpha;
+    const float* sa;
+    const int8_t* wa;
+    const uint16_t* x;
+    void* y;
+    int32_t* dbg_acc;
+    bool ok;                 // entry pointers valid
+};
+
+template <int R>
+__device__ __forceinline__ void load_lin(const DecodeArgs& a, int l, Lin& L) {
+    const DevDesc& d = a.desc[l];
+    const dfssm_stack_entry& e = entry_at(a.entries, a.single, l);
+    L.d_in = d.d_in;
+    L.d_out = d.d_out;
+    L.rb = d.d_in >> 3;
+    L.nchunks = (d.d_in + 1023) >> 10;
+    L.nblocks = (d.d_out + R - 1) / R;
+    L.y_dtype = d.y_dtype;
+    L.byte_rel = d.byte_begin - a.desc[0].byte_begin;
+    L.st_off = d.st_off;
+    L.sign = e.w.sign;
+    L.alpha = e.w.alpha;
+    L.sa = e.w.sa;
+    L.wa = e.w.wa;
+    L.x = reinterpret_cast<const uint16_t*>(e.x);
+    L.y = e.y;
+    L.dbg_acc = e.dbg.acc;
+    L.ok = entry_ptrs_ok(e);
 }
 
-template <int NT>
-__global__ void __launch_bounds__(kWarps * 32) decode_kernel(const DecodeArgs a) {
+struct Cursor {
+    int l, b, kc;   // linear, block within the linear, k-chunk within the block
+};
+
+template <int R>
+struct Walk {
+    Cursor c;
+    Lin L;
+    __device__ __forceinline__ bool valid(const DecodeArgs& a, int64_t hi) const {
+        return c.l < a.n && L.byte_rel + (int64_t)c.b * R * L.rb < hi;
+    }
+    __device__ __forceinline__ void advance(const DecodeArgs& a) {
+        if (++c.kc >= L.nchunks) {
+            c.kc = 0;
+            if (++c.b >= L.nblocks) {
+                c.b = 0;
+                if (++c.l < a.n) load_lin<R>(a, c.l, L);
+            }
+        }
+    }
+    // first block whose first sign byte is at or after `lo`
+    __device__ void start(const DecodeArgs& a, int64_t lo) {
+        const int64_t base = a.desc[0].byte_begin;
+        int lo_l = 0, hi_l = a.n - 1;
+        while (lo_l < hi_l) {
+            const int mid = (lo_l + hi_l + 1) >> 1;
+            if (a.desc[mid].byte_begin - base <= lo) lo_l = mid; else hi_l = mid - 1;
+        }
+        c = Cursor{lo_l, 0, 0};
+        load_lin<R>(a, c.l, L);
+        const int64_t bb = (int64_t)R * L.rb;
+        c.b = (int)((lo - L.byte_rel + bb - 1) / bb);
+        if (c.b >= L.nblocks) {
+            c.b = 0;
+            if (++c.l < a.n) load_lin<R>(a, c.l, L);
+        }
+    }
+};
+
+// Fill a ring slot with k-chunk kc of block b: R rows x (up to) 128 sign bytes,
+// plus alpha, s_A and W_A of the block when kc is its last chunk.
+template <int R>
+__device__ __forceinline__ void issue_step(const Cursor& c, const Lin& L, uint8_t* slot) {
+    if (!L.ok) return;                    // flagged by the quantisation kernel
+    const int row0 = c.b * R;
+    const int nrows = min(R, L.d_out - row0);
+    const int nch = min(kChunkBytes, L.rb - kChunkBytes * c.kc) >> 4;   // 1..8 16-byte chunks
+    const uint8_t* src = L.sign + (int64_t)row0 * L.rb + kChunkBytes * c.kc;
+    for (int ci = threadIdx.x; ci < nrows * 8; ci += kThreads) {
+        const int r = ci >> 3, j = ci & 7;
+        if (j < nch) ptx::cp_async16(slot + r * kChunkBytes + 16 * ((j + r) & 7), src + (int64_t)r * L.rb + 16 * j);
+    }
+    if (c.kc == L.nchunks - 1) {
+        uint8_t* par = slot + R * kChunkBytes;
+        const int n4 = (nrows + 3) >> 2;
+        for (int i = threadIdx.x; i < n4; i += kThreads) {
+            const uint32_t bytes = (uint32_t)min(16, 4 * (nrows - 4 * i));
+            ptx::cp_async16_zfill(par + 16 * i, L.alpha + row0 + 4 * i, bytes);
+            ptx::cp_async16_zfill(par + 4 * R + 16 * i, L.sa + row0 + 4 * i, bytes);
+        }
+        for (int r = threadIdx.x; r < nrows; r += kThreads)
+            ptx::cp_async16(par + 8 * R + 16 * r, L.wa + (int64_t)(row0 + r) * kRank);
+    }
+}
+
+struct TokShared {
+    float sx[kMaxTok];
+    int sumq[kMaxTok];
+    float red_f[kWarps][kMaxTok];
+    int red_i[kWarps][kMaxTok];
+    float u[kMaxTok][kRank];
+};
+
+// Quantise the m x d_in activations of linear L into the permuted int8 layout
+// (token stride d_in + kTokPad), with per-token s_x and sum q. Same arithmetic
+// as the quantisation kernel (epilogue.cuh), so the same bytes.
+__device__ void quantise_into_smem(const Lin& L, int m, uint8_t* q_s, TokShared& ts) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n8 = L.d_in >> 3;                      // 8-column chunks per row
+    const int qstride = L.d_in + kTokPad;
+    for (int t = 0; t < m; ++t) {
+        float am = 0.0f;
+        for (int ch = tid; ch < n8; ch += kThreads) {
+            const uint4 v = *reinterpret_cast<const uint4*>(L.x + (int64_t)t * L.d_in + 8 * ch);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) am = fmaxf(am, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+        if (lane == 0) ts.red_f[warp][t] = am;
+    }
+    __syncthreads();
+    for (int t = 0; t < m; ++t) {
+        float am = ts.red_f[0][t];
+#pragma unroll
+        for (int w = 1; w < kWarps; ++w) am = fmaxf(am, ts.red_f[w][t]);
+        const float inv = quant_inv(am);
+        const bool zero = am == 0.0f;
+        int sum = 0;
+        for (int ch = tid; ch < n8; ch += kThreads) {
+            const uint4 v = *reinterpret_cast<const uint4*>(L.x + (int64_t)t * L.d_in + 8 * ch);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            // columns 8 ch + p, p = 0..7 -> permuted byte 32 (ch / 4) + 4 p + ch % 4
+            uint8_t* dst = q_s + t * qstride + 32 * (ch >> 2) + (ch & 3);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int q0 = quant1(bf16_lo(w[i]), inv, zero), q1 = quant1(bf16_hi(w[i]), inv, zero);
+                sum += q0 + q1;
+                dst[4 * (2 * i)] = (uint8_t)q0;
+                dst[4 * (2 * i + 1)] = (uint8_t)q1;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (lane == 0) ts.red_i[warp][t] = sum;
+        if (tid == 0) ts.sx[t] = quant_sx(am);
+    }
+    __syncthreads();
+    if (tid < m) {
+        int s = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) s += ts.red_i[w][tid];
+        ts.sumq[tid] = s;
+    }
+    // (the caller synchronises before sumq is read)
+}
+
+template <int RT, int NT>
+__global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant__ DecodeArgs a) {
+    constexpr int R = 16 * RT * kWarps;
     extern __shared__ __align__(128) uint8_t smem[];
-    uint64_t* bar = reinterpret_cast<uint64_t*>(smem);
-    TokStats* st_s = reinterpret_cast<TokStats*>(smem + 16);
+    TokShared& ts = *reinterpret_cast<TokShared*>(smem);
+    uint8_t* q_s = smem + ((sizeof(TokShared) + 127) & ~(size_t)127);
+    uint8_t* ring = q_s + a.q_region;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, c = lane & 3;
-
-    const int lin = find_linear(a.desc, a.n, blockIdx.x);
-    const DevDesc d = a.desc[lin];
-    const dfssm_stack_entry& e = entry_at(a.entries, a.single, lin);
     const int m = a.m;
-    const int d_in = d.d_in;
-    const int rb = d_in >> 3;                      // sign bytes per row
-    const int wstride = rb + kRowPad;
-    const int qstride = d_in + kTokPad;
-    const int row0 = (blockIdx.x - (d.blk_begin - a.desc[0].blk_begin)) * kRowsPerCta;
-    const int nrows = min(kRowsPerCta, d.d_out - row0);
 
-    if (!entry_ptrs_ok(e)) return;     // flagged by the quantisation kernel
+    const int64_t lo = a.total_bytes * blockIdx.x / gridDim.x;
+    const int64_t hi = a.total_bytes * (blockIdx.x + 1) / gridDim.x;
+    Walk<R> cw, lw;
+    cw.start(a, lo);
+    lw = cw;
 
-    uint8_t* q_s = smem + 16 + ((m * (int)sizeof(TokStats) + 127) & ~127);
-    uint8_t* w_s = q_s + ((m * qstride + 127) & ~127);
-
-    if (tid == 0) {
-        ptx::mbar_init(bar, 1);
-        ptx::fence_mbar_init();
-    }
-    __syncthreads();
-
-    // ---- 1. weight rows: bulk copies, issued before waiting on the producer kernel
-    if (warp == 0) {
-        if (lane == 0) ptx::mbar_arrive_expect_tx(bar, (uint32_t)(nrows * rb));
-        __syncwarp();
-        const uint8_t* src = e.w.sign + (int64_t)row0 * rb;
-        for (int r = lane; r < nrows; r += 32)
-            ptx::bulk_g2s(w_s + r * wstride, src + (int64_t)r * rb, (uint32_t)rb, bar);
-    }
-
-    // epilogue parameters of this thread's two rows (independent of the producer)
-    const int oA = row0 + warp * 16 + g, oB = oA + 8;
-    float alphaA = 0.f, alphaB = 0.f, saA = 0.f, saB = 0.f;
-    int4 waA = make_int4(0, 0, 0, 0), waB = make_int4(0, 0, 0, 0);
-    if (oA < d.d_out) {
-        alphaA = e.w.alpha[oA]; saA = e.w.sa[oA];
-        waA = *reinterpret_cast<const int4*>(e.w.wa + (int64_t)oA * kRank);
-    }
-    if (oB < d.d_out) {
-        alphaB = e.w.alpha[oB]; saB = e.w.sa[oB];
-        waB = *reinterpret_cast<const int4*>(e.w.wa + (int64_t)oB * kRank);
-    }
-
-    // ---- 2. wait for q / stats, stage them
-    ptx::pdl_wait();
-    {
-        const uint4* src = reinterpret_cast<const uint4*>(a.st_ws + d.st_off);
-        uint4* dst = reinterpret_cast<uint4*>(st_s);
-        for (int i = tid; i < m * (int)(sizeof(TokStats) / 16); i += kWarps * 32) dst[i] = src[i];
-        // q rows, chunk (G, c', k) of a 64-byte block stored at slot (k + c') & 3
-        const int chunks = d_in >> 4;
-        for (int i = tid; i < m * chunks; i += kWarps * 32) {
-            const int t = i / chunks, s = i - t * chunks;
-            const int G = s >> 4, cc = (s >> 2) & 3, k = s & 3;
-            const uint4 v = *reinterpret_cast<const uint4*>(a.q_ws + d.q_off + (int64_t)t * d_in + 16 * s);
-            *reinterpret_cast<uint4*>(q_s + t * qstride + 256 * G + 64 * cc + 16 * ((k + cc) & 3)) = v;
+    // ---- prologue: kStages - 1 slots in flight
+#pragma unroll
+    for (int s = 0; s < kStages - 1; ++s) {
+        if (lw.valid(a, hi)) {
+            issue_step<R>(lw.c, lw.L, ring + s * a.slot_bytes);
+            lw.advance(a);
         }
-    }
-    __syncthreads();
-    if (a.entries != nullptr && e.desc_index != lin) {
-        if (tid == 0) atomicOr(a.err, DFSSM_DEVERR_ENTRY_DESC);
+        ptx::cp_async_commit();
     }
 
-    // ---- 3. wait for the weight rows
-    if (!ptx::mbar_wait(bar, 0)) {
-        if (lane == 0) atomicOr(a.err, DFSSM_DEVERR_TIMEOUT);
-        ptx::mbar_wait(bar, 0);   // second bounded wait for the copies still in flight
-        return;
-    }
+    int D[RT][NT][8][4];
+    int q_lin = -1, u_lin = -1;
+    // ldmatrix lane role: matrix (lane / 8) = (row half, 16-byte half of the 32-byte group)
+    const int lm_row = (lane & 7) + 8 * ((lane >> 3) & 1);
+    const int lm_hi = lane >> 4;
+    const int wrow0 = warp * 16 * RT;             // first row of this warp in a block
 
-    // ---- 4. main loop: 16 rows per warp, all of d_in
-    int D[NT][8][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int p = 0; p < 8; ++p)
-#pragma unroll
-            for (int r = 0; r < 4; ++r) D[nt][p][r] = 0;
+    for (int it = 0; cw.valid(a, hi); ++it) {
+        const Lin& L = cw.L;
+        if (cw.c.l != q_lin) {
+            // a new linear: quantise its activations (its weights are already streaming)
+            if (L.ok) quantise_into_smem(L, m, q_s, ts);
+            q_lin = cw.c.l;
+        }
+        if (lw.valid(a, hi)) {
+            issue_step<R>(lw.c, lw.L, ring + ((it + kStages - 1) % kStages) * a.slot_bytes);
+            lw.advance(a);
+        }
+        ptx::cp_async_commit();
+        ptx::cp_async_wait<kStages - 1>();
+        const bool last_chunk = cw.c.kc == L.nchunks - 1;
+        if (last_chunk && u_lin != cw.c.l) {
+            // the LoRA vector u = s_B * h of this linear, from the quantisation kernel
+            ptx::pdl_wait();
+            for (int i = tid; i < m * kRank; i += kThreads)
+                ts.u[i >> 4][i & 15] = a.st_ws[L.st_off + (i >> 4)].u[i & 15];
+            u_lin = cw.c.l;
+        }
+        __syncthreads();
 
-    const uint8_t* wrA = w_s + (warp * 16 + g) * wstride + 8 * c;
-    const uint8_t* wrB = wrA + 8 * wstride;
-    // groups of 256 columns; when d_in % 256 == 128 the last group is half full and
-    // only lanes with c < 2 (words 0..3 of the group) carry data
-    const int ngroups = (d_in + 255) >> 8;
-    const bool warp_active = warp * 16 < nrows;
-    if (warp_active) {
-        for (int G = 0; G < ngroups; ++G) {
-            const bool lane_has = (256 * G + 64 * c) < d_in;
-            const uint2 wa2 = lane_has ? *reinterpret_cast<const uint2*>(wrA + 32 * G) : make_uint2(0u, 0u);
-            const uint2 wb2 = lane_has ? *reinterpret_cast<const uint2*>(wrB + 32 * G) : make_uint2(0u, 0u);
-            uint32_t b[NT][4][4];
+        const uint8_t* slot = ring + (it % kStages) * a.slot_bytes;
+        const int row0 = cw.c.b * R;
+        const int nrows = min(R, L.d_out - row0);
+        const bool active = wrow0 < nrows && L.ok;
+        if (cw.c.kc == 0) {
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const int tk = nt * 8 + g;
-                if (tk < m && lane_has) {
-                    const uint8_t* qb = q_s + tk * qstride + 256 * G + 64 * c;
+            for (int rt = 0; rt < RT; ++rt)
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint4 v = *reinterpret_cast<const uint4*>(qb + 16 * ((k + c) & 3));
-                        b[nt][k][0] = v.x; b[nt][k][1] = v.y; b[nt][k][2] = v.z; b[nt][k][3] = v.w;
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int p = 0; p < 8; ++p)
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) D[rt][nt][p][r] = 0;
+        }
+        if (active) {
+            const int qstride = L.d_in + kTokPad;
+            const int cb = min(kChunkBytes, L.rb - kChunkBytes * cw.c.kc);
+            const int ng = (cb + 31) >> 5;                 // groups of 256 columns in this chunk
+            const uint32_t slot_s = ptx::smem_u32(slot);
+            const uint8_t* qrow[NT];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                qrow[nt] = q_s + (nt * 8 + g) * qstride + 32 * (32 * cw.c.kc + c);
+#pragma unroll
+            for (int G = 0; G < 4; ++G) {
+                if (G < ng) {
+                    const bool half = (cb - 32 * G) == 16;     // only 128 columns: words 4..7 absent
+                    uint32_t A[RT][4];
+#pragma unroll
+                    for (int rt = 0; rt < RT; ++rt) {
+                        const int row = wrow0 + 16 * rt + lm_row;
+                        const int chunk = 2 * G + lm_hi;
+                        ptx::ldmatrix_x4(slot_s + row * kChunkBytes + 16 * ((chunk + row) & 7), A[rt][0],
+                                         A[rt][1], A[rt][2], A[rt][3]);
+                        if (half) { A[rt][2] = 0u; A[rt][3] = 0u; }
                     }
-                } else {
+                    // B: thread (g, c) holds token g's q for words c (b0) and 4 + c (b1) of the group
+                    uint32_t bq[NT][2][8];
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
+                    for (int nt = 0; nt < NT; ++nt) {
+                        if (nt * 8 + g < m) {
+                            const uint8_t* qb = qrow[nt] + 256 * G;
+                            const uint4 v0 = *reinterpret_cast<const uint4*>(qb);
+                            const uint4 v1 = *reinterpret_cast<const uint4*>(qb + 16);
+                            bq[nt][0][0] = v0.x; bq[nt][0][1] = v0.y; bq[nt][0][2] = v0.z; bq[nt][0][3] = v0.w;
+                            bq[nt][0][4] = v1.x; bq[nt][0][5] = v1.y; bq[nt][0][6] = v1.z; bq[nt][0][7] = v1.w;
+                            if (!half) {
+                                const uint4 v2 = *reinterpret_cast<const uint4*>(qb + 128);
+                                const uint4 v3 = *reinterpret_cast<const uint4*>(qb + 144);
+                                bq[nt][1][0] = v2.x; bq[nt][1][1] = v2.y; bq[nt][1][2] = v2.z; bq[nt][1][3] = v2.w;
+                                bq[nt][1][4] = v3.x; bq[nt][1][5] = v3.y; bq[nt][1][6] = v3.z; bq[nt][1][7] = v3.w;
+                            } else {
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) b[nt][k][j] = 0u;
+                                for (int p = 0; p < 8; ++p) bq[nt][1][p] = 0u;
+                            }
+                        } else {
+#pragma unroll
+                            for (int p = 0; p < 8; ++p) { bq[nt][0][p] = 0u; bq[nt][1][p] = 0u; }
+                        }
+                    }
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) {
+                        const uint32_t msk = 0x01010101u << p;
+#pragma unroll
+                        for (int rt = 0; rt < RT; ++rt) {
+                            const uint32_t a0 = A[rt][0] & msk, a1 = A[rt][1] & msk;
+                            const uint32_t a2 = A[rt][2] & msk, a3 = A[rt][3] & msk;
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt)
+                                ptx::mma_u8s8(D[rt][nt][p], a0, a1, a2, a3, bq[nt][0][p], bq[nt][1][p]);
+                        }
+                    }
                 }
             }
-#pragma unroll
-            for (int p = 0; p < 8; ++p) {
-                const uint32_t msk = 0x01010101u << p;
-                const uint32_t a0 = wa2.x & msk, a1 = wb2.x & msk, a2 = wa2.y & msk, a3 = wb2.y & msk;
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    // chunk 0/1: b0 for p 0..3 / 4..7; chunk 2/3: b1 for p 0..3 / 4..7
-                    const uint32_t b0 = b[nt][p >> 2][p & 3];
-                    const uint32_t b1 = b[nt][2 + (p >> 2)][p & 3];
-                    ptx::mma_u8s8(D[nt][p], a0, a1, a2, a3, b0, b1);
-                }
-            }
-        }
-    }
 
-    // ---- 5. epilogue
-    if (!warp_active) return;
-    const int8_t* waAb = reinterpret_cast<const int8_t*>(&waA);
-    const int8_t* waBb = reinterpret_cast<const int8_t*>(&waB);
+            // ---- epilogue after the block's last k-chunk
+            if (last_chunk) {
+                // combine the bit-position accumulators: T = sum_p D_p * 2^(7-p) = 128 * S1
+                int T[RT][NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
+                for (int rt = 0; rt < RT; ++rt)
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            // d0: (row g, token 2c), d1: (row g, token 2c+1), d2/d3: row g + 8
-            int T = 0;
+                    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int p = 0; p < 8; ++p) T += D[nt][p][r] << (7 - p);
-            const int s1 = T >> 7;
-            const int t = nt * 8 + 2 * c + (r & 1);
-            const int o = (r < 2) ? oA : oB;
-            if (t >= m || o >= d.d_out) continue;
-            const TokStats& st = st_s[t];
-            const int acc = 2 * s1 - st.sumq;
-            const int8_t* wa = (r < 2) ? waAb : waBb;
-            float dot = 0.0f;
+                        for (int r = 0; r < 4; ++r) {
+                            int s = 0;
+                            if ((r & 1) == 0 || m > 1) {
 #pragma unroll
-            for (int k = 0; k < kRank; ++k) dot = __fmaf_rn((float)wa[k], st.u[k], dot);
-            const float alpha = (r < 2) ? alphaA : alphaB;
-            const float sa = (r < 2) ? saA : saB;
-            const float y = __fmul_rn(st.sx, __fmaf_rn(alpha, (float)acc, __fmul_rn(sa, dot)));
-            const int64_t idx = (int64_t)t * d.d_out + o;
-            if (d.y_dtype == DFSSM_BF16)
-                reinterpret_cast<__nv_bfloat16*>(e.y)[idx] = __float2bfloat16_rn(y);
-            else
-                reinterpret_cast<float*>(e.y)[idx] = y;
-            if (e.dbg.acc) e.dbg.acc[idx] = acc;
+                                for (int p = 0; p < 8; ++p) s += D[rt][nt][p][r] << (7 - p);
+                            }
+                            T[rt][nt][r] = s;
+                        }
+                // lane -> (row of this warp, n-tile); D fragment of (row, token t) sits in
+                // thread (row % 8) * 4 + (t % 8) / 2, register 2 * ((row / 8) % 2) + t % 2
+                constexpr int kRowsW = 16 * RT;
+                const int my_row = lane % kRowsW;
+                const int my_nt = lane / kRowsW;            // 0, or 1 when RT = 1 and NT = 2
+                const int rr = wrow0 + my_row;
+                const bool row_ok = rr < nrows;
+                const float* alpha_s = reinterpret_cast<const float*>(slot + R * kChunkBytes);
+                const float* sa_s = alpha_s + R;
+                const int4* wa_s = reinterpret_cast<const int4*>(slot + R * kChunkBytes + 8 * R);
+                const float alpha = alpha_s[rr], sa = sa_s[rr];
+                const WaRow wa = wa_row_from_int4(wa_s[rr]);
+                const int jmax = NT == 1 ? m : 8;
+                for (int j = 0; j < jmax; ++j) {
+                    const int src = (my_row & 7) * 4 + (j >> 1);
+                    int v_lo[RT][NT], v_hi[RT][NT];
+#pragma unroll
+                    for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            v_lo[rt][nt] = __shfl_sync(0xffffffffu, T[rt][nt][j & 1], src);
+                            v_hi[rt][nt] = __shfl_sync(0xffffffffu, T[rt][nt][2 + (j & 1)], src);
+                        }
+                    int val = 0;
+#pragma unroll
+                    for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt)
+                            if (rt == (my_row >> 4) && nt == my_nt) val = ((my_row >> 3) & 1) ? v_hi[rt][nt] : v_lo[rt][nt];
+                    const int t = 8 * my_nt + j;
+                    if (t < m && row_ok) {
+                        const int acc = 2 * (val >> 7) - ts.sumq[t];
+                        const float y = dequant(ts.sx[t], alpha, sa, acc, lora_dot(wa, ts.u[t]));
+                        const int64_t idx = (int64_t)t * L.d_out + row0 + rr;
+                        if (L.y_dtype == DFSSM_BF16)
+                            reinterpret_cast<uint16_t*>(L.y)[idx] = f32_to_bf16_bits(y);
+                        else
+                            reinterpret_cast<float*>(L.y)[idx] = y;
+                        if (L.dbg_acc) L.dbg_acc[idx] = acc;
+                    }
+                }
+            }
         }
+        __syncthreads();     // slot it % kStages is refilled by the next iteration
+        cw.advance(a);
     }
+    ptx::cp_async_wait<0>();
 }
 
-template <int NT>
-cudaError_t launch_nt(const LaunchCtx& c, int blocks) {
-    DecodeArgs a{c.entries, c.single, c.desc, c.n, c.m, c.q_ws, c.st_ws, c.err};
-    const int rb_max = c.max_d_in / 8;
-    size_t smem = 16 + ((c.m * sizeof(TokStats) + 127) & ~(size_t)127) +
-                  ((size_t)(c.m * (c.max_d_in + kTokPad) + 127) & ~(size_t)127) +
-                  (size_t)kRowsPerCta * (rb_max + kRowPad);
+struct Geometry {
+    int slot_bytes, q_region;
+    size_t smem;
+};
+
+template <int RT>
+Geometry geometry(int m, int max_d_in) {
+    constexpr int R = 16 * RT * kWarps;
+    Geometry g;
+    g.slot_bytes = (R * kChunkBytes + R * (4 + 4 + kRank) + 127) & ~127;
+    g.q_region = (m * (max_d_in + kTokPad) + 127) & ~127;
+    g.smem = ((sizeof(TokShared) + 127) & ~(size_t)127) + g.q_region + (size_t)kStages * g.slot_bytes;
+    return g;
+}
+
+template <int RT, int NT>
+cudaError_t launch_cfg(const LaunchCtx& c) {
+    constexpr int R = 16 * RT * kWarps;
+    const Geometry geo = geometry<RT>(c.m, c.max_d_in);
+    int64_t total_bytes = 0;
+    int blocks = 0;
+    for (int i = 0; i < c.n; ++i) {
+        total_bytes += (int64_t)c.host_desc[i].d_out * (c.host_desc[i].d_in / 8);
+        blocks += (c.host_desc[i].d_out + R - 1) / R;
+    }
+    int per_sm = 0;
+    cudaError_t err =
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<RT, NT>, kThreads, geo.smem);
+    if (err != cudaSuccess) return err;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    int grid = c.sm_count * per_sm;
+    if (grid > blocks) grid = blocks;
+    DecodeArgs a{c.entries, c.single, c.desc, c.n, c.m, c.st_ws, total_bytes, geo.slot_bytes, geo.q_region};
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(blocks);
-    cfg.blockDim = dim3(kWarps * 32);
-    cfg.dynamicSmemBytes = smem;
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = geo.smem;
     cfg.stream = c.stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_kernel<NT>, a);
+    return cudaLaunchKernelEx(&cfg, decode_kernel<RT, NT>, a);
 }
 
 }  // namespace
 
-int decode_blocks(const DevDesc* host_desc, int n) {
-    int total = 0;
-    for (int i = 0; i < n; ++i) total += (host_desc[i].d_out + kRowsPerCta - 1) / kRowsPerCta;
-    return total;
-}
-
 cudaError_t launch_decode(const LaunchCtx& c) {
-    const int blocks = decode_blocks(c.host_desc, c.n);
-    if (c.m <= 8) return launch_nt<1>(c, blocks);
-    return launch_nt<2>(c, blocks);
+    if (c.m <= 8) return launch_cfg<2, 1>(c);
+    return launch_cfg<1, 2>(c);
 }
 
-void set_decode_attr(int max_dyn_smem) {
-    cudaFuncSetAttribute(decode_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn_smem);
-    cudaFuncSetAttribute(decode_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn_smem);
+cudaError_t set_decode_attr(int optin) {
+    cudaError_t e = allow_dyn_smem(decode_kernel<2, 1>, optin);
+    return e != cudaSuccess ? e : allow_dyn_smem(decode_kernel<1, 2>, optin);
 }
 
 }  // namespace dfssm

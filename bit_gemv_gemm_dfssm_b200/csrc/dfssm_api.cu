@@ -20,17 +20,18 @@
 using namespace dfssm;
 
 namespace dfssm {
-void set_quant_attr(int max_dyn_smem);
-void set_decode_attr(int max_dyn_smem);
-void set_prefill_attr(int max_dyn_smem);
+cudaError_t set_quant_attr(int optin);
+cudaError_t set_decode_attr(int optin);
+cudaError_t set_prefill_attr(int optin);
 int prefill_box_tokens();
 int prefill_box_bytes();
 
 // Allow each kernel the opt-in shared memory size (a permission, not a reservation).
-static void set_kernel_attributes(int max_dyn_smem) {
-    set_quant_attr(max_dyn_smem);
-    set_decode_attr(max_dyn_smem);
-    set_prefill_attr(max_dyn_smem);
+static cudaError_t set_kernel_attributes(int optin) {
+    cudaError_t e = set_quant_attr(optin);
+    if (e == cudaSuccess) e = set_decode_attr(optin);
+    if (e == cudaSuccess) e = set_prefill_attr(optin);
+    return e;
 }
 }
 
@@ -43,6 +44,8 @@ struct dfssm_plan_s {
     int8_t* q_ws = nullptr;
     TokStats* st_ws = nullptr;
     uint32_t* err = nullptr;
+    int* part = nullptr;
+    unsigned int* tickets = nullptr;
     CUtensorMap* tmaps = nullptr;
     size_t ws_bytes = 0;
 };
@@ -112,6 +115,8 @@ void free_plan(dfssm_plan_s* p) {
     if (p->q_ws) cudaFree(p->q_ws);
     if (p->st_ws) cudaFree(p->st_ws);
     if (p->err) cudaFree(p->err);
+    if (p->part) cudaFree(p->part);
+    if (p->tickets) cudaFree(p->tickets);
     if (p->tmaps) cudaFree(p->tmaps);
     delete p;
 }
@@ -160,7 +165,7 @@ dfssm_status dfssm_linear_plan(const dfssm_linear_desc* descs, int n_descs, dfss
     }
     p->n = n_descs;
     p->hdesc.resize(n_descs);
-    int64_t q_bytes = 0, st_count = 0;
+    int64_t q_bytes = 0, st_count = 0, sign_bytes = 0;
     int32_t blk = 0, rt = 0;
     for (int i = 0; i < n_descs; ++i) {
         DevDesc& d = p->hdesc[i];
@@ -172,6 +177,8 @@ dfssm_status dfssm_linear_plan(const dfssm_linear_desc* descs, int n_descs, dfss
         d.st_off = st_count;
         d.blk_begin = blk;
         d.rt_begin = rt;
+        d.byte_begin = sign_bytes;
+        sign_bytes += (int64_t)d.d_out * (d.d_in / 8);
         q_bytes += (int64_t)d.max_m * d.d_in;       // d_in % 128 == 0 keeps every region 128-byte aligned
         st_count += d.max_m;
         blk += (d.d_out + 63) / 64;
@@ -183,13 +190,16 @@ dfssm_status dfssm_linear_plan(const dfssm_linear_desc* descs, int n_descs, dfss
     if (e == cudaSuccess) e = cudaMalloc(&p->st_ws, sizeof(TokStats) * (size_t)st_count);
     if (e == cudaSuccess) e = cudaMalloc(&p->err, 16);
     if (e == cudaSuccess) e = cudaMalloc(&p->tmaps, sizeof(CUtensorMap) * n_descs);
+    const size_t part_bytes = sizeof(int) * (size_t)n_descs * kMaxSplits * kPartTok * 20;
+    if (e == cudaSuccess) e = cudaMalloc(&p->part, part_bytes);
+    if (e == cudaSuccess) e = cudaMalloc(&p->tickets, sizeof(unsigned int) * n_descs);
     if (e != cudaSuccess) {
         cudaGetLastError();
         free_plan(p);
         return e == cudaErrorMemoryAllocation ? DFSSM_ERR_NO_MEMORY : DFSSM_ERR_CUDA;
     }
     p->ws_bytes = sizeof(DevDesc) * n_descs + (size_t)q_bytes + sizeof(TokStats) * st_count + 16 +
-                  sizeof(CUtensorMap) * n_descs;
+                  sizeof(CUtensorMap) * n_descs + part_bytes + sizeof(unsigned int) * n_descs;
 
     // tensor maps over each linear's int8 activation rows (prefill B operand)
     std::vector<CUtensorMap> tm(n_descs);
@@ -210,7 +220,8 @@ dfssm_status dfssm_linear_plan(const dfssm_linear_desc* descs, int n_descs, dfss
     e = cudaMemcpy(p->tmaps, tm.data(), sizeof(CUtensorMap) * n_descs, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(p->ddesc, p->hdesc.data(), sizeof(DevDesc) * n_descs, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemset(p->err, 0, 16);
-    if (e == cudaSuccess) set_kernel_attributes(optin);
+    if (e == cudaSuccess) e = cudaMemset(p->tickets, 0, sizeof(unsigned int) * n_descs);
+    if (e == cudaSuccess) e = set_kernel_attributes(optin);
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) { free_plan(p); return DFSSM_ERR_CUDA; }
     *out = p;
@@ -265,6 +276,8 @@ dfssm_status dfssm_linear_fwd(dfssm_plan plan, int32_t desc_index, const dfssm_l
     c.q_ws = plan->q_ws;
     c.st_ws = plan->st_ws;
     c.err = plan->err;
+    c.part = plan->part + (size_t)desc_index * kMaxSplits * kPartTok * 20;
+    c.tickets = plan->tickets + desc_index;
     c.tmaps = plan->tmaps + desc_index;
     c.max_d_in = hd.d_in;
     c.total_rows = hd.d_out;
@@ -296,6 +309,8 @@ dfssm_status dfssm_linear_stack_fwd(dfssm_plan plan, const dfssm_stack_entry* en
     c.q_ws = plan->q_ws;
     c.st_ws = plan->st_ws;
     c.err = plan->err;
+    c.part = plan->part;
+    c.tickets = plan->tickets;
     c.tmaps = plan->tmaps;
     c.max_d_in = max_d_in;
     c.total_rows = rows;

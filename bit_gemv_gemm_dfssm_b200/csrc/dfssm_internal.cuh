@@ -12,6 +12,8 @@ namespace dfssm {
 constexpr int kRank = 16;
 constexpr int kMaxDIn = 8192;
 constexpr int kMaxM = 65536;
+constexpr int kMaxSplits = 8;        // d_in splits of the quantisation kernel for m <= 16
+constexpr int kPartTok = 16;         // tokens covered by the split partials
 
 // Per-linear shape and workspace offsets, resident in device memory.
 struct DevDesc {
@@ -23,6 +25,7 @@ struct DevDesc {
     int64_t st_off;     // index of its first TokStats record
     int32_t blk_begin;  // first 64-row decode block of this linear in the flattened stack order
     int32_t rt_begin;   // first 128-row prefill tile row of this linear in the same order
+    int64_t byte_begin; // sign bytes of all preceding linears (decode work balance)
 };
 
 // Per-token values the main kernels need after quantisation.
@@ -62,6 +65,8 @@ struct LaunchCtx {
     int8_t* q_ws;
     TokStats* st_ws;
     uint32_t* err;
+    int* part;                         // split partials: n x kMaxSplits x 16 tokens x 20 ints
+    unsigned int* tickets;             // n split tickets, zero between calls
     const void* tmaps;                 // device array of CUtensorMap (prefill), one per desc
     int max_d_in;                      // largest d_in among the n linears
     int64_t total_rows;                // sum of d_out over the n linears
@@ -74,6 +79,16 @@ cudaError_t launch_pack_sign(const void* src, int src_dtype, int d_out, int d_in
 cudaError_t launch_quant(const LaunchCtx& c);
 cudaError_t launch_decode(const LaunchCtx& c);
 cudaError_t launch_prefill(const LaunchCtx& c);
+
+// Allow `kernel` the opt-in dynamic shared memory (minus its static shared memory).
+template <typename K>
+inline cudaError_t allow_dyn_smem(K kernel, int optin) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                optin - (int)fa.sharedSizeBytes);
+}
 
 // ---- small device helpers -----------------------------------------------------------
 

@@ -12,7 +12,7 @@
 //   D[o, t] = sum_k b[o, k] * q[t, k]    (b = sign bit as 0/1, int32 in TMEM)
 //   acc     = 2 * D - sum_k q[t, k]       (a +-1 weight is 2b - 1)
 //
-// Persistent kernel, one CTA per SM, 12 warps with fixed roles:
+// Persistent kernel, one CTA per SM, 16 warps with fixed roles:
 //   warp 0      TMA producer: 256-token x 128-byte tiles of the int8
 //               activations (permuted column order, 128B swizzle), no multicast
 //   warp 1      TMEM owner and MMA issuer: tcgen05.mma.kind::i8, M=128 rows,
@@ -20,15 +20,18 @@
 //   warps 4-7   bit expansion: each thread owns one weight row of the tile,
 //               loads 16 bytes of sign bits per k-block and writes 128 0/1 bytes
 //               into the K-major SWIZZLE_128B layout the MMA reads
-//   warps 8-11  epilogue: tcgen05.ld of its 32 TMEM lanes (= output rows),
-//               acc = 2D - sum q, LoRA up-projection and dequantisation,
-//               coalesced stores of y along the output dimension
+//   warps 8-15  epilogue: tcgen05.ld of its 32 TMEM lanes (= output rows) and
+//               half of the 256 token columns, acc = 2D - sum q, LoRA
+//               up-projection and dequantisation, coalesced stores of y along
+//               the output dimension; the per-token scalars of each 16-token
+//               chunk are staged in a warp-private, double-buffered smem slice
 // 4-stage shared-memory ring (mbarriers), two TMEM accumulator buffers of 256
 // columns so the epilogue of one tile overlaps the main loop of the next.
 // Every mbarrier wait is bounded; a timeout sets the plan's error word.
 #include <cuda.h>
 
 #include "dfssm_internal.cuh"
+#include "epilogue.cuh"
 #include "ptx.cuh"
 
 namespace dfssm {
@@ -41,8 +44,12 @@ constexpr int BK = 128;            // k (bytes) per stage
 constexpr int STAGES = 4;
 constexpr int A_STAGE = BM * BK;   // 16 KB
 constexpr int B_STAGE = BN * BK;   // 32 KB
-constexpr int NUM_THREADS = 12 * 32;
-constexpr int SMEM_BYTES = STAGES * (A_STAGE + B_STAGE) + 256 + 1024;
+constexpr int NUM_THREADS = 16 * 32;
+constexpr int EPI_WARPS = 8;                         // warps 8..15
+constexpr int EPI_THREADS = EPI_WARPS * 32;
+constexpr int STAT_CHUNK = 16 * (int)sizeof(TokStats);  // per-token scalars of 16 tokens (1280 B)
+constexpr int STAT_BYTES = EPI_WARPS * 2 * STAT_CHUNK;  // double-buffered, one pair per epilogue warp
+constexpr int SMEM_BYTES = STAGES * (A_STAGE + B_STAGE) + STAT_BYTES + 256 + 1024;
 constexpr uint32_t TMEM_COLS = 512;
 
 struct PrefillArgs {
@@ -93,15 +100,18 @@ __device__ __forceinline__ void set_err(uint32_t* err, uint32_t bit) { atomicOr(
 
 __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_constant__ PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    // 1024-byte aligned base (SWIZZLE_128B atoms), offset from the __shared__ array so the
+    // compiler keeps shared-memory addressing
+    uint8_t* smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* sA = smem;
     uint8_t* sB = smem + STAGES * A_STAGE;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE);
+    uint8_t* sStat = sB + STAGES * B_STAGE;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sStat + STAT_BYTES);
     uint64_t* full_a = bars;               // [STAGES], 128 arrivals (expansion threads)
     uint64_t* full_b = bars + STAGES;      // [STAGES], TMA transaction bytes
     uint64_t* empty = bars + 2 * STAGES;   // [STAGES], MMA commit
     uint64_t* acc_full = bars + 3 * STAGES;       // [2], MMA commit
-    uint64_t* acc_empty = bars + 3 * STAGES + 2;  // [2], 128 epilogue arrivals
+    uint64_t* acc_empty = bars + 3 * STAGES + 2;  // [2], EPI_THREADS epilogue arrivals
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 4);
     volatile uint32_t* abort_flag = tmem_slot + 1;
 
@@ -116,7 +126,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(&acc_full[b], 1);
-            ptx::mbar_init(&acc_empty[b], 128);
+            ptx::mbar_init(&acc_empty[b], EPI_THREADS);
         }
         *abort_flag = 0;
         ptx::fence_mbar_init();
@@ -229,10 +239,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
             if (!ok) break;
         }
     } else if (warp >= 8) {
-        // ------------------------------------------------ epilogue (TMEM lanes 32*(warp%4) ..)
+        // ------------------------------------------------ epilogue
+        // warp 8 + 4h + q handles TMEM lanes 32q.. (output rows) and token columns [128h, 128h + 128)
         ptx::pdl_wait();
         const int q4 = warp & 3;
+        const int half = (warp - 8) >> 2;
         const int r = q4 * 32 + lane;
+        uint8_t* stat_buf = sStat + (warp - 8) * 2 * STAT_CHUNK;
         int tcount = 0;
         for (int tile = blockIdx.x; tile < a.n_tiles && !*abort_flag; tile += gridDim.x, ++tcount) {
             const TileCoord tc = tile_coord(a.desc, a.n, n_tt, tile);
@@ -240,18 +253,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
             const dfssm_stack_entry& e = entry_at(a.entries, a.single, tc.lin);
             const int o = tc.row0 + r;
             const bool valid = o < d.d_out && entry_ptrs_ok(e);
-            float alpha = 0.f, sa = 0.f, wa[kRank];
+            float alpha = 0.f, sa = 0.f;
+            WaRow wa = wa_row_from_int4(make_int4(0, 0, 0, 0));
             if (valid) {
                 alpha = e.w.alpha[o];
                 sa = e.w.sa[o];
-                const int4 w4 = *reinterpret_cast<const int4*>(e.w.wa + (int64_t)o * kRank);
-                const int8_t* wb = reinterpret_cast<const int8_t*>(&w4);
-#pragma unroll
-                for (int k = 0; k < kRank; ++k) wa[k] = (float)wb[k];
-            } else {
-#pragma unroll
-                for (int k = 0; k < kRank; ++k) wa[k] = 0.f;
+                wa = wa_row_from_int4(*reinterpret_cast<const int4*>(e.w.wa + (int64_t)o * kRank));
             }
+            // per-token scalars: chunk ch covers tokens tok_base + 16 ch .. + 15 (80 x 16 bytes)
+            const int tok_base = tc.tok0 + half * (BN / 2);
+            const uint4* st_src = reinterpret_cast<const uint4*>(a.st_ws + d.st_off);
+            auto load_chunk = [&](int ch, uint4 (&rg)[3]) {
+#pragma unroll
+                for (int u = 0; u < 3; ++u) {
+                    const int idx = lane + 32 * u;                  // uint4 index inside the chunk
+                    const int tok = tok_base + 16 * ch + idx / 5;
+                    rg[u] = (idx < 80 && tok < a.m) ? st_src[(int64_t)(tok_base + 16 * ch) * 5 + idx]
+                                                    : make_uint4(0u, 0u, 0u, 0u);
+                }
+            };
+            auto store_chunk = [&](int buf_i, const uint4 (&rg)[3]) {
+                uint4* dst = reinterpret_cast<uint4*>(stat_buf + buf_i * STAT_CHUNK);
+#pragma unroll
+                for (int u = 0; u < 3; ++u)
+                    if (lane + 32 * u < 80) dst[lane + 32 * u] = rg[u];
+            };
+            uint4 rg[3];
+            load_chunk(0, rg);
+            store_chunk(0, rg);
+
             const int buf = tcount & 1;
             const uint32_t acc_ph = (uint32_t)(tcount >> 1) & 1u;
             const bool got = __all_sync(0xffffffffu, ptx::mbar_wait(&acc_full[buf], acc_ph));
@@ -260,32 +290,52 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
                 break;
             }
             ptx::tc_fence_after();
-            const TokStats* st = a.st_ws + d.st_off;
-            const uint32_t taddr = tmem_base + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(buf * BN);
-            for (int cb = 0; cb < BN; cb += 16) {
+            const uint32_t taddr = tmem_base + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(buf * BN + half * (BN / 2));
+            constexpr int NCH = BN / 2 / 16;
+            for (int ch = 0; ch < NCH; ++ch) {
+                __syncwarp();
+                const bool more = ch + 1 < NCH && tok_base + 16 * (ch + 1) < a.m;
+                if (more) load_chunk(ch + 1, rg);
                 uint32_t v[16];
-                ptx::tmem_ld_32x32b_x16(taddr + (uint32_t)cb, v);
+                ptx::tmem_ld_32x32b_x16(taddr + (uint32_t)(16 * ch), v);
                 ptx::tmem_ld_wait();
-                if (tc.tok0 + cb >= a.m) continue;
+                const TokStats* stc = reinterpret_cast<const TokStats*>(stat_buf + (ch & 1) * STAT_CHUNK);
+                const int t0c = tok_base + 16 * ch;
+                if (t0c < a.m) {
+                    const int nj = min(16, a.m - t0c);
+                    const int64_t base_idx = (int64_t)t0c * d.d_out + o;
+                    if (nj == 16 && valid) {
+                        // full chunk: no per-token checks
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int t = tc.tok0 + cb + j;
-                    if (t >= a.m) break;
-                    const TokStats& s = st[t];
-                    const int acc = 2 * (int)v[j] - s.sumq;
-                    float dot = 0.0f;
+                        for (int j = 0; j < 16; ++j) {
+                            const TokStats& st = stc[j];
+                            const int acc = 2 * (int)v[j] - st.sumq;
+                            const float y = dequant(st.sx, alpha, sa, acc, lora_dot(wa, st.u));
+                            const int64_t idx = base_idx + (int64_t)j * d.d_out;
+                            if (d.y_dtype == DFSSM_BF16)
+                                reinterpret_cast<uint16_t*>(e.y)[idx] = f32_to_bf16_bits(y);
+                            else
+                                reinterpret_cast<float*>(e.y)[idx] = y;
+                            if (e.dbg.acc) e.dbg.acc[idx] = acc;
+                        }
+                    } else if (valid) {
 #pragma unroll
-                    for (int k = 0; k < kRank; ++k) dot = __fmaf_rn(wa[k], s.u[k], dot);
-                    const float y = __fmul_rn(s.sx, __fmaf_rn(alpha, (float)acc, __fmul_rn(sa, dot)));
-                    if (valid) {
-                        const int64_t idx = (int64_t)t * d.d_out + o;
-                        if (d.y_dtype == DFSSM_BF16)
-                            reinterpret_cast<__nv_bfloat16*>(e.y)[idx] = __float2bfloat16_rn(y);
-                        else
-                            reinterpret_cast<float*>(e.y)[idx] = y;
-                        if (e.dbg.acc) e.dbg.acc[idx] = acc;
+                        for (int j = 0; j < 16; ++j) {
+                            if (j >= nj) break;
+                            const TokStats& st = stc[j];
+                            const int acc = 2 * (int)v[j] - st.sumq;
+                            const float y = dequant(st.sx, alpha, sa, acc, lora_dot(wa, st.u));
+                            const int64_t idx = base_idx + (int64_t)j * d.d_out;
+                            if (d.y_dtype == DFSSM_BF16)
+                                reinterpret_cast<uint16_t*>(e.y)[idx] = f32_to_bf16_bits(y);
+                            else
+                                reinterpret_cast<float*>(e.y)[idx] = y;
+                            if (e.dbg.acc) e.dbg.acc[idx] = acc;
+                        }
                     }
                 }
+                __syncwarp();
+                if (more) store_chunk((ch + 1) & 1, rg);
             }
             ptx::tc_fence_before();
             ptx::mbar_arrive(&acc_empty[buf]);
@@ -324,9 +374,9 @@ cudaError_t launch_prefill(const LaunchCtx& c) {
     return cudaLaunchKernelEx(&cfg, prefill_kernel, a);
 }
 
-void set_prefill_attr(int max_dyn_smem) {
-    cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         max_dyn_smem < SMEM_BYTES ? max_dyn_smem : SMEM_BYTES);
+cudaError_t set_prefill_attr(int optin) {
+    return cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                optin < SMEM_BYTES ? optin : SMEM_BYTES);
 }
 
 int prefill_box_tokens() { return BN; }

@@ -9,12 +9,27 @@
 //   q[t,j] = clamp(rint(x[t,j] * (127/amax)), +-127), s_x = amax/127 (IEEE fp32,
 //            round-to-nearest; amax == 0 gives q = 0, s_x = 0)
 //   sumq   = sum_j q[t,j]                          (int32)
-//   h[t,k] = sum_j W_B[k,j] q[t,j]                 (int32, dp4a)
+//   h[t,k] = sum_j W_B[k,j] q[t,j]                 (int32, warp MMA s8 x s8)
 //   u[t,k] = s_B[k] * h[t,k]                       (fp32)
 // and stores q in the permuted int8 layout the scaffold kernels read, plus
-// s_x, sumq and u. One block owns one linear and a group of tokens; W_B is
-// staged in shared memory once per block.
+// s_x, sumq and u.
+//
+// A block owns one linear and up to kTokPerBlock tokens, processed in rounds of
+// 16 tokens (one MMA tile). The 8 warps split the 32-column k-blocks of d_in
+// between them: pass 1 finds each token's amax, pass 2 quantises x straight
+// into MMA A fragments (16 tokens x 32 columns), runs h += q * W_B^T on the
+// warp MMA (m16n8k32, two n-tiles for the 16 LoRA rows) and writes q to a
+// shared tile, from which the block stores the permuted rows with 16-byte
+// stores (a 4x4 byte transpose with PRMT per 16 bytes).
+//
+// Few tokens (m <= 16, one round): the k-blocks of a linear are split over S
+// blocks so that W_B (the only large read) streams through many SMs. Every
+// split block finds the full-row amax itself, handles its own columns, and
+// writes partial h and sum q; the last split block to finish (atomic ticket)
+// adds the partials in split order, writes the per-token scalars and resets
+// the ticket for the next call.
 #include "dfssm_internal.cuh"
+#include "epilogue.cuh"
 #include "ptx.cuh"
 
 namespace dfssm {
@@ -23,24 +38,84 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kMaxChunks = kMaxDIn / 8 / kThreads;   // 8-column chunks per thread (<= 4)
+constexpr int kTok = 16;              // tokens per round
+constexpr int kTokPerBlock = 64;      // rounds per block: 4
 
-struct QuantSmem {
-    float red_f[kWarps];
-    int red_i[kWarps];
-    int red_h[kWarps][kRank];
+struct QuantRed {
+    float amax[kWarps][kTok];
+    int sumq[kWarps][kTok];
+    int h[kWarps][kTok][kRank];
+    float inv[kTok];
+    float sx[kTok];
 };
 
-__global__ void __launch_bounds__(kThreads) quant_kernel(
-    const dfssm_stack_entry* __restrict__ entries, const dfssm_stack_entry single,
-    const DevDesc* __restrict__ descs, int m, int tok_per_block,
-    int8_t* __restrict__ q_ws, TokStats* __restrict__ st_ws, uint32_t* __restrict__ err) {
+// 4 bf16 (8 bytes) -> 4 int8 packed little-endian
+__device__ __forceinline__ uint32_t quant4(uint2 raw, float inv, bool zero, int& sum) {
+    const int q0 = quant1(bf16_bits_to_float(raw.x & 0xFFFFu), inv, zero);
+    const int q1 = quant1(bf16_bits_to_float(raw.x >> 16), inv, zero);
+    const int q2 = quant1(bf16_bits_to_float(raw.y & 0xFFFFu), inv, zero);
+    const int q3 = quant1(bf16_bits_to_float(raw.y >> 16), inv, zero);
+    sum += q0 + q1 + q2 + q3;
+    return (uint32_t)(q0 & 0xFF) | ((uint32_t)(q1 & 0xFF) << 8) | ((uint32_t)(q2 & 0xFF) << 16) |
+           ((uint32_t)(q3 & 0xFF) << 24);
+}
+
+__device__ __forceinline__ float absmax8(uint4 v, float m) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        m = fmaxf(m, fabsf(bf16_bits_to_float(w[i] & 0xFFFFu)));
+        m = fmaxf(m, fabsf(bf16_bits_to_float(w[i] >> 16)));
+    }
+    return m;
+}
+
+__device__ __forceinline__ void mma_s8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) { return __byte_perm(a, b, sel); }
+
+// word r of the result = byte r of a, b, c, d (4x4 byte transpose)
+__device__ __forceinline__ uint4 transpose4x4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    const uint32_t t0 = prmt(a, b, 0x5140), t1 = prmt(a, b, 0x7362);
+    const uint32_t t2 = prmt(c, d, 0x5140), t3 = prmt(c, d, 0x7362);
+    return make_uint4(prmt(t0, t2, 0x5410), prmt(t0, t2, 0x7632), prmt(t1, t3, 0x5410), prmt(t1, t3, 0x7632));
+}
+
+struct QuantArgs {
+    const dfssm_stack_entry* entries;
+    dfssm_stack_entry single;
+    const DevDesc* descs;
+    int m;
+    int splits;             // blocks per linear along d_in (1 when m > 16)
+    int8_t* q_ws;
+    TokStats* st_ws;
+    int* part;              // [linear][split][16 tokens][kPartInts] partial h and sum q (splits > 1)
+    unsigned int* tickets;  // one per linear, zero between calls
+    uint32_t* err;
+};
+
+constexpr int kPartInts = 20;   // 16 h + sum q, padded
+
+__global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__ QuantArgs qa) {
+    const dfssm_stack_entry* entries = qa.entries;
+    const DevDesc* descs = qa.descs;
+    const int m = qa.m;
+    int8_t* __restrict__ q_ws = qa.q_ws;
+    TokStats* __restrict__ st_ws = qa.st_ws;
+    uint32_t* err = qa.err;
     extern __shared__ __align__(16) uint8_t smem_raw[];
     // let the dependent scaffold kernel start streaming weights right away;
     // it waits for this grid's results before reading them
     ptx::pdl_launch_dependents();
     const int lin = blockIdx.y;
-    const dfssm_stack_entry& e = entry_at(entries, single, lin);
+    const dfssm_stack_entry& e = entry_at(entries, qa.single, lin);
     const DevDesc d = descs[lin];
     if (entries && e.desc_index != lin) {
         if (threadIdx.x == 0) atomicOr(err, DFSSM_DEVERR_ENTRY_DESC);
@@ -51,154 +126,185 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(
         return;
     }
     const int d_in = d.d_in;
-    const int n_chunk = d_in / 8;                 // 8-column chunks per row
+    const int nkb = d_in >> 5;                    // 32-column k-blocks
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, c = lane & 3;
 
-    int8_t* wb_s = reinterpret_cast<int8_t*>(smem_raw);             // 16 x d_in
-    int8_t* qrow = wb_s + kRank * d_in;                              // d_in
-    QuantSmem& red = *reinterpret_cast<QuantSmem*>(qrow + d_in);
+    QuantRed& red = *reinterpret_cast<QuantRed*>(smem_raw);
+    int8_t* q_s = reinterpret_cast<int8_t*>(smem_raw + ((sizeof(QuantRed) + 127) & ~(size_t)127));  // [kTok][d_in]
 
-    // stage W_B
-    {
-        const uint4* src = reinterpret_cast<const uint4*>(e.w.wb);
-        uint4* dst = reinterpret_cast<uint4*>(wb_s);
-        for (int i = tid; i < kRank * d_in / 16; i += kThreads) dst[i] = src[i];
-    }
-    float sb[kRank];
-#pragma unroll
-    for (int k = 0; k < kRank; ++k) sb[k] = e.w.sb[k];
-    __syncthreads();
+    const uint16_t* xg = reinterpret_cast<const uint16_t*>(e.x);
+    const uint8_t* wb = reinterpret_cast<const uint8_t*>(e.w.wb);
 
-    const int t0 = blockIdx.x * tok_per_block;
-    const int t1 = min(m, t0 + tok_per_block);
-    const uint16_t* xbase = reinterpret_cast<const uint16_t*>(e.x);
+    // split along d_in (few tokens) or along tokens (many tokens)
+    const int split = qa.splits > 1 ? (int)blockIdx.x : 0;
+    const int kb_lo = split * nkb / qa.splits, kb_hi = (split + 1) * nkb / qa.splits;
+    const int tb0 = qa.splits > 1 ? 0 : blockIdx.x * kTokPerBlock;
+    const int tb1 = min(m, tb0 + kTokPerBlock);
+    for (int t0 = tb0; t0 < tb1; t0 += kTok) {
+        const int nt = min(kTok, tb1 - t0);
 
-    for (int t = t0; t < t1; ++t) {
-        // ---- load x and find amax
-        float xv[kMaxChunks][8];
-        float amax = 0.0f;
-#pragma unroll
-        for (int c = 0; c < kMaxChunks; ++c) {
-            int ch = tid + c * kThreads;
-            if (ch < n_chunk) {
-                uint4 raw = *reinterpret_cast<const uint4*>(xbase + (int64_t)t * d_in + ch * 8);
-                uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    xv[c][2 * i] = bf16_bits_to_float(wv[i] & 0xFFFFu);
-                    xv[c][2 * i + 1] = bf16_bits_to_float(wv[i] >> 16);
+        // ---- pass 1: amax. lane l covers token l/2, columns 16*(l&1) .. +15 of each k-block
+        {
+            const int tk = lane >> 1, hf = lane & 1;
+            float am = 0.0f;
+            if (tk < nt) {
+                const uint16_t* row = xg + (int64_t)(t0 + tk) * d_in + 16 * hf;
+#pragma unroll 4
+                for (int kb = warp; kb < nkb; kb += kWarps) {
+                    const uint4* p = reinterpret_cast<const uint4*>(row + 32 * kb);
+                    am = absmax8(p[0], am);
+                    am = absmax8(p[1], am);
                 }
-#pragma unroll
-                for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(xv[c][i]));
             }
+            am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+            if (hf == 0) red.amax[warp][tk] = am;
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        if (lane == 0) red.red_f[warp] = amax;
         __syncthreads();
-        amax = red.red_f[0];
+        if (tid < kTok) {
+            float am = 0.0f;
 #pragma unroll
-        for (int w = 1; w < kWarps; ++w) amax = fmaxf(amax, red.red_f[w]);
-        // NaN compares false in fmaxf chains, so check finiteness of the inputs' max explicitly
-        if (!isfinite(amax) && tid == 0) atomicOr(err, DFSSM_DEVERR_NONFINITE);
+            for (int w = 0; w < kWarps; ++w) am = fmaxf(am, red.amax[w][tid]);
+            if (tid < nt && !isfinite(am)) atomicOr(err, DFSSM_DEVERR_NONFINITE);
+            red.inv[tid] = quant_inv(am);
+            red.sx[tid] = quant_sx(am);
+        }
+        __syncthreads();
 
-        const bool zero = (amax == 0.0f);
-        const float inv = zero ? 0.0f : __fdiv_rn(127.0f, amax);
-        const float sx = zero ? 0.0f : __fdiv_rn(amax, 127.0f);
+        // ---- pass 2: quantise into A fragments, h += q * W_B^T, q -> shared tile
+        const float invA = red.inv[g], invB = red.inv[g + 8];
+        const bool zA = invA == 0.0f, zB = invB == 0.0f;
+        const bool hasA = g < nt, hasB = g + 8 < nt;
+        const uint16_t* xA = xg + (int64_t)(t0 + g) * d_in + 4 * c;
+        const uint16_t* xB = xg + (int64_t)(t0 + g + 8) * d_in + 4 * c;
+        int D0[4] = {0, 0, 0, 0}, D1[4] = {0, 0, 0, 0};
+        int sA = 0, sB = 0;
+#pragma unroll 2
+        for (int kb = kb_lo + warp; kb < kb_hi; kb += kWarps) {
+            const int col = 32 * kb;
+            const uint2 zero2 = make_uint2(0u, 0u);
+            const uint2 xa0 = hasA ? *reinterpret_cast<const uint2*>(xA + col) : zero2;
+            const uint2 xa1 = hasA ? *reinterpret_cast<const uint2*>(xA + col + 16) : zero2;
+            const uint2 xb0 = hasB ? *reinterpret_cast<const uint2*>(xB + col) : zero2;
+            const uint2 xb1 = hasB ? *reinterpret_cast<const uint2*>(xB + col + 16) : zero2;
+            const uint32_t a0 = quant4(xa0, invA, zA, sA);
+            const uint32_t a2 = quant4(xa1, invA, zA, sA);
+            const uint32_t a1 = quant4(xb0, invB, zB, sB);
+            const uint32_t a3 = quant4(xb1, invB, zB, sB);
+            // B fragments: W_B rows g (n-tile 0) and g + 8 (n-tile 1), k = 4c.. and 16 + 4c..
+            const uint32_t b00 = *reinterpret_cast<const uint32_t*>(wb + (int64_t)g * d_in + col + 4 * c);
+            const uint32_t b01 = *reinterpret_cast<const uint32_t*>(wb + (int64_t)g * d_in + col + 16 + 4 * c);
+            const uint32_t b10 = *reinterpret_cast<const uint32_t*>(wb + (int64_t)(g + 8) * d_in + col + 4 * c);
+            const uint32_t b11 = *reinterpret_cast<const uint32_t*>(wb + (int64_t)(g + 8) * d_in + col + 16 + 4 * c);
+            mma_s8s8(D0, a0, a1, a2, a3, b00, b01);
+            mma_s8s8(D1, a0, a1, a2, a3, b10, b11);
+            *reinterpret_cast<uint32_t*>(q_s + g * d_in + col + 4 * c) = a0;
+            *reinterpret_cast<uint32_t*>(q_s + g * d_in + col + 16 + 4 * c) = a2;
+            *reinterpret_cast<uint32_t*>(q_s + (g + 8) * d_in + col + 4 * c) = a1;
+            *reinterpret_cast<uint32_t*>(q_s + (g + 8) * d_in + col + 16 + 4 * c) = a3;
+        }
+        // quad reduction of the token sums
+        sA += __shfl_xor_sync(0xffffffffu, sA, 1);
+        sA += __shfl_xor_sync(0xffffffffu, sA, 2);
+        sB += __shfl_xor_sync(0xffffffffu, sB, 1);
+        sB += __shfl_xor_sync(0xffffffffu, sB, 2);
+        if (c == 0) {
+            red.sumq[warp][g] = sA;
+            red.sumq[warp][g + 8] = sB;
+        }
+        // D fragment: (token g, lora 2c), (g, 2c+1), (g+8, 2c), (g+8, 2c+1); D1 for lora + 8
+        red.h[warp][g][2 * c] = D0[0];
+        red.h[warp][g][2 * c + 1] = D0[1];
+        red.h[warp][g + 8][2 * c] = D0[2];
+        red.h[warp][g + 8][2 * c + 1] = D0[3];
+        red.h[warp][g][8 + 2 * c] = D1[0];
+        red.h[warp][g][8 + 2 * c + 1] = D1[1];
+        red.h[warp][g + 8][8 + 2 * c] = D1[2];
+        red.h[warp][g + 8][8 + 2 * c + 1] = D1[3];
+        __syncthreads();
 
-        // ---- quantise, sum, LoRA down-projection
-        int sumq = 0;
-        int hp[kRank];
+        // ---- per-token scalars: thread (token tid / 16, lora row tid % 16)
+        {
+            const int tk = tid >> 4, k = tid & 15;
+            int h = 0, sq = 0;
 #pragma unroll
-        for (int k = 0; k < kRank; ++k) hp[k] = 0;
+            for (int w = 0; w < kWarps; ++w) h += red.h[w][tk][k];
+            if (k == 0) {
 #pragma unroll
-        for (int c = 0; c < kMaxChunks; ++c) {
-            int ch = tid + c * kThreads;
-            if (ch < n_chunk) {
-                uint32_t qw[2] = {0u, 0u};
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    int qi = zero ? 0 : __float2int_rn(__fmul_rn(xv[c][i], inv));
-                    qi = max(-127, min(127, qi));
-                    sumq += qi;
-                    qw[i >> 2] |= (uint32_t)(qi & 0xFF) << (8 * (i & 3));
+                for (int w = 0; w < kWarps; ++w) sq += red.sumq[w][tk];
+            }
+            bool final_block = true;
+            if (qa.splits > 1) {
+                int* mine = qa.part + ((int64_t)lin * qa.splits + split) * kTok * kPartInts + tk * kPartInts;
+                mine[k] = h;
+                if (k == 0) mine[16] = sq;
+                __threadfence();
+                __syncthreads();
+                __shared__ unsigned int ticket;
+                if (tid == 0) ticket = atomicAdd(qa.tickets + lin, 1u);
+                __syncthreads();
+                final_block = ticket == (unsigned int)(qa.splits - 1);
+                if (final_block) {
+                    __threadfence();
+                    h = 0;
+                    sq = 0;
+                    for (int sp = 0; sp < qa.splits; ++sp) {
+                        const int* pp = qa.part + ((int64_t)lin * qa.splits + sp) * kTok * kPartInts + tk * kPartInts;
+                        h += __ldcg(pp + k);
+                        if (k == 0) sq += __ldcg(pp + 16);
+                    }
+                    if (tid == 0) qa.tickets[lin] = 0u;
                 }
-                *reinterpret_cast<uint2*>(qrow + ch * 8) = make_uint2(qw[0], qw[1]);
-                if (e.dbg.q)
-                    *reinterpret_cast<uint2*>(e.dbg.q + (int64_t)t * d_in + ch * 8) = make_uint2(qw[0], qw[1]);
-#pragma unroll
-                for (int k = 0; k < kRank; ++k) {
-                    uint2 wbk = *reinterpret_cast<const uint2*>(wb_s + k * d_in + ch * 8);
-                    hp[k] = __dp4a((int)qw[0], (int)wbk.x, hp[k]);
-                    hp[k] = __dp4a((int)qw[1], (int)wbk.y, hp[k]);
+            }
+            if (final_block && tk < nt) {
+                TokStats* st = st_ws + d.st_off + t0 + tk;
+                st->u[k] = __fmul_rn(e.w.sb[k], (float)h);
+                if (e.dbg.h) e.dbg.h[(int64_t)(t0 + tk) * kRank + k] = h;
+                if (k == 0) {
+                    st->sx = red.sx[tk];
+                    st->sumq = sq;
+                    if (e.dbg.sx) e.dbg.sx[t0 + tk] = red.sx[tk];
                 }
             }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sumq += __shfl_xor_sync(0xffffffffu, sumq, o);
-#pragma unroll
-        for (int k = 0; k < kRank; ++k) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) hp[k] += __shfl_xor_sync(0xffffffffu, hp[k], o);
-        }
-        if (lane == 0) {
-            red.red_i[warp] = sumq;
-#pragma unroll
-            for (int k = 0; k < kRank; ++k) red.red_h[warp][k] = hp[k];
-        }
-        __syncthreads();   // qrow complete, partial sums visible
 
-        // ---- per-token scalars
-        TokStats* st = st_ws + d.st_off + t;
-        if (tid < kRank) {
-            int h = 0;
-#pragma unroll
-            for (int w = 0; w < kWarps; ++w) h += red.red_h[w][tid];
-            st->u[tid] = __fmul_rn(sb[tid], (float)h);
-            if (e.dbg.h) e.dbg.h[(int64_t)t * kRank + tid] = h;
+        // ---- q rows: permuted (position 32G + 4p + i <- column 32G + 8i + p) and natural (debug)
+        const int c_lo = 2 * kb_lo, nchunk = 2 * (kb_hi - kb_lo);    // 16-byte output chunks of this block
+        for (int i = tid; i < nt * nchunk; i += kThreads) {
+            const int tk = i / nchunk, s16 = c_lo + (i - tk * nchunk);
+            const int G = s16 >> 1, hlf = s16 & 1;
+            // output word r holds p = 4 hlf + r: bytes src[p], src[8+p], src[16+p], src[24+p],
+            // i.e. byte r of source words hlf, 2 + hlf, 4 + hlf, 6 + hlf of the 32-byte group
+            const uint32_t* src = reinterpret_cast<const uint32_t*>(q_s + tk * d_in + 32 * G);
+            const uint4 o4 = transpose4x4(src[hlf], src[2 + hlf], src[4 + hlf], src[6 + hlf]);
+            // the decode kernel (m <= 16) quantises for itself; only the prefill path reads q_ws
+            if (qa.splits == 1) *reinterpret_cast<uint4*>(q_ws + d.q_off + (int64_t)(t0 + tk) * d_in + 16 * s16) = o4;
+            if (e.dbg.q)
+                *reinterpret_cast<uint4*>(e.dbg.q + (int64_t)(t0 + tk) * d_in + 16 * s16) =
+                    *reinterpret_cast<const uint4*>(q_s + tk * d_in + 16 * s16);
         }
-        if (tid == kRank) {
-            int s = 0;
-#pragma unroll
-            for (int w = 0; w < kWarps; ++w) s += red.red_i[w];
-            st->sx = sx;
-            st->sumq = s;
-            if (e.dbg.sx) e.dbg.sx[t] = sx;
-        }
-
-        // ---- permuted int8 row: position 32g + 4p + i <- column 32g + 8i + p
-        int8_t* qdst = q_ws + d.q_off + (int64_t)t * d_in;
-        for (int s16 = tid; s16 < d_in / 16; s16 += kThreads) {
-            const int g = s16 >> 1, half = s16 & 1;
-            uint32_t outw[4];
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {           // output word r: p = 4*half + r, i = 0..3
-                const int p = 4 * half + r;
-                uint32_t wv = 0;
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    wv |= (uint32_t)(uint8_t)qrow[32 * g + 8 * i + p] << (8 * i);
-                outw[r] = wv;
-            }
-            *reinterpret_cast<uint4*>(qdst + 16 * s16) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
-        }
-        __syncthreads();   // qrow / red reused by the next token
+        __syncthreads();   // q_s and red are reused by the next round
     }
 }
 
 }  // namespace
 
 cudaError_t launch_quant(const LaunchCtx& c) {
-    int tpb = c.m >= 256 ? 32 : (c.m >= 64 ? 8 : (c.m >= 16 ? 2 : 1));
-    dim3 grid((c.m + tpb - 1) / tpb, c.n);
-    size_t smem = (size_t)(kRank + 1) * c.max_d_in + sizeof(QuantSmem);
-    quant_kernel<<<grid, kThreads, smem, c.stream>>>(c.entries, c.single, c.desc, c.m, tpb,
-                                                     c.q_ws, c.st_ws, c.err);
+    int splits = 1;
+    if (c.m <= kTok) {
+        // enough blocks to cover the SMs twice, at least 8 k-blocks (one per warp) per split
+        int min_nkb = 1 << 30;
+        for (int i = 0; i < c.n; ++i) min_nkb = min(min_nkb, c.host_desc[i].d_in / 32);
+        splits = (2 * c.sm_count + c.n - 1) / c.n;
+        splits = max(1, min(splits, min(kMaxSplits, min_nkb / kWarps)));
+    }
+    dim3 grid(splits > 1 ? splits : (c.m + kTokPerBlock - 1) / kTokPerBlock, c.n);
+    const size_t smem = ((sizeof(QuantRed) + 127) & ~(size_t)127) + (size_t)kTok * c.max_d_in;
+    QuantArgs qa{c.entries, c.single, c.desc, c.m, splits, c.q_ws, c.st_ws, c.part, c.tickets, c.err};
+    quant_kernel<<<grid, kThreads, smem, c.stream>>>(qa);
     return cudaGetLastError();
 }
 
-void set_quant_attr(int max_dyn_smem) {
-    cudaFuncSetAttribute(quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_dyn_smem);
-}
+cudaError_t set_quant_attr(int optin) { return allow_dyn_smem(quant_kernel, optin); }
 
 }  // namespace dfssm

@@ -8,9 +8,10 @@ order. For every element the fp32 rounding error is bounded by a few units of
 and the checks use eb_i = 2^-16 * T_i (about 250x that bound):
   * fp32 output: |y_gpu - y_ref| <= eb_i elementwise, and the normwise
     max-abs-rel error max|y_gpu - y_ref| / max|y_ref| <= 1e-3;
-  * bf16 output: y_gpu equals bf16_RNE(y_ref) except where y_ref lies within
-    eb_i of a bf16 rounding midpoint, where either neighbour is accepted; the
-    normwise error against bf16_RNE(y_ref) over the other elements is 0.
+  * bf16 output: y_gpu equals bf16_RNE(y_ref), except where bf16_RNE(y_ref - eb_i)
+    and bf16_RNE(y_ref + eb_i) differ (y_ref near a rounding midpoint), where any
+    bf16 value between those two is accepted; the normwise error against
+    bf16_RNE(y_ref) over the other elements is 0.
 Integer results (q, s_x, sum terms acc and h) must match bit for bit.
 """
 from __future__ import annotations
@@ -100,12 +101,15 @@ def check_y(y_gpu, y_ref, eb, y_dtype):
         return dict(normwise=e, ambiguous=0)
     ref_b = oracle.f64_to_bf16(y_ref)
     exact = y_gpu == ref_b
-    # elements whose exact value is within eb of a bf16 midpoint: either neighbour is fine
+    # The kernel rounds an fp32 value within eb of y_ref, and rounding is monotone, so its
+    # bf16 result lies between bf16(y_ref - eb) and bf16(y_ref + eb). Where those differ
+    # (y_ref near a midpoint, or eb wider than an ulp after cancellation) any value in
+    # that range is correct.
     lo = oracle.bf16_bits_to_f64(oracle.f64_to_bf16(y_ref - eb))
     hi = oracle.bf16_bits_to_f64(oracle.f64_to_bf16(y_ref + eb))
     amb = lo != hi
     got = oracle.bf16_bits_to_f64(y_gpu)
-    ok_amb = amb & ((got == lo) | (got == hi))
+    ok_amb = amb & (got >= lo) & (got <= hi)
     bad = ~(exact | ok_amb)
     assert not bad.any(), (f"{bad.sum()} bf16 outputs differ from bf16(y_ref) "
                            f"(first at {np.argwhere(bad)[0]}: got {got[bad][0]!r}, "
