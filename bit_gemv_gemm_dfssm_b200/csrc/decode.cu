@@ -27,7 +27,10 @@
 //  * These bytes are the u8 A operand of the warp MMA m16n8k32 (u8 x s8 -> s32),
 //    loaded with ldmatrix.x4 straight from the staged bits; the int8
 //    activations in the matching permuted column order (byte 4p + i of a
-//    32-column group = column 8i + p) are the s8 B operand, tokens = N.
+//    32-column group = column 8i + p) are the s8 B operand, tokens = N. In
+//    shared memory each 256-column group of a token row is laid out so that
+//    thread c of a quad reads its 16 B-fragment words with four 16-byte loads
+//    as (b0, b1) register pairs, one pair per bit position p.
 //  * One accumulator set per p, so set p sums 2^p * S_p exactly;
 //    S1 = sum_p D_p / 2^p = sum_{bit = 1} q, and acc = 2 * S1 - sum_j q
 //    (a +-1 weight is 2b - 1).
@@ -45,7 +48,10 @@ namespace {
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr int kChunkBytes = 128;   // sign bytes per row per k-chunk (1024 columns)
-constexpr int kTokPad = 16;        // q row stride = d_in + 16 (= 16 mod 128: conflict-free B reads)
+constexpr int kTokPad = 64;        // q row stride = round_up(d_in, 256) + 64 (= 64 mod 128: conflict-free B reads)
+
+// every 256-column group of a staged q row takes 256 bytes, even a half-filled last one
+__host__ __device__ __forceinline__ int q_stride(int d_in) { return ((d_in + 255) & ~255) + kTokPad; }
 constexpr int kStages = 3;
 constexpr int kMaxTok = 16;
 
@@ -146,9 +152,16 @@ __device__ __forceinline__ void issue_step(const Cursor& c, const Lin& L, uint8_
     const int nrows = min(R, L.d_out - row0);
     const int nch = min(kChunkBytes, L.rb - kChunkBytes * c.kc) >> 4;   // 1..8 16-byte chunks
     const uint8_t* src = L.sign + (int64_t)row0 * L.rb + kChunkBytes * c.kc;
-    for (int ci = threadIdx.x; ci < nrows * 8; ci += kThreads) {
-        const int r = ci >> 3, j = ci & 7;
-        if (j < nch) ptx::cp_async16(slot + r * kChunkBytes + 16 * ((j + r) & 7), src + (int64_t)r * L.rb + 16 * j);
+    // thread t copies 16-byte chunk j = t % 8 of rows t / 8, t / 8 + 16, ...; rows step by 16,
+    // so the rotated slot position (j + r) mod 8 is the same for all of them
+    const int j = threadIdx.x & 7;
+    int r = threadIdx.x >> 3;
+    if (j < nch) {
+        uint8_t* dst = slot + r * kChunkBytes + 16 * ((j + r) & 7);
+        const uint8_t* s0 = src + (int64_t)r * L.rb + 16 * j;
+        const int64_t sstep = (int64_t)(kThreads / 8) * L.rb;
+        for (; r < nrows; r += kThreads / 8, dst += (kThreads / 8) * kChunkBytes, s0 += sstep)
+            ptx::cp_async16(dst, s0);
     }
     if (c.kc == L.nchunks - 1) {
         uint8_t* par = slot + R * kChunkBytes;
@@ -161,6 +174,18 @@ __device__ __forceinline__ void issue_step(const Cursor& c, const Lin& L, uint8_
         for (int r = threadIdx.x; r < nrows; r += kThreads)
             ptx::cp_async16(par + 8 * R + 16 * r, L.wa + (int64_t)(row0 + r) * kRank);
     }
+}
+
+// Shared-memory position of q for column 32 gg + 8 i + p of a token row (gg: 32-column
+// group, i = 0..3, p = bit position). The 256-column group G = gg / 8 occupies 256
+// bytes; thread c = gg % 4 of an MMA quad owns 64 of them, holding for each p the
+// word of group gg (w = 0, B fragment b0) next to the word of group gg + 4 (w = 1,
+// b1). Logical 16-byte chunk k = p / 2 of that block is stored at (k + c) mod 4, so
+// the 8 lanes of a quarter-warp hit 8 different bank groups (with a token stride of
+// 64 mod 128).
+__device__ __forceinline__ int q_pos(int gg, int i, int p) {
+    const int G = gg >> 3, c = gg & 3, w = (gg >> 2) & 1;
+    return 256 * G + 64 * c + 16 * (((p >> 1) + c) & 3) + 8 * (p & 1) + 4 * w + i;
 }
 
 struct TokShared {
@@ -177,7 +202,7 @@ struct TokShared {
 __device__ void quantise_into_smem(const Lin& L, int m, uint8_t* q_s, TokShared& ts) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int n8 = L.d_in >> 3;                      // 8-column chunks per row
-    const int qstride = L.d_in + kTokPad;
+    const int qstride = q_stride(L.d_in);
     for (int t = 0; t < m; ++t) {
         float am = 0.0f;
         for (int ch = tid; ch < n8; ch += kThreads) {
@@ -201,14 +226,14 @@ __device__ void quantise_into_smem(const Lin& L, int m, uint8_t* q_s, TokShared&
         for (int ch = tid; ch < n8; ch += kThreads) {
             const uint4 v = *reinterpret_cast<const uint4*>(L.x + (int64_t)t * L.d_in + 8 * ch);
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            // columns 8 ch + p, p = 0..7 -> permuted byte 32 (ch / 4) + 4 p + ch % 4
-            uint8_t* dst = q_s + t * qstride + 32 * (ch >> 2) + (ch & 3);
+            // columns 8 ch + p (p = 0..7) of 32-column group gg = ch / 4 (i = ch % 4)
+            uint8_t* row = q_s + t * qstride;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int q0 = quant1(bf16_lo(w[i]), inv, zero), q1 = quant1(bf16_hi(w[i]), inv, zero);
                 sum += q0 + q1;
-                dst[4 * (2 * i)] = (uint8_t)q0;
-                dst[4 * (2 * i + 1)] = (uint8_t)q1;
+                row[q_pos(ch >> 2, ch & 3, 2 * i)] = (uint8_t)q0;
+                row[q_pos(ch >> 2, ch & 3, 2 * i + 1)] = (uint8_t)q1;
             }
         }
 #pragma unroll
@@ -299,14 +324,17 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
                         for (int r = 0; r < 4; ++r) D[rt][nt][p][r] = 0;
         }
         if (active) {
-            const int qstride = L.d_in + kTokPad;
+            const int qstride = q_stride(L.d_in);
             const int cb = min(kChunkBytes, L.rb - kChunkBytes * cw.c.kc);
             const int ng = (cb + 31) >> 5;                 // groups of 256 columns in this chunk
             const uint32_t slot_s = ptx::smem_u32(slot);
+            // B rows: tokens nt * 8 + g; lanes past m read token 0 (their MMA columns are never stored)
             const uint8_t* qrow[NT];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-                qrow[nt] = q_s + (nt * 8 + g) * qstride + 32 * (32 * cw.c.kc + c);
+            for (int nt = 0; nt < NT; ++nt) {
+                const int tk = nt * 8 + g;
+                qrow[nt] = q_s + (tk < m ? tk : 0) * qstride + 256 * (4 * cw.c.kc) + 64 * c;
+            }
 #pragma unroll
             for (int G = 0; G < 4; ++G) {
                 if (G < ng) {
@@ -318,32 +346,16 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
                         const int chunk = 2 * G + lm_hi;
                         ptx::ldmatrix_x4(slot_s + row * kChunkBytes + 16 * ((chunk + row) & 7), A[rt][0],
                                          A[rt][1], A[rt][2], A[rt][3]);
+                        // half group: zero A slots 16..31, so whatever b1 holds there adds nothing
                         if (half) { A[rt][2] = 0u; A[rt][3] = 0u; }
                     }
-                    // B: thread (g, c) holds token g's q for words c (b0) and 4 + c (b1) of the group
-                    uint32_t bq[NT][2][8];
+                    // B: chunk k (bit positions 2k, 2k+1) = (b0, b1) of p = 2k, then of p = 2k + 1
+                    uint4 bq[NT][4];
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        if (nt * 8 + g < m) {
-                            const uint8_t* qb = qrow[nt] + 256 * G;
-                            const uint4 v0 = *reinterpret_cast<const uint4*>(qb);
-                            const uint4 v1 = *reinterpret_cast<const uint4*>(qb + 16);
-                            bq[nt][0][0] = v0.x; bq[nt][0][1] = v0.y; bq[nt][0][2] = v0.z; bq[nt][0][3] = v0.w;
-                            bq[nt][0][4] = v1.x; bq[nt][0][5] = v1.y; bq[nt][0][6] = v1.z; bq[nt][0][7] = v1.w;
-                            if (!half) {
-                                const uint4 v2 = *reinterpret_cast<const uint4*>(qb + 128);
-                                const uint4 v3 = *reinterpret_cast<const uint4*>(qb + 144);
-                                bq[nt][1][0] = v2.x; bq[nt][1][1] = v2.y; bq[nt][1][2] = v2.z; bq[nt][1][3] = v2.w;
-                                bq[nt][1][4] = v3.x; bq[nt][1][5] = v3.y; bq[nt][1][6] = v3.z; bq[nt][1][7] = v3.w;
-                            } else {
+                    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                                for (int p = 0; p < 8; ++p) bq[nt][1][p] = 0u;
-                            }
-                        } else {
-#pragma unroll
-                            for (int p = 0; p < 8; ++p) { bq[nt][0][p] = 0u; bq[nt][1][p] = 0u; }
-                        }
-                    }
+                        for (int k = 0; k < 4; ++k)
+                            bq[nt][k] = *reinterpret_cast<const uint4*>(qrow[nt] + 256 * G + 16 * ((k + c) & 3));
 #pragma unroll
                     for (int p = 0; p < 8; ++p) {
                         const uint32_t msk = 0x01010101u << p;
@@ -352,8 +364,11 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
                             const uint32_t a0 = A[rt][0] & msk, a1 = A[rt][1] & msk;
                             const uint32_t a2 = A[rt][2] & msk, a3 = A[rt][3] & msk;
 #pragma unroll
-                            for (int nt = 0; nt < NT; ++nt)
-                                ptx::mma_u8s8(D[rt][nt][p], a0, a1, a2, a3, bq[nt][0][p], bq[nt][1][p]);
+                            for (int nt = 0; nt < NT; ++nt) {
+                                const uint4& v = bq[nt][p >> 1];
+                                if (p & 1) ptx::mma_u8s8(D[rt][nt][p], a0, a1, a2, a3, v.z, v.w);
+                                else       ptx::mma_u8s8(D[rt][nt][p], a0, a1, a2, a3, v.x, v.y);
+                            }
                         }
                     }
                 }
@@ -435,7 +450,7 @@ Geometry geometry(int m, int max_d_in) {
     constexpr int R = 16 * RT * kWarps;
     Geometry g;
     g.slot_bytes = (R * kChunkBytes + R * (4 + 4 + kRank) + 127) & ~127;
-    g.q_region = (m * (max_d_in + kTokPad) + 127) & ~127;
+    g.q_region = (m * q_stride(max_d_in) + 127) & ~127;
     g.smem = ((sizeof(TokShared) + 127) & ~(size_t)127) + g.q_region + (size_t)kStages * g.slot_bytes;
     return g;
 }

@@ -220,7 +220,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
                     const int s = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
                     ++it;
-                    if (!ptx::mbar_wait(&empty[s], ph ^ 1u)) { set_err(a.err, DFSSM_DEVERR_TIMEOUT); *abort_flag = 1; ok = false; break; }
+                    // one lane polls, the warp follows
+                    bool got = true;
+                    if ((threadIdx.x & 31) == 0) got = ptx::mbar_wait(&empty[s], ph ^ 1u);
+                    got = __shfl_sync(0xffffffffu, got, 0);
+                    __syncwarp();
+                    if (!got) { if ((threadIdx.x & 31) == 0) { set_err(a.err, DFSSM_DEVERR_TIMEOUT); *abort_flag = 1; } ok = false; break; }
                     uint8_t* dst = sA + s * A_STAGE + rrow;
                     const uint32_t wv[4] = {bits.x, bits.y, bits.z, bits.w};
 #pragma unroll
@@ -253,6 +258,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
             const dfssm_stack_entry& e = entry_at(a.entries, a.single, tc.lin);
             const int o = tc.row0 + r;
             const bool valid = o < d.d_out && entry_ptrs_ok(e);
+            // entry fields in registers: the stores below must not force reloads
+            void* const y_ptr = e.y;
+            int32_t* const dbg_acc = e.dbg.acc;
+            const bool y_bf16 = d.y_dtype == DFSSM_BF16;
+            const int d_out = d.d_out;
             float alpha = 0.f, sa = 0.f;
             WaRow wa = wa_row_from_int4(make_int4(0, 0, 0, 0));
             if (valid) {
@@ -284,7 +294,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
 
             const int buf = tcount & 1;
             const uint32_t acc_ph = (uint32_t)(tcount >> 1) & 1u;
-            const bool got = __all_sync(0xffffffffu, ptx::mbar_wait(&acc_full[buf], acc_ph));
+            bool got = true;
+            if (lane == 0) got = ptx::mbar_wait(&acc_full[buf], acc_ph);
+            got = __shfl_sync(0xffffffffu, got, 0);
+            __syncwarp();
             if (!got) {
                 if (lane == 0) { set_err(a.err, DFSSM_DEVERR_TIMEOUT); *abort_flag = 1; }
                 break;
@@ -301,36 +314,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
                 ptx::tmem_ld_wait();
                 const TokStats* stc = reinterpret_cast<const TokStats*>(stat_buf + (ch & 1) * STAT_CHUNK);
                 const int t0c = tok_base + 16 * ch;
-                if (t0c < a.m) {
+                if (t0c < a.m && valid) {
                     const int nj = min(16, a.m - t0c);
-                    const int64_t base_idx = (int64_t)t0c * d.d_out + o;
-                    if (nj == 16 && valid) {
-                        // full chunk: no per-token checks
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const TokStats& st = stc[j];
-                            const int acc = 2 * (int)v[j] - st.sumq;
-                            const float y = dequant(st.sx, alpha, sa, acc, lora_dot(wa, st.u));
-                            const int64_t idx = base_idx + (int64_t)j * d.d_out;
-                            if (d.y_dtype == DFSSM_BF16)
-                                reinterpret_cast<uint16_t*>(e.y)[idx] = f32_to_bf16_bits(y);
-                            else
-                                reinterpret_cast<float*>(e.y)[idx] = y;
-                            if (e.dbg.acc) e.dbg.acc[idx] = acc;
-                        }
-                    } else if (valid) {
+                    // element (t0c + j, o) of y / acc: base + j * d_out (32-bit offsets inside a chunk)
+                    const int64_t base_idx = (int64_t)t0c * d_out + o;
+                    if (y_bf16) {
+                        uint16_t* yb = reinterpret_cast<uint16_t*>(y_ptr) + base_idx;
+                        int32_t* ab = dbg_acc ? dbg_acc + base_idx : nullptr;
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             if (j >= nj) break;
                             const TokStats& st = stc[j];
                             const int acc = 2 * (int)v[j] - st.sumq;
-                            const float y = dequant(st.sx, alpha, sa, acc, lora_dot(wa, st.u));
-                            const int64_t idx = base_idx + (int64_t)j * d.d_out;
-                            if (d.y_dtype == DFSSM_BF16)
-                                reinterpret_cast<uint16_t*>(e.y)[idx] = f32_to_bf16_bits(y);
-                            else
-                                reinterpret_cast<float*>(e.y)[idx] = y;
-                            if (e.dbg.acc) e.dbg.acc[idx] = acc;
+                            yb[j * d_out] = f32_to_bf16_bits(dequant(st.sx, alpha, sa, acc, lora_dot(wa, st.u)));
+                            if (ab) ab[j * d_out] = acc;
+                        }
+                    } else {
+                        float* yf = reinterpret_cast<float*>(y_ptr) + base_idx;
+                        int32_t* ab = dbg_acc ? dbg_acc + base_idx : nullptr;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            if (j >= nj) break;
+                            const TokStats& st = stc[j];
+                            const int acc = 2 * (int)v[j] - st.sumq;
+                            yf[j * d_out] = dequant(st.sx, alpha, sa, acc, lora_dot(wa, st.u));
+                            if (ab) ab[j * d_out] = acc;
                         }
                     }
                 }

@@ -42,7 +42,7 @@ constexpr int kTok = 16;              // tokens per round
 constexpr int kTokPerBlock = 64;      // rounds per block: 4
 
 struct QuantRed {
-    float amax[kWarps][kTok];
+    unsigned int amax[kTok];     // fp32 bits of a non-negative max (order-preserving as unsigned)
     int sumq[kWarps][kTok];
     int h[kWarps][kTok][kRank];
     float inv[kTok];
@@ -144,27 +144,22 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__
     for (int t0 = tb0; t0 < tb1; t0 += kTok) {
         const int nt = min(kTok, tb1 - t0);
 
-        // ---- pass 1: amax. lane l covers token l/2, columns 16*(l&1) .. +15 of each k-block
+        // ---- pass 1: amax over (token, 16-column piece) items spread over all threads
+        if (tid < kTok) red.amax[tid] = 0u;
+        __syncthreads();
         {
-            const int tk = lane >> 1, hf = lane & 1;
-            float am = 0.0f;
-            if (tk < nt) {
-                const uint16_t* row = xg + (int64_t)(t0 + tk) * d_in + 16 * hf;
+            const int pieces = d_in >> 4;
 #pragma unroll 4
-                for (int kb = warp; kb < nkb; kb += kWarps) {
-                    const uint4* p = reinterpret_cast<const uint4*>(row + 32 * kb);
-                    am = absmax8(p[0], am);
-                    am = absmax8(p[1], am);
-                }
+            for (int it = tid; it < nt * pieces; it += kThreads) {
+                const int tk = it / pieces, pc = it - tk * pieces;
+                const uint4* p = reinterpret_cast<const uint4*>(xg + (int64_t)(t0 + tk) * d_in + 16 * pc);
+                const float am = absmax8(p[1], absmax8(p[0], 0.0f));
+                atomicMax(&red.amax[tk], __float_as_uint(am));
             }
-            am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
-            if (hf == 0) red.amax[warp][tk] = am;
         }
         __syncthreads();
         if (tid < kTok) {
-            float am = 0.0f;
-#pragma unroll
-            for (int w = 0; w < kWarps; ++w) am = fmaxf(am, red.amax[w][tid]);
+            const float am = __uint_as_float(red.amax[tid]);
             if (tid < nt && !isfinite(am)) atomicOr(err, DFSSM_DEVERR_NONFINITE);
             red.inv[tid] = quant_inv(am);
             red.sx[tid] = quant_sx(am);
