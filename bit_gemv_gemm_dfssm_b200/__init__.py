@@ -15,7 +15,9 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libdfssm.so")
+# DFSSM_LIBRARY may name another build of the same library (for example a copy built
+# with different tile sizes); by default the in-tree build is used.
+LIB_PATH = os.environ.get("DFSSM_LIBRARY") or os.path.join(_HERE, "libdfssm.so")
 
 DFSSM_OK = 0
 DFSSM_ERR_INVALID_ARG = 1
@@ -37,7 +39,9 @@ RANK = 16
 EXPORTS = (
     "dfssm_linear_plan", "dfssm_plan_destroy", "dfssm_pack_sign", "dfssm_linear_fwd",
     "dfssm_linear_stack_fwd", "dfssm_plan_check", "dfssm_plan_workspace_bytes", "dfssm_status_string",
+    "dfssm_linear_fwd_noalloc",
 )
+DFSSM_NOALLOC_MAX_M = 16
 
 
 class DfssmError(RuntimeError):
@@ -81,6 +85,8 @@ def _load():
     lib.dfssm_linear_fwd.argtypes = [vp, i32, ctypes.POINTER(LinearWeights), vp, i32, vp,
                                      ctypes.POINTER(Debug), vp]
     lib.dfssm_linear_stack_fwd.argtypes = [vp, vp, i32, i32, vp]
+    lib.dfssm_linear_fwd_noalloc.argtypes = [ctypes.POINTER(LinearDesc), ctypes.POINTER(LinearWeights), vp, i32,
+                                             vp, vp]
     lib.dfssm_plan_check.argtypes = [vp, u32p]
     lib.dfssm_plan_workspace_bytes.argtypes = [vp, ctypes.POINTER(ctypes.c_size_t)]
     lib.dfssm_status_string.restype = ctypes.c_char_p
@@ -140,6 +146,15 @@ def dfssm_linear_fwd(plan: int, desc_index: int, w: LinearWeights, x_ptr: int, m
 
 def dfssm_linear_stack_fwd(plan: int, entries_dev_ptr: int, n_entries: int, m: int, stream: int = 0) -> None:
     _check(lib().dfssm_linear_stack_fwd(plan, entries_dev_ptr, n_entries, m, stream), "dfssm_linear_stack_fwd")
+
+
+def dfssm_linear_fwd_noalloc(desc, w: LinearWeights, x_ptr: int, m: int, y_ptr: int, stream: int = 0) -> None:
+    """One linear, m <= 16 tokens, without any device allocation (fixed device scratch)."""
+    if not isinstance(desc, LinearDesc):
+        d_in, d_out, y_dtype = desc
+        desc = LinearDesc(d_in, d_out, RANK, m, y_dtype, 0)
+    _check(lib().dfssm_linear_fwd_noalloc(ctypes.byref(desc), ctypes.byref(w), x_ptr, m, y_ptr, stream),
+           "dfssm_linear_fwd_noalloc")
 
 
 def dfssm_plan_check(plan: int):

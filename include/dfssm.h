@@ -159,6 +159,27 @@ dfssm_status dfssm_linear_fwd(dfssm_plan plan, int32_t desc_index, const dfssm_l
 dfssm_status dfssm_linear_stack_fwd(dfssm_plan plan, const dfssm_stack_entry* entries_dev,
                                     int32_t n_entries, int32_t m, void* stream);
 
+/* The layer for one linear and a few tokens, allocating nothing.
+ * No counterpart in the paper: this is for callers that cannot call cudaMalloc
+ * (code running while a CUDA graph is being captured, allocators that must not
+ * be re-entered, hosts with a fixed memory budget). It needs no plan: its
+ * scratch (per-token scalars, split partials, int8 activations, descriptor,
+ * error word) is a file-scope device array of about 140 KB that every GPU using
+ * this library keeps until the process exits.
+ * desc: HOST pointer to the linear's shape (rank 16, 128 <= d_in <= 8192,
+ * d_in % 128 == 0; max_m is ignored); w: HOST struct of device pointers;
+ * x: m x d_in bf16 (device); y: m x d_out of desc->y_dtype (device);
+ * 1 <= m <= DFSSM_NOALLOC_MAX_M. Larger shapes return
+ * DFSSM_ERR_UNSUPPORTED_SHAPE and enqueue nothing. All calls share the one
+ * array, so calls that overlap on the GPU (unordered streams) race; the array
+ * keeps the last call's contents, and what must start at zero is reset by the
+ * kernels themselves. The first call on each device looks up the array's device
+ * address and sets kernel attributes: make it before any stream capture.
+ * Device-side error conditions are not reported by this entry point. */
+#define DFSSM_NOALLOC_MAX_M 16
+dfssm_status dfssm_linear_fwd_noalloc(const dfssm_linear_desc* desc, const dfssm_linear_weights* w,
+                                      const void* x, int32_t m, void* y, void* stream);
+
 /* Synchronise the plan's device, read and clear its error word.
  * Returns DFSSM_OK or DFSSM_ERR_DEVICE_CHECK (*bits, if not NULL, gets the word). */
 dfssm_status dfssm_plan_check(dfssm_plan plan, uint32_t* bits);
