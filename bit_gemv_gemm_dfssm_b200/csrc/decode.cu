@@ -47,12 +47,20 @@ namespace {
 
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
-constexpr int kChunkBytes = 128;   // sign bytes per row per k-chunk (1024 columns)
+#ifndef DFSSM_DECODE_CHUNK_BYTES
+#define DFSSM_DECODE_CHUNK_BYTES 128
+#endif
+#ifndef DFSSM_DECODE_STAGES
+#define DFSSM_DECODE_STAGES 3
+#endif
+constexpr int kChunkBytes = DFSSM_DECODE_CHUNK_BYTES;   // sign bytes per row per k-chunk (8 columns per byte)
+constexpr int kChunkJ = kChunkBytes / 16;                // 16-byte pieces per row per chunk
+constexpr int kGroups = kChunkBytes / 32;                // 256-column groups per chunk
 constexpr int kTokPad = 64;        // q row stride = round_up(d_in, 256) + 64 (= 64 mod 128: conflict-free B reads)
 
 // every 256-column group of a staged q row takes 256 bytes, even a half-filled last one
 __host__ __device__ __forceinline__ int q_stride(int d_in) { return ((d_in + 255) & ~255) + kTokPad; }
-constexpr int kStages = 3;
+constexpr int kStages = DFSSM_DECODE_STAGES;
 constexpr int kMaxTok = 16;
 
 struct DecodeArgs {
@@ -89,7 +97,7 @@ __device__ __forceinline__ void load_lin(const DecodeArgs& a, int l, Lin& L) {
     L.d_in = d.d_in;
     L.d_out = d.d_out;
     L.rb = d.d_in >> 3;
-    L.nchunks = (d.d_in + 1023) >> 10;
+    L.nchunks = (d.d_in / 8 + kChunkBytes - 1) / kChunkBytes;
     L.nblocks = (d.d_out + R - 1) / R;
     L.y_dtype = d.y_dtype;
     L.byte_rel = d.byte_begin - a.desc[0].byte_begin;
@@ -150,18 +158,17 @@ __device__ __forceinline__ void issue_step(const Cursor& c, const Lin& L, uint8_
     if (!L.ok) return;                    // flagged by the quantisation kernel
     const int row0 = c.b * R;
     const int nrows = min(R, L.d_out - row0);
-    const int nch = min(kChunkBytes, L.rb - kChunkBytes * c.kc) >> 4;   // 1..8 16-byte chunks
+    const int nch = min(kChunkBytes, L.rb - kChunkBytes * c.kc) >> 4;   // 16-byte pieces in this chunk
     const uint8_t* src = L.sign + (int64_t)row0 * L.rb + kChunkBytes * c.kc;
-    // thread t copies 16-byte chunk j = t % 8 of rows t / 8, t / 8 + 16, ...; rows step by 16,
-    // so the rotated slot position (j + r) mod 8 is the same for all of them
-    const int j = threadIdx.x & 7;
-    int r = threadIdx.x >> 3;
+    // thread t copies 16-byte piece j = t % kChunkJ of rows t / kChunkJ + k * kRowStep
+    constexpr int kRowStep = kThreads / kChunkJ;
+    const int j = threadIdx.x % kChunkJ;
+    int r = threadIdx.x / kChunkJ;
     if (j < nch) {
-        uint8_t* dst = slot + r * kChunkBytes + 16 * ((j + r) & 7);
         const uint8_t* s0 = src + (int64_t)r * L.rb + 16 * j;
-        const int64_t sstep = (int64_t)(kThreads / 8) * L.rb;
-        for (; r < nrows; r += kThreads / 8, dst += (kThreads / 8) * kChunkBytes, s0 += sstep)
-            ptx::cp_async16(dst, s0);
+        const int64_t sstep = (int64_t)kRowStep * L.rb;
+        for (; r < nrows; r += kRowStep, s0 += sstep)
+            ptx::cp_async16(slot + r * kChunkBytes + 16 * ((j + r) % kChunkJ), s0);
     }
     if (c.kc == L.nchunks - 1) {
         uint8_t* par = slot + R * kChunkBytes;
@@ -326,52 +333,64 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
         if (active) {
             const int qstride = q_stride(L.d_in);
             const int cb = min(kChunkBytes, L.rb - kChunkBytes * cw.c.kc);
-            const int ng = (cb + 31) >> 5;                 // groups of 256 columns in this chunk
             const uint32_t slot_s = ptx::smem_u32(slot);
+            // ldmatrix row addresses: row r's 16-byte piece j sits at (j + r) mod kChunkJ; rows
+            // of a tile are 8-aligned, so the rotation depends on (lane % 8) only
+            const int rot = (lm_row & 7) + lm_hi;
+            uint32_t a_addr[RT][kGroups];
+#pragma unroll
+            for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+                for (int G = 0; G < kGroups; ++G)
+                    a_addr[rt][G] = slot_s + (wrow0 + 16 * rt + lm_row) * kChunkBytes + 16 * ((2 * G + rot) % kChunkJ);
             // B rows: tokens nt * 8 + g; lanes past m read token 0 (their MMA columns are never stored)
-            const uint8_t* qrow[NT];
+            const uint8_t* qk[NT][4];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 const int tk = nt * 8 + g;
-                qrow[nt] = q_s + (tk < m ? tk : 0) * qstride + 256 * (4 * cw.c.kc) + 64 * c;
-            }
+                const uint8_t* qrow = q_s + (tk < m ? tk : 0) * qstride + 256 * (kGroups * cw.c.kc) + 64 * c;
 #pragma unroll
-            for (int G = 0; G < 4; ++G) {
-                if (G < ng) {
-                    const bool half = (cb - 32 * G) == 16;     // only 128 columns: words 4..7 absent
-                    uint32_t A[RT][4];
+                for (int k = 0; k < 4; ++k) qk[nt][k] = qrow + 16 * ((k + c) & 3);
+            }
+            auto group = [&](int G, bool half) {
+                uint32_t A[RT][4];
+#pragma unroll
+                for (int rt = 0; rt < RT; ++rt) {
+                    ptx::ldmatrix_x4(a_addr[rt][G], A[rt][0], A[rt][1], A[rt][2], A[rt][3]);
+                    // half group: zero A slots 16..31, so whatever b1 holds there adds nothing
+                    if (half) { A[rt][2] = 0u; A[rt][3] = 0u; }
+                }
+                // B: chunk k (bit positions 2k, 2k+1) = (b0, b1) of p = 2k, then of p = 2k + 1
+                uint4 bq[NT][4];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) bq[nt][k] = *reinterpret_cast<const uint4*>(qk[nt][k] + 256 * G);
+#pragma unroll
+                for (int p = 0; p < 8; ++p) {
+                    const uint32_t msk = 0x01010101u << p;
 #pragma unroll
                     for (int rt = 0; rt < RT; ++rt) {
-                        const int row = wrow0 + 16 * rt + lm_row;
-                        const int chunk = 2 * G + lm_hi;
-                        ptx::ldmatrix_x4(slot_s + row * kChunkBytes + 16 * ((chunk + row) & 7), A[rt][0],
-                                         A[rt][1], A[rt][2], A[rt][3]);
-                        // half group: zero A slots 16..31, so whatever b1 holds there adds nothing
-                        if (half) { A[rt][2] = 0u; A[rt][3] = 0u; }
-                    }
-                    // B: chunk k (bit positions 2k, 2k+1) = (b0, b1) of p = 2k, then of p = 2k + 1
-                    uint4 bq[NT][4];
+                        const uint32_t a0 = A[rt][0] & msk, a1 = A[rt][1] & msk;
+                        const uint32_t a2 = A[rt][2] & msk, a3 = A[rt][3] & msk;
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            bq[nt][k] = *reinterpret_cast<const uint4*>(qrow[nt] + 256 * G + 16 * ((k + c) & 3));
-#pragma unroll
-                    for (int p = 0; p < 8; ++p) {
-                        const uint32_t msk = 0x01010101u << p;
-#pragma unroll
-                        for (int rt = 0; rt < RT; ++rt) {
-                            const uint32_t a0 = A[rt][0] & msk, a1 = A[rt][1] & msk;
-                            const uint32_t a2 = A[rt][2] & msk, a3 = A[rt][3] & msk;
-#pragma unroll
-                            for (int nt = 0; nt < NT; ++nt) {
-                                const uint4& v = bq[nt][p >> 1];
-                                if (p & 1) ptx::mma_u8s8(D[rt][nt][p], a0, a1, a2, a3, v.z, v.w);
-                                else       ptx::mma_u8s8(D[rt][nt][p], a0, a1, a2, a3, v.x, v.y);
-                            }
+                        for (int nt = 0; nt < NT; ++nt) {
+                            const uint4& v = bq[nt][p >> 1];
+                            if (p & 1) ptx::mma_u8s8(D[rt][nt][p], a0, a1, a2, a3, v.z, v.w);
+                            else       ptx::mma_u8s8(D[rt][nt][p], a0, a1, a2, a3, v.x, v.y);
                         }
                     }
                 }
+            };
+            if (cb == kChunkBytes) {
+                // full chunk: whole groups, straight-line code
+#pragma unroll
+                for (int G = 0; G < kGroups; ++G) group(G, false);
+            } else {
+                const int ng = (cb + 31) >> 5;             // groups of 256 columns in this chunk
+#pragma unroll
+                for (int G = 0; G < kGroups; ++G)
+                    if (G < ng) group(G, (cb - 32 * G) == 16);
             }
 
             // ---- epilogue after the block's last k-chunk
