@@ -46,13 +46,15 @@ struct dfssm_plan_s {
     uint32_t* err = nullptr;
     int* part = nullptr;
     unsigned int* tickets = nullptr;
-    CUtensorMap* tmaps = nullptr;
+    CUtensorMap* tmaps = nullptr;       // prefill: activation rows of each linear
+    CUtensorMap* sign_tmpl = nullptr;   // decode: sign rows of each linear, address set on the device
+    CUtensorMap* map_slots = nullptr;   // decode: per-CTA tensor maps edited on the device
     size_t ws_bytes = 0;
 };
 
 namespace {
 
-constexpr int kDecodeMaxM = 16;
+constexpr int kDecodeMaxM = kImgTokens;   // the quantisation kernel writes the decode image up to here
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -93,21 +95,6 @@ dfssm_status check_dbg(const dfssm_debug& g) {
     return DFSSM_OK;
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (fn) return fn;
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-        return nullptr;
-    fn = reinterpret_cast<EncodeTiledFn>(p);
-    return fn;
-}
 
 void free_plan(dfssm_plan_s* p) {
     if (!p) return;
@@ -118,6 +105,8 @@ void free_plan(dfssm_plan_s* p) {
     if (p->part) cudaFree(p->part);
     if (p->tickets) cudaFree(p->tickets);
     if (p->tmaps) cudaFree(p->tmaps);
+    if (p->sign_tmpl) cudaFree(p->sign_tmpl);
+    if (p->map_slots) cudaFree(p->map_slots);
     delete p;
 }
 
@@ -166,30 +155,36 @@ dfssm_status dfssm_linear_plan(const dfssm_linear_desc* descs, int n_descs, dfss
     p->n = n_descs;
     p->hdesc.resize(n_descs);
     int64_t q_bytes = 0, st_count = 0, sign_bytes = 0;
-    int32_t blk = 0, rt = 0;
+    int32_t rt = 0;
     for (int i = 0; i < n_descs; ++i) {
         DevDesc& d = p->hdesc[i];
+        std::memset(&d, 0, sizeof(d));
         d.d_in = descs[i].d_in;
         d.d_out = descs[i].d_out;
         d.y_dtype = descs[i].y_dtype;
         d.max_m = descs[i].max_m;
+        d.qrow = seg_qrow(d.d_in);
+        // every region is a multiple of 256 bytes, so every offset stays 256-byte aligned
+        d.dq_off = q_bytes;
+        q_bytes += (int64_t)kImgTokens * d.qrow;
         d.q_off = q_bytes;
+        if (d.max_m > kDecodeMaxM) q_bytes += (int64_t)d.max_m * d.qrow;
         d.st_off = st_count;
-        d.blk_begin = blk;
         d.rt_begin = rt;
         d.byte_begin = sign_bytes;
         sign_bytes += (int64_t)d.d_out * (d.d_in / 8);
-        q_bytes += (int64_t)d.max_m * d.d_in;       // d_in % 128 == 0 keeps every region 128-byte aligned
         st_count += d.max_m;
-        blk += (d.d_out + 63) / 64;
         rt += (d.d_out + 127) / 128;
     }
+    const int n_slots = p->sm_count * decode_map_slots();
     cudaError_t e = cudaSuccess;
     e = cudaMalloc(&p->ddesc, sizeof(DevDesc) * n_descs);
     if (e == cudaSuccess) e = cudaMalloc(&p->q_ws, (size_t)q_bytes);
     if (e == cudaSuccess) e = cudaMalloc(&p->st_ws, sizeof(TokStats) * (size_t)st_count);
     if (e == cudaSuccess) e = cudaMalloc(&p->err, 16);
     if (e == cudaSuccess) e = cudaMalloc(&p->tmaps, sizeof(CUtensorMap) * n_descs);
+    if (e == cudaSuccess) e = cudaMalloc(&p->sign_tmpl, sizeof(CUtensorMap) * n_descs);
+    if (e == cudaSuccess) e = cudaMalloc(&p->map_slots, sizeof(CUtensorMap) * n_slots);
     const size_t part_bytes = sizeof(int) * (size_t)n_descs * kMaxSplits * kPartTok * 20;
     if (e == cudaSuccess) e = cudaMalloc(&p->part, part_bytes);
     if (e == cudaSuccess) e = cudaMalloc(&p->tickets, sizeof(unsigned int) * n_descs);
@@ -199,25 +194,35 @@ dfssm_status dfssm_linear_plan(const dfssm_linear_desc* descs, int n_descs, dfss
         return e == cudaErrorMemoryAllocation ? DFSSM_ERR_NO_MEMORY : DFSSM_ERR_CUDA;
     }
     p->ws_bytes = sizeof(DevDesc) * n_descs + (size_t)q_bytes + sizeof(TokStats) * st_count + 16 +
-                  sizeof(CUtensorMap) * n_descs + part_bytes + sizeof(unsigned int) * n_descs;
+                  sizeof(CUtensorMap) * (2 * n_descs + n_slots) + part_bytes + sizeof(unsigned int) * n_descs;
 
-    // tensor maps over each linear's int8 activation rows (prefill B operand)
-    std::vector<CUtensorMap> tm(n_descs);
+    // prefill: tensor maps over each linear's activation rows (B operand, 128-byte swizzle);
+    // decode: tensor maps over each linear's sign rows with a placeholder address (the
+    // kernel sets the address of the call's sign tensor)
+    std::vector<CUtensorMap> tm(n_descs), sm(n_descs);
     std::memset(tm.data(), 0, sizeof(CUtensorMap) * n_descs);
+    std::memset(sm.data(), 0, sizeof(CUtensorMap) * n_descs);
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) { free_plan(p); return DFSSM_ERR_CUDA; }
     for (int i = 0; i < n_descs; ++i) {
         const DevDesc& d = p->hdesc[i];
-        cuuint64_t dims[2] = {(cuuint64_t)d.d_in, (cuuint64_t)d.max_m};
-        cuuint64_t strides[1] = {(cuuint64_t)d.d_in};
-        cuuint32_t box[2] = {(cuuint32_t)prefill_box_bytes(), (cuuint32_t)prefill_box_tokens()};
-        cuuint32_t estr[2] = {1, 1};
-        CUresult r = enc(&tm[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, p->q_ws + d.q_off, dims, strides, box, estr,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) { free_plan(p); return DFSSM_ERR_CUDA; }
+        if (d.max_m > kDecodeMaxM) {
+            cuuint64_t dims[2] = {(cuuint64_t)d.qrow, (cuuint64_t)d.max_m};
+            cuuint64_t strides[1] = {(cuuint64_t)d.qrow};
+            cuuint32_t box[2] = {(cuuint32_t)prefill_box_bytes(), (cuuint32_t)prefill_box_tokens()};
+            cuuint32_t estr[2] = {1, 1};
+            CUresult r = enc(&tm[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, p->q_ws + d.q_off, dims, strides, box, estr,
+                             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            if (r != CUDA_SUCCESS) { free_plan(p); return DFSSM_ERR_CUDA; }
+        }
+        if (encode_sign_map(enc, &sm[i], p->q_ws, d.d_in, d.d_out) != CUDA_SUCCESS) {
+            free_plan(p);
+            return DFSSM_ERR_CUDA;
+        }
     }
     e = cudaMemcpy(p->tmaps, tm.data(), sizeof(CUtensorMap) * n_descs, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(p->sign_tmpl, sm.data(), sizeof(CUtensorMap) * n_descs, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(p->ddesc, p->hdesc.data(), sizeof(DevDesc) * n_descs, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemset(p->err, 0, 16);
     if (e == cudaSuccess) e = cudaMemset(p->tickets, 0, sizeof(unsigned int) * n_descs);
@@ -279,6 +284,9 @@ dfssm_status dfssm_linear_fwd(dfssm_plan plan, int32_t desc_index, const dfssm_l
     c.part = plan->part + (size_t)desc_index * kMaxSplits * kPartTok * 20;
     c.tickets = plan->tickets + desc_index;
     c.tmaps = plan->tmaps + desc_index;
+    c.sign_tmpl = plan->sign_tmpl + desc_index;
+    c.map_slots = plan->map_slots;
+    c.map_slot_ctas = plan->sm_count;
     c.max_d_in = hd.d_in;
     c.total_rows = hd.d_out;
     c.sm_count = plan->sm_count;
@@ -312,6 +320,9 @@ dfssm_status dfssm_linear_stack_fwd(dfssm_plan plan, const dfssm_stack_entry* en
     c.part = plan->part;
     c.tickets = plan->tickets;
     c.tmaps = plan->tmaps;
+    c.sign_tmpl = plan->sign_tmpl;
+    c.map_slots = plan->map_slots;
+    c.map_slot_ctas = plan->sm_count;
     c.max_d_in = max_d_in;
     c.total_rows = rows;
     c.sm_count = plan->sm_count;

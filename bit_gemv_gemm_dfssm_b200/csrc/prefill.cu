@@ -18,8 +18,10 @@
 //   warp 1      TMEM owner and MMA issuer: tcgen05.mma.kind::i8, M=128 rows,
 //               N=256 tokens, K=32 per instruction, 4 per 128-column block
 //   warps 4-7   bit expansion: each thread owns one weight row of the tile,
-//               loads 16 bytes of sign bits per k-block and writes 128 0/1 bytes
-//               into the K-major SWIZZLE_128B layout the MMA reads
+//               loads the 32 sign bytes of a 256-column segment and writes, per
+//               128-byte k-block (four bit planes of that segment, the activation
+//               order of dfssm_internal.cuh), 128 0/1 bytes into the K-major
+//               SWIZZLE_128B layout the MMA reads
 //   warps 8-15  epilogue: tcgen05.ld of its 32 TMEM lanes (= output rows) and
 //               half of the 256 token columns, acc = 2D - sum q, LoRA
 //               up-projection and dequantisation, coalesced stores of y along
@@ -148,7 +150,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
             for (int tile = blockIdx.x; tile < a.n_tiles && !*abort_flag; tile += gridDim.x) {
                 const TileCoord tc = tile_coord(a.desc, a.n, n_tt, tile);
                 const CUtensorMap* tm = a.tmaps + tc.lin;
-                const int nkb = a.desc[tc.lin].d_in / BK;
+                const int nkb = a.desc[tc.lin].qrow / BK;
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
@@ -164,7 +166,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
             int it = 0, tcount = 0;
             for (int tile = blockIdx.x; tile < a.n_tiles && !*abort_flag; tile += gridDim.x, ++tcount) {
                 const TileCoord tc = tile_coord(a.desc, a.n, n_tt, tile);
-                const int nkb = a.desc[tc.lin].d_in / BK;
+                const int nkb = a.desc[tc.lin].qrow / BK;
                 const int buf = tcount & 1;
                 const uint32_t acc_ph = (uint32_t)(tcount >> 1) & 1u;
                 if (!ptx::mbar_wait(&acc_empty[buf], acc_ph ^ 1u)) { set_err(a.err, DFSSM_DEVERR_TIMEOUT); *abort_flag = 1; break; }
@@ -197,26 +199,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
             const TileCoord tc = tile_coord(a.desc, a.n, n_tt, tile);
             const DevDesc d = a.desc[tc.lin];
             const dfssm_stack_entry& e = entry_at(a.entries, a.single, tc.lin);
-            const int nkb = d.d_in / BK;
+            const int nseg = d.qrow / kSegCols;
+            const int rb = d.d_in >> 3;                 // sign bytes per row
             const int o = tc.row0 + r;
             const bool valid = o < d.d_out && entry_ptrs_ok(e);
-            const uint4* src = reinterpret_cast<const uint4*>(e.w.sign + (int64_t)(valid ? o : 0) * (d.d_in >> 3));
-            // rolling prefetch of the next 4 k-blocks of this row's bits
-            uint4 pf[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-                pf[u] = (valid && u < nkb) ? __ldg(src + u) : make_uint4(0, 0, 0, 0);
+            const uint8_t* src = e.w.sign + (int64_t)(valid ? o : 0) * rb;
+            // segment sg of this row: words 0..3 and 4..7 (the second half is absent in a final half segment)
+            auto load_seg = [&](int sg, uint4& lo, uint4& hi) {
+                lo = make_uint4(0, 0, 0, 0);
+                hi = make_uint4(0, 0, 0, 0);
+                if (valid && sg < nseg) {
+                    lo = __ldg(reinterpret_cast<const uint4*>(src + 32 * sg));
+                    if (32 * sg + 16 < rb) hi = __ldg(reinterpret_cast<const uint4*>(src + 32 * sg + 16));
+                }
+            };
+            // two segments of look-ahead
+            uint4 c_lo, c_hi, n_lo, n_hi;
+            load_seg(0, c_lo, c_hi);
+            load_seg(1, n_lo, n_hi);
             // swizzled destination of this row: atom (r/8), row-in-atom (r%8)
             const uint32_t rrow = (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u;
             const uint32_t xr = (uint32_t)(r & 7);
             bool ok = true;
-            for (int kb0 = 0; kb0 < nkb && ok; kb0 += 4) {
+            for (int sg = 0; sg < nseg && ok; ++sg) {
+                const uint32_t w[8] = {c_lo.x, c_lo.y, c_lo.z, c_lo.w, c_hi.x, c_hi.y, c_hi.z, c_hi.w};
+                c_lo = n_lo;
+                c_hi = n_hi;
+                load_seg(sg + 2, n_lo, n_hi);
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int kb = kb0 + u;
-                    if (kb >= nkb) break;
-                    const uint4 bits = pf[u];
-                    pf[u] = (valid && kb + 4 < nkb) ? __ldg(src + kb + 4) : make_uint4(0, 0, 0, 0);
+                for (int h = 0; h < 2; ++h) {
                     const int s = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
                     ++it;
@@ -227,15 +238,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
                     __syncwarp();
                     if (!got) { if ((threadIdx.x & 31) == 0) { set_err(a.err, DFSSM_DEVERR_TIMEOUT); *abort_flag = 1; } ok = false; break; }
                     uint8_t* dst = sA + s * A_STAGE + rrow;
-                    const uint32_t wv[4] = {bits.x, bits.y, bits.z, bits.w};
+                    // k-block 2 sg + h: bytes 32 p' + 4 c + i of plane p = 4 h + p' (0/1 bytes);
+                    // 16-byte chunk 2 p' holds words c = 0..3, chunk 2 p' + 1 words 4..7
 #pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        uint32_t e4[8];
-#pragma unroll
-                        for (int p = 0; p < 8; ++p) e4[p] = (wv[w] >> p) & 0x01010101u;
-                        const uint32_t c0 = (uint32_t)(2 * w), c1 = c0 + 1;
-                        *reinterpret_cast<uint4*>(dst + ((c0 ^ xr) << 4)) = make_uint4(e4[0], e4[1], e4[2], e4[3]);
-                        *reinterpret_cast<uint4*>(dst + ((c1 ^ xr) << 4)) = make_uint4(e4[4], e4[5], e4[6], e4[7]);
+                    for (int pp = 0; pp < 4; ++pp) {
+                        const int p = 4 * h + pp;
+                        const uint4 e0 = make_uint4((w[0] >> p) & 0x01010101u, (w[1] >> p) & 0x01010101u,
+                                                    (w[2] >> p) & 0x01010101u, (w[3] >> p) & 0x01010101u);
+                        const uint4 e1 = make_uint4((w[4] >> p) & 0x01010101u, (w[5] >> p) & 0x01010101u,
+                                                    (w[6] >> p) & 0x01010101u, (w[7] >> p) & 0x01010101u);
+                        *reinterpret_cast<uint4*>(dst + (((uint32_t)(2 * pp) ^ xr) << 4)) = e0;
+                        *reinterpret_cast<uint4*>(dst + (((uint32_t)(2 * pp + 1) ^ xr) << 4)) = e1;
                     }
                     ptx::fence_proxy_async_smem();
                     ptx::mbar_arrive(&full_a[s]);

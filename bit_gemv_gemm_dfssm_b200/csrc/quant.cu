@@ -11,19 +11,21 @@
 //   sumq   = sum_j q[t,j]                          (int32)
 //   h[t,k] = sum_j W_B[k,j] q[t,j]                 (int32, warp MMA s8 x s8)
 //   u[t,k] = s_B[k] * h[t,k]                       (fp32)
-// and stores q in the permuted int8 layout the scaffold kernels read, plus
-// s_x, sumq and u.
+// and stores q in the plane-major int8 layouts the scaffold kernels read (the
+// 16-token decode image for m <= 16, token rows for the prefill otherwise),
+// plus s_x, sumq and u.
 //
 // A block owns one linear and up to kTokPerBlock tokens, processed in rounds of
 // 16 tokens (one MMA tile). The 8 warps split the 32-column k-blocks of d_in
 // between them: pass 1 finds each token's amax, pass 2 quantises x straight
 // into MMA A fragments (16 tokens x 32 columns), runs h += q * W_B^T on the
 // warp MMA (m16n8k32, two n-tiles for the 16 LoRA rows) and writes q to a
-// shared tile, from which the block stores the permuted rows with 16-byte
-// stores (a 4x4 byte transpose with PRMT per 16 bytes).
+// shared tile. From there each thread takes 128 columns of a token and stores
+// them as eight 16-byte plane pieces (two 4x4 byte transposes with PRMT per
+// 32-column group).
 //
-// Few tokens (m <= 16, one round): the k-blocks of a linear are split over S
-// blocks so that W_B (the only large read) streams through many SMs. Every
+// Few tokens (m <= 16, one round): the 128-column pieces of a linear are split
+// over S blocks so that W_B (the only large read) streams through many SMs. Every
 // split block finds the full-row amax itself, handles its own columns, and
 // writes partial h and sum q; the last split block to finish (atomic ticket)
 // adds the partials in split order, writes the per-token scalars and resets
@@ -126,7 +128,7 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__
         return;
     }
     const int d_in = d.d_in;
-    const int nkb = d_in >> 5;                    // 32-column k-blocks
+    const int nquad = d_in >> 7;                  // 128-column pieces (4 k-blocks of 32 columns)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, c = lane & 3;
 
@@ -138,7 +140,8 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__
 
     // split along d_in (few tokens) or along tokens (many tokens)
     const int split = qa.splits > 1 ? (int)blockIdx.x : 0;
-    const int kb_lo = split * nkb / qa.splits, kb_hi = (split + 1) * nkb / qa.splits;
+    const int pc_lo = split * nquad / qa.splits, pc_hi = (split + 1) * nquad / qa.splits;
+    const int kb_lo = 4 * pc_lo, kb_hi = 4 * pc_hi;
     const int tb0 = qa.splits > 1 ? 0 : blockIdx.x * kTokPerBlock;
     const int tb1 = min(m, tb0 + kTokPerBlock);
     for (int t0 = tb0; t0 < tb1; t0 += kTok) {
@@ -263,20 +266,38 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__
             }
         }
 
-        // ---- q rows: permuted (position 32G + 4p + i <- column 32G + 8i + p) and natural (debug)
-        const int c_lo = 2 * kb_lo, nchunk = 2 * (kb_hi - kb_lo);    // 16-byte output chunks of this block
-        for (int i = tid; i < nt * nchunk; i += kThreads) {
-            const int tk = i / nchunk, s16 = c_lo + (i - tk * nchunk);
-            const int G = s16 >> 1, hlf = s16 & 1;
-            // output word r holds p = 4 hlf + r: bytes src[p], src[8+p], src[16+p], src[24+p],
-            // i.e. byte r of source words hlf, 2 + hlf, 4 + hlf, 6 + hlf of the 32-byte group
-            const uint32_t* src = reinterpret_cast<const uint32_t*>(q_s + tk * d_in + 32 * G);
-            const uint4 o4 = transpose4x4(src[hlf], src[2 + hlf], src[4 + hlf], src[6 + hlf]);
-            // the decode kernel (m <= 16) quantises for itself; only the prefill path reads q_ws
-            if (qa.splits == 1) *reinterpret_cast<uint4*>(q_ws + d.q_off + (int64_t)(t0 + tk) * d_in + 16 * s16) = o4;
-            if (e.dbg.q)
-                *reinterpret_cast<uint4*>(e.dbg.q + (int64_t)(t0 + tk) * d_in + 16 * s16) =
-                    *reinterpret_cast<const uint4*>(q_s + tk * d_in + 16 * s16);
+        // ---- q out: token tk, 128-column piece pc = half hc of segment sg. For each 32-column
+        // group c4 of the piece, words W0..W7 of the natural bytes give plane p's four bytes
+        // (columns 32c + 8i + p, i = 0..3) as byte p % 4 of W[p / 4], W[2 + p / 4], W[4 + p / 4],
+        // W[6 + p / 4]; the four groups' words of plane p form one 16-byte piece.
+        const int npc = pc_hi - pc_lo;
+        const bool to_image = m <= kImgTokens;
+        for (int i = tid; i < nt * npc; i += kThreads) {
+            const int tk = i / npc, pc = pc_lo + (i - tk * npc);
+            const int sg = pc >> 1, hc = pc & 1, t = t0 + tk;
+            const uint32_t* src = reinterpret_cast<const uint32_t*>(q_s + tk * d_in + 128 * pc);
+            uint32_t P[8][4];
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const uint32_t* W = src + 8 * c4;
+                const uint4 lo = transpose4x4(W[0], W[2], W[4], W[6]);   // planes 0..3
+                const uint4 hi = transpose4x4(W[1], W[3], W[5], W[7]);   // planes 4..7
+                P[0][c4] = lo.x; P[1][c4] = lo.y; P[2][c4] = lo.z; P[3][c4] = lo.w;
+                P[4][c4] = hi.x; P[5][c4] = hi.y; P[6][c4] = hi.z; P[7][c4] = hi.w;
+            }
+            // decode image: unit 8 sg + p, token group t / 8, K half hc, row t % 8; prefill rows: 32 p + 16 hc
+            int8_t* base = to_image ? q_ws + d.dq_off + 4096 * sg + 256 * (t >> 3) + 128 * hc + 16 * (t & 7)
+                                    : q_ws + d.q_off + (int64_t)t * d.qrow + 256 * sg + 16 * hc;
+            const int pstride = to_image ? 512 : 32;
+#pragma unroll
+            for (int p = 0; p < 8; ++p)
+                *reinterpret_cast<uint4*>(base + p * pstride) = make_uint4(P[p][0], P[p][1], P[p][2], P[p][3]);
+            if (e.dbg.q) {
+                const uint4* sq = reinterpret_cast<const uint4*>(src);
+                uint4* dq = reinterpret_cast<uint4*>(e.dbg.q + (int64_t)t * d_in + 128 * pc);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) dq[u] = sq[u];
+            }
         }
         __syncthreads();   // q_s and red are reused by the next round
     }
@@ -287,11 +308,12 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__
 cudaError_t launch_quant(const LaunchCtx& c) {
     int splits = 1;
     if (c.m <= kTok) {
-        // enough blocks to cover the SMs twice, at least 8 k-blocks (one per warp) per split
-        int min_nkb = 1 << 30;
-        for (int i = 0; i < c.n; ++i) min_nkb = min(min_nkb, c.host_desc[i].d_in / 32);
+        // enough blocks to cover the SMs twice, at least two 128-column pieces (8 k-blocks,
+        // one per warp) per split
+        int min_pc = 1 << 30;
+        for (int i = 0; i < c.n; ++i) min_pc = min(min_pc, c.host_desc[i].d_in / 128);
         splits = (2 * c.sm_count + c.n - 1) / c.n;
-        splits = max(1, min(splits, min(kMaxSplits, min_nkb / kWarps)));
+        splits = max(1, min(splits, min(kMaxSplits, min_pc / 2)));
     }
     dim3 grid(splits > 1 ? splits : (c.m + kTokPerBlock - 1) / kTokPerBlock, c.n);
     const size_t smem = ((sizeof(QuantRed) + 127) & ~(size_t)127) + (size_t)kTok * c.max_d_in;
