@@ -1,54 +1,42 @@
 // Decode path (1 <= m <= 16 tokens): the scaffold contraction streamed from HBM
-// on the tcgen05 tensor cores, with the LoRA up-projection and both
-// dequantisation epilogues fused.
+// with the LoRA up-projection and both dequantisation epilogues fused.
 //
 // "Density Field State Space Models" (gist.science technical summary), §2.C:
 // the 1-bit scaffold weights are expanded on the fly to int8 and fed to int8
 // tensor cores, which cuts weight traffic 8x against int8 weights; at batch 1
-// the layer is bound by that weight stream. The expansion is the only work
-// left on the SM's integer pipes here:
+// the layer is bound by that weight stream. Here the bits never exist as int8
+// bytes in memory:
 //
-//  * Bit planes. For a 32-bit word w of sign bits (columns 32c .. 32c+31 of a
-//    256-column segment) and a bit position p, w & (0x01010101 << p) is four
-//    bytes, each 0 or 2^p: the bits of columns 32c + 8i + p (i = 0..3), scaled
-//    by 2^p. One LOP3 expands four weights. The eight words of a segment give,
-//    for each p, 32 bytes: the K = 32 operand of one int8 MMA.
-//  * A operand in tensor memory. Each expander thread owns one of the 128 rows
-//    of a tile (= one TMEM lane) and writes its 64 expanded words with
-//    tcgen05.st; the MMA reads A from TMEM, so the 8x larger expanded operand
-//    never passes through shared memory. Planes 0-3 are taken as
-//    (w >> p) & 0x01010101 (bytes 0 or 1), planes 4-7 as (w >> p) & 0x10101010
-//    (bytes 0 or 16), so two int32 accumulators per tile suffice:
-//    D_lo = sum_{p<4} S_p and D_hi = 16 * sum_{p>=4} S_p, exactly.
-//  * B operand: the int8 activations of up to 16 tokens (MMA N = 16) in the
-//    same plane-major order (K position 32p + 4c + i <-> column 32c + 8i + p),
-//    copied once per linear into shared memory as 8-row x 16-byte core
-//    matrices (the quantisation kernel writes them in that layout).
-//  * S1 = D_lo + D_hi / 16 = sum_{bit = 1} q, and acc = 2 * S1 - sum_j q (a +-1
-//    weight is 2b - 1).
-//
-// Persistent kernel, one CTA per SM, 16 warps with fixed roles:
-//   warp 0       TMA producer of sign tiles (128 rows x 128 bytes, 128B swizzle,
-//                no multicast) through a per-linear tensor map whose global
-//                address it sets on the device (tensormap.replace); 4 stages
-//   warp 1       TMEM owner; bulk copy of each linear's activation image
-//   warps 4-11   two expander warpgroups taking alternate 256-column segments
-//                of a tile; a group writes a segment into one of its three TMEM
-//                slots and hands it over at a named barrier
-//   warps 2, 3   one MMA issuer per group: after the barrier it issues the
-//                segment's 8 MMAs (tcgen05.mma.kind::i8, A in TMEM) into the
-//                group's own pair of accumulators. Two issue streams, each a
-//                single thread (so each accumulator is written in issue order),
-//                and a hardware barrier instead of an mbarrier round trip per
-//                segment
-//   warps 12-15  epilogue: add the groups' accumulators, LoRA up-projection,
-//                dequantisation (epilogue.cuh), coalesced stores
-// Work: the 128-row tiles of all linears of the call, split into contiguous
-// ranges holding equal shares of the sign bytes. Every mbarrier wait is
-// bounded; a timeout sets the error word, later waits return at once, and the
-// CTA runs to its end without blocking.
-#include <cuda.h>
-
+//  * Work: blocks of R = 64 * RT output rows (4 warps, RT 16-row tiles per
+//    warp), flattened over all linears of the call. Each CTA is persistent and
+//    owns a contiguous range of blocks holding an equal share of the sign bytes.
+//  * Streaming: a block is consumed in k-chunks of 1024 columns (128 bytes per
+//    row). A ring of kStages shared-memory slots is filled with 16-byte
+//    cp.async; in slot row r, 16-byte chunk j sits at (j + r) mod 8, so the
+//    ldmatrix reads of 8 rows hit 8 different bank groups. The last k-chunk of
+//    a block also brings its alpha, s_A and W_A.
+//  * Activations: when a CTA reaches a new linear it quantises that linear's
+//    x itself (same fp32 arithmetic as the quantisation kernel, so the same
+//    bits) into shared memory, while its weight chunks are already in flight.
+//    Only the LoRA vector u = s_B * h comes from the quantisation kernel, and
+//    the CTA waits for that kernel (programmatic dependent launch) just before
+//    its first epilogue.
+//  * Expansion: for a 32-bit word of sign bits w and bit position p,
+//    w & (0x01010101 << p) is four bytes, each 0 or 2^p: the bits of columns
+//    8i + p (i = 0..3) scaled by 2^p. One LOP3 expands four weights.
+//  * These bytes are the u8 A operand of the warp MMA m16n8k32 (u8 x s8 -> s32),
+//    loaded with ldmatrix.x4 straight from the staged bits; the int8
+//    activations in the matching permuted column order (byte 4p + i of a
+//    32-column group = column 8i + p) are the s8 B operand, tokens = N. In
+//    shared memory each 256-column group of a token row is laid out so that
+//    thread c of a quad reads its 16 B-fragment words with four 16-byte loads
+//    as (b0, b1) register pairs, one pair per bit position p.
+//  * One accumulator set per p, so set p sums 2^p * S_p exactly;
+//    S1 = sum_p D_p / 2^p = sum_{bit = 1} q, and acc = 2 * S1 - sum_j q
+//    (a +-1 weight is 2b - 1).
+//  * Epilogue (epilogue.cuh): lane i of a warp takes output row i, gathers its
+//    sums with warp shuffles, and applies the LoRA up-projection and the
+//    dequantisation in the same fp32 order as the prefill path.
 #include "dfssm_internal.cuh"
 #include "epilogue.cuh"
 #include "ptx.cuh"
@@ -57,582 +45,476 @@ namespace dfssm {
 
 namespace {
 
-constexpr int BM = 128;                    // rows per tile: MMA M, TMEM lanes
-constexpr int NTOK = 16;                   // MMA N: token columns (columns >= m are dropped)
-constexpr int STAGE_ROW_BYTES = 128;       // sign bytes per row per TMA stage (4 segments)
-constexpr int SIGN_STAGE = BM * STAGE_ROW_BYTES;   // 16 KB
-constexpr int NS = 4;                      // sign ring stages
-constexpr int NGRP = 2;                    // expander / issuer warpgroups
-constexpr int NSLOT = 3;                   // TMEM A slots per group
-constexpr uint32_t A_COLS = 64;            // TMEM columns per A slot: 8 planes x 8 words
-constexpr uint32_t D_COLS = 2 * NTOK;      // accumulators of one group and buffer: lo, hi (16 tokens each)
-constexpr uint32_t A_COL0 = NGRP * 2 * D_COLS;   // A slots after [group][buffer] accumulators
-constexpr uint32_t TMEM_COLS = 512;
-static_assert(A_COL0 + NGRP * NSLOT * A_COLS <= TMEM_COLS, "TMEM budget");
-constexpr int THREADS = 512;
-constexpr int EPI_WARP0 = 12;
-constexpr int STAT_FLOATS = NTOK * (2 + kRank);   // per-token s_x, sum q, u[16] of one linear
-constexpr int kMapSlots = 4;               // per-CTA ring of device-edited sign tensor maps
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+#ifndef DFSSM_DECODE_CHUNK_BYTES
+#define DFSSM_DECODE_CHUNK_BYTES 128
+#endif
+#ifndef DFSSM_DECODE_STAGES
+#define DFSSM_DECODE_STAGES 3
+#endif
+constexpr int kChunkBytes = DFSSM_DECODE_CHUNK_BYTES;   // sign bytes per row per k-chunk (8 columns per byte)
+constexpr int kChunkJ = kChunkBytes / 16;                // 16-byte pieces per row per chunk
+constexpr int kGroups = kChunkBytes / 32;                // 256-column groups per chunk
+constexpr int kTokPad = 64;        // q row stride = round_up(d_in, 256) + 64 (= 64 mod 128: conflict-free B reads)
 
-// kind::i8 instruction descriptor: D s32, A u8 (bytes 0 or 2^p), B s8, both K-major, N = 16, M = 128.
-constexpr uint32_t kIdesc = (2u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(NTOK >> 3) << 17) |
-                            ((uint32_t)(BM >> 4) << 24);
+// every 256-column group of a staged q row takes 256 bytes, even a half-filled last one
+__host__ __device__ __forceinline__ int q_stride(int d_in) { return ((d_in + 255) & ~255) + kTokPad; }
+constexpr int kStages = DFSSM_DECODE_STAGES;
+constexpr int kMaxTok = 16;
 
 struct DecodeArgs {
     const dfssm_stack_entry* entries;
     dfssm_stack_entry single;
-    const DevDesc* desc;           // desc[0] is the first linear of this launch
-    const CUtensorMap* sign_tmpl;  // per linear: its sign map with a placeholder address
-    CUtensorMap* map_slots;        // kMapSlots per CTA
-    const int8_t* q_ws;
-    const TokStats* st_ws;
-    uint32_t* err;
+    const DevDesc* desc;     // desc[0] is the first linear of this launch
     int n;
     int m;
-    int total_tiles;
-    int img_bytes;                 // bytes of one activation-image buffer (16 x qrow of the widest linear)
-    int img_bufs;                  // 1 or 2
-    int64_t total_bytes;           // sign bytes of the n linears
+    const TokStats* st_ws;
+    int64_t total_bytes;     // sign bytes of the n linears
+    int slot_bytes;          // bytes of one ring slot
+    int q_region;            // bytes of the staged-q region
 };
 
-// Shared-memory B descriptor, K-major, no swizzle: core matrices of 8 rows x 16 bytes,
-// the two 16-byte K halves 128 bytes apart (leading offset), groups of 8 token rows
-// 256 bytes apart (stride offset), descriptor version 1.
-__device__ __forceinline__ uint64_t img_desc(uint32_t saddr) {
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)(256 >> 4) << 32) |
-           ((uint64_t)1 << 46);
+// Fields of one linear, cached in registers while a cursor is on it.
+struct Lin {
+    int d_in, d_out, rb, nchunks, nblocks, y_dtype;
+    int64_t byte_rel;        // first sign byte relative to desc[0]
+    int64_t st_off;
+    const uint8_t* sign;
+    const float* alpha;
+    const float* sa;
+    const int8_t* wa;
+    const uint16_t* x;
+    void* y;
+    int32_t* dbg_acc;
+    bool ok;                 // entry pointers valid
+};
+
+template <int R>
+__device__ __forceinline__ void load_lin(const DecodeArgs& a, int l, Lin& L) {
+    const DevDesc& d = a.desc[l];
+    const dfssm_stack_entry& e = entry_at(a.entries, a.single, l);
+    L.d_in = d.d_in;
+    L.d_out = d.d_out;
+    L.rb = d.d_in >> 3;
+    L.nchunks = (d.d_in / 8 + kChunkBytes - 1) / kChunkBytes;
+    L.nblocks = (d.d_out + R - 1) / R;
+    L.y_dtype = d.y_dtype;
+    L.byte_rel = d.byte_begin - a.desc[0].byte_begin;
+    L.st_off = d.st_off;
+    L.sign = e.w.sign;
+    L.alpha = e.w.alpha;
+    L.sa = e.w.sa;
+    L.wa = e.w.wa;
+    L.x = reinterpret_cast<const uint16_t*>(e.x);
+    L.y = e.y;
+    L.dbg_acc = e.dbg.acc;
+    L.ok = entry_ptrs_ok(e);
 }
 
-__device__ __forceinline__ void set_err(uint32_t* err, uint32_t bit) { atomicOr(err, bit); }
-
-// The linear a tile belongs to, with the fields every role needs.
 struct Cursor {
-    int lin, t_in, ntiles, nseg, nstage, d_out;
-    __device__ void load(const DecodeArgs& a, int l) {
-        const DevDesc& d = a.desc[l];
-        lin = l;
-        d_out = d.d_out;
-        ntiles = (d.d_out + BM - 1) / BM;
-        nseg = d.qrow >> 8;
-        nstage = (d.d_in / 8 + STAGE_ROW_BYTES - 1) / STAGE_ROW_BYTES;
+    int l, b, kc;   // linear, block within the linear, k-chunk within the block
+};
+
+template <int R>
+struct Walk {
+    Cursor c;
+    Lin L;
+    __device__ __forceinline__ bool valid(const DecodeArgs& a, int64_t hi) const {
+        return c.l < a.n && L.byte_rel + (int64_t)c.b * R * L.rb < hi;
     }
-    // position on flattened tile T, which lies in linear l or a later one
-    __device__ void start(const DecodeArgs& a, int l, int T) {
-        load(a, l);
-        t_in = T - (a.desc[l].rt_begin - a.desc[0].rt_begin);
-        while (t_in >= ntiles && lin + 1 < a.n) {
-            t_in -= ntiles;
-            load(a, lin + 1);
+    __device__ __forceinline__ void advance(const DecodeArgs& a) {
+        if (++c.kc >= L.nchunks) {
+            c.kc = 0;
+            if (++c.b >= L.nblocks) {
+                c.b = 0;
+                if (++c.l < a.n) load_lin<R>(a, c.l, L);
+            }
         }
     }
-    // next tile; true when it belongs to another linear
-    __device__ bool advance(const DecodeArgs& a) {
-        if (++t_in < ntiles) return false;
-        t_in = 0;
-        if (lin + 1 < a.n) load(a, lin + 1);
-        return true;
+    // first block whose first sign byte is at or after `lo`
+    __device__ void start(const DecodeArgs& a, int64_t lo) {
+        const int64_t base = a.desc[0].byte_begin;
+        int lo_l = 0, hi_l = a.n - 1;
+        while (lo_l < hi_l) {
+            const int mid = (lo_l + hi_l + 1) >> 1;
+            if (a.desc[mid].byte_begin - base <= lo) lo_l = mid; else hi_l = mid - 1;
+        }
+        c = Cursor{lo_l, 0, 0};
+        load_lin<R>(a, c.l, L);
+        const int64_t bb = (int64_t)R * L.rb;
+        c.b = (int)((lo - L.byte_rel + bb - 1) / bb);
+        if (c.b >= L.nblocks) {
+            c.b = 0;
+            if (++c.l < a.n) load_lin<R>(a, c.l, L);
+        }
     }
 };
 
-// First flattened tile of linear l whose first sign byte is at or after byte `pos`
-// of the call (the first tile of linear l + 1 if there is none).
-__device__ int tile_at(const DecodeArgs& a, int l, int64_t pos) {
-    const DevDesc& d = a.desc[l];
-    const int64_t tb = (int64_t)BM * (d.d_in / 8);
-    const int64_t t = (pos - (d.byte_begin - a.desc[0].byte_begin) + tb - 1) / tb;
-    const int nt = (d.d_out + BM - 1) / BM;
-    return d.rt_begin - a.desc[0].rt_begin + (int)(t < nt ? t : nt);
+// Fill a ring slot with k-chunk kc of block b: R rows x (up to) 128 sign bytes,
+// plus alpha, s_A and W_A of the block when kc is its last chunk.
+template <int R>
+__device__ __forceinline__ void issue_step(const Cursor& c, const Lin& L, uint8_t* slot) {
+    if (!L.ok) return;                    // flagged by the quantisation kernel
+    const int row0 = c.b * R;
+    const int nrows = min(R, L.d_out - row0);
+    const int nch = min(kChunkBytes, L.rb - kChunkBytes * c.kc) >> 4;   // 16-byte pieces in this chunk
+    const uint8_t* src = L.sign + (int64_t)row0 * L.rb + kChunkBytes * c.kc;
+    // thread t copies 16-byte piece j = t % kChunkJ of rows t / kChunkJ + k * kRowStep
+    constexpr int kRowStep = kThreads / kChunkJ;
+    const int j = threadIdx.x % kChunkJ;
+    int r = threadIdx.x / kChunkJ;
+    if (j < nch) {
+        const uint8_t* s0 = src + (int64_t)r * L.rb + 16 * j;
+        const int64_t sstep = (int64_t)kRowStep * L.rb;
+        for (; r < nrows; r += kRowStep, s0 += sstep)
+            ptx::cp_async16(slot + r * kChunkBytes + 16 * ((j + r) % kChunkJ), s0);
+    }
+    if (c.kc == L.nchunks - 1) {
+        uint8_t* par = slot + R * kChunkBytes;
+        const int n4 = (nrows + 3) >> 2;
+        for (int i = threadIdx.x; i < n4; i += kThreads) {
+            const uint32_t bytes = (uint32_t)min(16, 4 * (nrows - 4 * i));
+            ptx::cp_async16_zfill(par + 16 * i, L.alpha + row0 + 4 * i, bytes);
+            ptx::cp_async16_zfill(par + 4 * R + 16 * i, L.sa + row0 + 4 * i, bytes);
+        }
+        for (int r = threadIdx.x; r < nrows; r += kThreads)
+            ptx::cp_async16(par + 8 * R + 16 * r, L.wa + (int64_t)(row0 + r) * kRank);
+    }
 }
 
-// lane 0 waits, the warp follows. Returns false on timeout, or at once once
-// `abort` is set; the caller then sets `abort` (and the error word) and keeps
-// walking its loop without waiting, so no partner is left blocked.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, int lane, volatile uint32_t* abort) {
-    bool ok = true;
-    if (lane == 0) ok = !*abort && ptx::mbar_wait(bar, parity);
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    __syncwarp();
-    return ok;
-}
-__device__ __forceinline__ bool thread_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort) {
-    return !*abort && ptx::mbar_wait(bar, parity);
-}
-__device__ __forceinline__ void fail(uint32_t* err, volatile uint32_t* abort) {
-    set_err(err, DFSSM_DEVERR_TIMEOUT);
-    *abort = 1;
+// Shared-memory position of q for column 32 gg + 8 i + p of a token row (gg: 32-column
+// group, i = 0..3, p = bit position). The 256-column group G = gg / 8 occupies 256
+// bytes; thread c = gg % 4 of an MMA quad owns 64 of them, holding for each p the
+// word of group gg (w = 0, B fragment b0) next to the word of group gg + 4 (w = 1,
+// b1). Logical 16-byte chunk k = p / 2 of that block is stored at (k + c) mod 4, so
+// the 8 lanes of a quarter-warp hit 8 different bank groups (with a token stride of
+// 64 mod 128).
+__device__ __forceinline__ int q_pos(int gg, int i, int p) {
+    const int G = gg >> 3, c = gg & 3, w = (gg >> 2) & 1;
+    return 256 * G + 64 * c + 16 * (((p >> 1) + c) & 3) + 8 * (p & 1) + 4 * w + i;
 }
 
-template <int NT>
-__global__ void __launch_bounds__(THREADS, 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
-    extern __shared__ uint8_t smem_raw[];
-    // 1024-byte aligned base, offset from the __shared__ array so addressing stays in shared space
-    uint8_t* smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint8_t* ring = smem;                                       // NS sign stages
-    uint8_t* img = ring + NS * SIGN_STAGE;                      // img_bufs activation images
-    float* stats = reinterpret_cast<float*>(img + a.img_bufs * a.img_bytes);   // [4 epilogue warps][STAT_FLOATS]
-    uint8_t* map_s = reinterpret_cast<uint8_t*>(stats + 4 * STAT_FLOATS);        // 128 bytes, 128-aligned
-    uint64_t* bars = reinterpret_cast<uint64_t*>(map_s + 128);
-    uint64_t* sign_full = bars;                      // [NS] TMA bytes
-    uint64_t* sign_empty = bars + NS;                // [NS] 8 expander warps
-    uint64_t* a_empty = bars + 2 * NS;               // [NGRP][NSLOT] MMA commit
-    uint64_t* d_full = a_empty + NGRP * NSLOT;       // [2] one arrival per group
-    uint64_t* d_empty = d_full + 2;                  // [2] 4 epilogue warps
-    uint64_t* q_full = d_empty + 2;                  // [2] bulk-copy bytes
-    uint64_t* q_empty = q_full + 2;                  // [2] one arrival per group
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_empty + 2);
-    volatile uint32_t* abort_flag = tmem_slot + 1;
+struct TokShared {
+    float sx[kMaxTok];
+    int sumq[kMaxTok];
+    float red_f[kWarps][kMaxTok];
+    int red_i[kWarps][kMaxTok];
+    float u[kMaxTok][kRank];
+};
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int* loc = reinterpret_cast<int*>(tmem_slot + 2);   // linears holding this CTA's first and end byte
+// Quantise the m x d_in activations of linear L into the permuted int8 layout
+// (token stride d_in + kTokPad), with per-token s_x and sum q. Same arithmetic
+// as the quantisation kernel (epilogue.cuh), so the same bytes.
+__device__ void quantise_into_smem(const Lin& L, int m, uint8_t* q_s, TokShared& ts) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n8 = L.d_in >> 3;                      // 8-column chunks per row
+    const int qstride = q_stride(L.d_in);
+    for (int t = 0; t < m; ++t) {
+        float am = 0.0f;
+        for (int ch = tid; ch < n8; ch += kThreads) {
+            const uint4 v = *reinterpret_cast<const uint4*>(L.x + (int64_t)t * L.d_in + 8 * ch);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) am = fmaxf(am, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+        if (lane == 0) ts.red_f[warp][t] = am;
+    }
+    __syncthreads();
+    for (int t = 0; t < m; ++t) {
+        float am = ts.red_f[0][t];
+#pragma unroll
+        for (int w = 1; w < kWarps; ++w) am = fmaxf(am, ts.red_f[w][t]);
+        const float inv = quant_inv(am);
+        const bool zero = am == 0.0f;
+        int sum = 0;
+        for (int ch = tid; ch < n8; ch += kThreads) {
+            const uint4 v = *reinterpret_cast<const uint4*>(L.x + (int64_t)t * L.d_in + 8 * ch);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            // columns 8 ch + p (p = 0..7) of 32-column group gg = ch / 4 (i = ch % 4)
+            uint8_t* row = q_s + t * qstride;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int q0 = quant1(bf16_lo(w[i]), inv, zero), q1 = quant1(bf16_hi(w[i]), inv, zero);
+                sum += q0 + q1;
+                row[q_pos(ch >> 2, ch & 3, 2 * i)] = (uint8_t)q0;
+                row[q_pos(ch >> 2, ch & 3, 2 * i + 1)] = (uint8_t)q1;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (lane == 0) ts.red_i[warp][t] = sum;
+        if (tid == 0) ts.sx[t] = quant_sx(am);
+    }
+    __syncthreads();
+    if (tid < m) {
+        int s = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) s += ts.red_i[w][tid];
+        ts.sumq[tid] = s;
+    }
+    // (the caller synchronises before sumq is read)
+}
 
-    // This CTA's byte range [lo, hi) of the call's sign bytes; every thread tests a few
-    // linears at once, so locating it costs one round of loads instead of a search.
+template <int RT, int NT>
+__global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant__ DecodeArgs a) {
+    constexpr int R = 16 * RT * kWarps;
+    extern __shared__ __align__(128) uint8_t smem[];
+    TokShared& ts = *reinterpret_cast<TokShared*>(smem);
+    uint8_t* q_s = smem + ((sizeof(TokShared) + 127) & ~(size_t)127);
+    uint8_t* ring = q_s + a.q_region;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, c = lane & 3;
+    const int m = a.m;
+
     const int64_t lo = a.total_bytes * blockIdx.x / gridDim.x;
     const int64_t hi = a.total_bytes * (blockIdx.x + 1) / gridDim.x;
-    {
-        const int64_t b0 = a.desc[0].byte_begin;
-        for (int i = threadIdx.x; i < a.n; i += THREADS) {
-            const int64_t b = a.desc[i].byte_begin - b0;
-            const int64_t bn = i + 1 < a.n ? a.desc[i + 1].byte_begin - b0 : INT64_MAX;
-            if (b <= lo && lo < bn) loc[0] = i;     // exactly one linear matches each position
-            if (b <= hi && hi < bn) loc[1] = i;
+    Walk<R> cw, lw;
+    cw.start(a, lo);
+    lw = cw;
+
+    // ---- prologue: kStages - 1 slots in flight
+#pragma unroll
+    for (int s = 0; s < kStages - 1; ++s) {
+        if (lw.valid(a, hi)) {
+            issue_step<R>(lw.c, lw.L, ring + s * a.slot_bytes);
+            lw.advance(a);
         }
+        ptx::cp_async_commit();
     }
 
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < NS; ++s) {
-            ptx::mbar_init(&sign_full[s], 1);
-            ptx::mbar_init(&sign_empty[s], NGRP * 4);
-        }
-        for (int s = 0; s < NGRP * NSLOT; ++s) ptx::mbar_init(&a_empty[s], 1);
-        for (int b = 0; b < 2; ++b) {
-            ptx::mbar_init(&d_full[b], NGRP);
-            ptx::mbar_init(&d_empty[b], 4);
-            ptx::mbar_init(&q_full[b], 1);
-            ptx::mbar_init(&q_empty[b], NGRP);
-        }
-        *abort_flag = 0;
-        ptx::fence_mbar_init();
-    }
-    if (warp == 1) {
-        ptx::tmem_alloc(tmem_slot, TMEM_COLS);
-        ptx::tmem_relinquish();
-    }
-    ptx::tc_fence_before();
-    __syncthreads();
-    ptx::tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
+    int D[RT][NT][8][4];
+    int q_lin = -1, u_lin = -1;
+    // ldmatrix lane role: matrix (lane / 8) = (row half, 16-byte half of the 32-byte group)
+    const int lm_row = (lane & 7) + 8 * ((lane >> 3) & 1);
+    const int lm_hi = lane >> 4;
+    const int wrow0 = warp * 16 * RT;             // first row of this warp in a block
 
-    const int lin0 = loc[0];
-    const int t_lo = tile_at(a, lin0, lo);
-    const int t_hi = blockIdx.x + 1 == gridDim.x ? a.total_tiles : tile_at(a, loc[1], hi);
-    const uint32_t nb = (uint32_t)a.img_bufs;
+    for (int it = 0; cw.valid(a, hi); ++it) {
+        const Lin& L = cw.L;
+        if (cw.c.l != q_lin) {
+            // a new linear: quantise its activations (its weights are already streaming)
+            if (L.ok) quantise_into_smem(L, m, q_s, ts);
+            q_lin = cw.c.l;
+        }
+        if (lw.valid(a, hi)) {
+            issue_step<R>(lw.c, lw.L, ring + ((it + kStages - 1) % kStages) * a.slot_bytes);
+            lw.advance(a);
+        }
+        ptx::cp_async_commit();
+        ptx::cp_async_wait<kStages - 1>();
+        const bool last_chunk = cw.c.kc == L.nchunks - 1;
+        if (last_chunk && u_lin != cw.c.l) {
+            // the LoRA vector u = s_B * h of this linear, from the quantisation kernel
+            ptx::pdl_wait();
+            for (int i = tid; i < m * kRank; i += kThreads)
+                ts.u[i >> 4][i & 15] = a.st_ws[L.st_off + (i >> 4)].u[i & 15];
+            u_lin = cw.c.l;
+        }
+        __syncthreads();
 
-    if (warp == 0) {
-        // ------------------------------------------------ sign producer (whole warp: the map copy is warp-wide)
-        Cursor cur;
-        if (t_lo < t_hi) cur.start(a, lin0, t_lo);
-        uint32_t S = 0;
-        int map_i = 0, prev_lin = -1;
-        const CUtensorMap* gmap = nullptr;
-        bool lin_ok = false;
-        for (int T = t_lo; T < t_hi && !*abort_flag; ++T) {
-            const int row0 = cur.t_in * BM;
-            const bool new_lin = cur.lin != prev_lin;
-            prev_lin = cur.lin;
-            for (int k = 0; k < cur.nstage; ++k, ++S) {
-                const int s = (int)(S % NS);
-                if (!warp_wait(&sign_empty[s], ((S / NS) & 1u) ^ 1u, lane, abort_flag)) {
-                    if (lane == 0) fail(a.err, abort_flag);
-                    break;
-                }
-                if (k == 0 && new_lin) {
-                    // Stage S - NS has been consumed, so every load issued before it has
-                    // completed; the slot edited here was last used at least NS stages ago.
-                    const dfssm_stack_entry& e = entry_at(a.entries, a.single, cur.lin);
-                    lin_ok = entry_ptrs_ok(e);
-                    if (lin_ok) {
-                        CUtensorMap* slot = a.map_slots + (size_t)blockIdx.x * kMapSlots + map_i;
-                        map_i = (map_i + 1) % kMapSlots;
-                        if (lane < 8)
-                            reinterpret_cast<uint4*>(map_s)[lane] =
-                                reinterpret_cast<const uint4*>(a.sign_tmpl + cur.lin)[lane];
-                        __syncwarp();
-                        if (lane == 0) ptx::tensormap_replace_addr(map_s, e.w.sign);
-                        __syncwarp();
-                        ptx::tensormap_copy_release(slot, map_s);
-                        if (lane == 0) ptx::tensormap_acquire(slot);
-                        __syncwarp();
-                        gmap = slot;
-                    }
-                }
-                if (lane == 0) {
-                    if (lin_ok) {
-                        ptx::mbar_arrive_expect_tx(&sign_full[s], SIGN_STAGE);
-                        ptx::tma_load_2d(ring + s * SIGN_STAGE, gmap, k * STAGE_ROW_BYTES, row0, &sign_full[s]);
-                    } else {
-                        ptx::mbar_arrive(&sign_full[s]);    // an entry with bad pointers: nothing is read
-                    }
-                }
-                __syncwarp();
-            }
-            cur.advance(a);
+        const uint8_t* slot = ring + (it % kStages) * a.slot_bytes;
+        const int row0 = cw.c.b * R;
+        const int nrows = min(R, L.d_out - row0);
+        const bool active = wrow0 < nrows && L.ok;
+        if (cw.c.kc == 0) {
+#pragma unroll
+            for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int p = 0; p < 8; ++p)
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) D[rt][nt][p][r] = 0;
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------ activation images (from the quantisation kernel)
-        if (lane == 0) {
-            Cursor cur;
-            if (t_lo < t_hi) cur.start(a, lin0, t_lo);
-            uint32_t qv = 0;
-            int prev_lin = -1;
-            bool waited = false;
-            for (int T = t_lo; T < t_hi && !*abort_flag; ++T) {
-                if (cur.lin != prev_lin) {
-                    prev_lin = cur.lin;
-                    const uint32_t qb = qv % nb;
-                    if (!thread_wait(&q_empty[qb], ((qv / nb) & 1u) ^ 1u, abort_flag)) {
-                        fail(a.err, abort_flag);
-                        break;
-                    }
-                    ++qv;
-                    if (!waited) { ptx::pdl_wait(); waited = true; }
-                    const dfssm_stack_entry& e = entry_at(a.entries, a.single, cur.lin);
-                    if (entry_ptrs_ok(e)) {
-                        const DevDesc& d = a.desc[cur.lin];
-                        const uint32_t bytes = (uint32_t)(NTOK * d.qrow);
-                        ptx::mbar_arrive_expect_tx(&q_full[qb], bytes);
-                        const uint8_t* src = reinterpret_cast<const uint8_t*>(a.q_ws) + d.dq_off;
-                        uint8_t* dst = img + qb * a.img_bytes;
-                        for (uint32_t off = 0; off < bytes; off += 32768u)
-                            ptx::bulk_g2s(dst + off, src + off, min(32768u, bytes - off), &q_full[qb]);
-                    } else {
-                        ptx::mbar_arrive(&q_full[qb]);
+        if (active) {
+            const int qstride = q_stride(L.d_in);
+            const int cb = min(kChunkBytes, L.rb - kChunkBytes * cw.c.kc);
+            const uint32_t slot_s = ptx::smem_u32(slot);
+            // ldmatrix row addresses: row r's 16-byte piece j sits at (j + r) mod kChunkJ; rows
+            // of a tile are 8-aligned, so the rotation depends on (lane % 8) only
+            const int rot = (lm_row & 7) + lm_hi;
+            uint32_t a_addr[RT][kGroups];
+#pragma unroll
+            for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+                for (int G = 0; G < kGroups; ++G)
+                    a_addr[rt][G] = slot_s + (wrow0 + 16 * rt + lm_row) * kChunkBytes + 16 * ((2 * G + rot) % kChunkJ);
+            // B rows: tokens nt * 8 + g; lanes past m read token 0 (their MMA columns are never stored)
+            const uint8_t* qk[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int tk = nt * 8 + g;
+                const uint8_t* qrow = q_s + (tk < m ? tk : 0) * qstride + 256 * (kGroups * cw.c.kc) + 64 * c;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) qk[nt][k] = qrow + 16 * ((k + c) & 3);
+            }
+            auto group = [&](int G, bool half) {
+                uint32_t A[RT][4];
+#pragma unroll
+                for (int rt = 0; rt < RT; ++rt) {
+                    ptx::ldmatrix_x4(a_addr[rt][G], A[rt][0], A[rt][1], A[rt][2], A[rt][3]);
+                    // half group: zero A slots 16..31, so whatever b1 holds there adds nothing
+                    if (half) { A[rt][2] = 0u; A[rt][3] = 0u; }
+                }
+                // B: chunk k (bit positions 2k, 2k+1) = (b0, b1) of p = 2k, then of p = 2k + 1
+                uint4 bq[NT][4];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) bq[nt][k] = *reinterpret_cast<const uint4*>(qk[nt][k] + 256 * G);
+#pragma unroll
+                for (int p = 0; p < 8; ++p) {
+                    const uint32_t msk = 0x01010101u << p;
+#pragma unroll
+                    for (int rt = 0; rt < RT; ++rt) {
+                        const uint32_t a0 = A[rt][0] & msk, a1 = A[rt][1] & msk;
+                        const uint32_t a2 = A[rt][2] & msk, a3 = A[rt][3] & msk;
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            const uint4& v = bq[nt][p >> 1];
+                            if (p & 1) ptx::mma_u8s8(D[rt][nt][p], a0, a1, a2, a3, v.z, v.w);
+                            else       ptx::mma_u8s8(D[rt][nt][p], a0, a1, a2, a3, v.x, v.y);
+                        }
                     }
                 }
-                cur.advance(a);
-            }
-        }
-    } else if (warp == 2 || warp == 3) {
-        // ------------------------------------------------ MMA issuer of group g (one thread, so the
-        // group's MMAs into its accumulators are issued in order by one thread)
-        const int g = warp - 2;
-        uint64_t* my_empty = a_empty + g * NSLOT;
-        const uint64_t desc0 = img_desc(ptx::smem_u32(img));
-        Cursor cur;
-        if (t_lo < t_hi) cur.start(a, lin0, t_lo);
-        uint32_t L = 0, tc = 0, qv = 0, qb = 0;
-        int prev_lin = -1;
-        // No early exit: the issuer meets its expander group at a named barrier every segment.
-        for (int T = t_lo; T < t_hi; ++T, ++tc) {
-            const bool new_lin = cur.lin != prev_lin;
-            if (new_lin) {
-                qb = qv % nb;
-                ++qv;
-                prev_lin = cur.lin;
-            }
-            const bool last_tile = cur.t_in + 1 == cur.ntiles || T + 1 == t_hi;
-            const uint32_t buf = tc & 1u;
-            const uint32_t d_lo = tmem_base + (uint32_t)(2 * g + (int)buf) * D_COLS;
-            const uint64_t bdesc = desc0 + (uint64_t)((qb * (uint32_t)a.img_bytes) >> 4);
-            for (int j = g; j < cur.nseg; j += NGRP, ++L) {
-                const uint32_t slot = L % NSLOT;
-                ptx::named_barrier(1 + g, 160);          // the group has written segment j into the slot
-                ptx::tc_fence_after();
-                if (ptx::elect_one()) {
-                    const bool first = j == g, last = j + NGRP >= cur.nseg;
-                    bool ok = true;
-                    if (first) {
-                        if (new_lin) ok = thread_wait(&q_full[qb], ((qv - 1) / nb) & 1u, abort_flag);
-                        ok = ok && thread_wait(&d_empty[buf], ((tc >> 1) & 1u) ^ 1u, abort_flag);
-                        if (!ok) fail(a.err, abort_flag);
-                        ptx::tc_fence_after();
-                    }
-                    if (!*abort_flag) {
-                        const uint32_t a_tmem = tmem_base + A_COL0 + (uint32_t)(g * NSLOT + (int)slot) * A_COLS;
-                        const uint64_t bj = bdesc + (uint64_t)(256 * j);
+            };
+            if (cb == kChunkBytes) {
+                // full chunk: whole groups, straight-line code
 #pragma unroll
-                        for (int p = 0; p < 4; ++p)
-                            ptx::mma_i8_ts(d_lo, a_tmem + 8 * p, bj + 32 * p, kIdesc, !first || p > 0);
+                for (int G = 0; G < kGroups; ++G) group(G, false);
+            } else {
+                const int ng = (cb + 31) >> 5;             // groups of 256 columns in this chunk
 #pragma unroll
-                        for (int p = 0; p < 4; ++p)
-                            ptx::mma_i8_ts(d_lo + NTOK, a_tmem + 32 + 8 * p, bj + 32 * (4 + p), kIdesc,
-                                           !first || p > 0);
-                    }
-                    // each commit arrives once this thread's earlier MMAs have completed
-                    ptx::mma_commit(&my_empty[slot]);
-                    if (last) {
-                        ptx::mma_commit(&d_full[buf]);
-                        if (last_tile) ptx::mma_commit(&q_empty[qb]);
-                    }
-                }
-                __syncwarp();
+                for (int G = 0; G < kGroups; ++G)
+                    if (G < ng) group(G, (cb - 32 * G) == 16);
             }
-            if (cur.nseg <= g && lane == 0) {
-                // no segment of this tile for the group: its arrivals, without MMAs
-                ptx::mbar_arrive(&d_full[buf]);
-                if (last_tile) ptx::mbar_arrive(&q_empty[qb]);
-            }
-            __syncwarp();
-            cur.advance(a);
-        }
-    } else if (warp >= 4 && warp < EPI_WARP0) {
-        // ------------------------------------------------ bit-plane expansion into TMEM
-        const int g = (warp - 4) >> 2;                    // segments j with j % 2 == g
-        const int q4 = warp & 3;                          // TMEM lanes 32 q4 .. 32 q4 + 31
-        const int r = q4 * 32 + lane;                     // tile row of this thread
-        const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
-        const uint32_t xr = (uint32_t)(r & 7);
-        const uint32_t row_off = (uint32_t)r * STAGE_ROW_BYTES;
-        uint64_t* my_empty = a_empty + g * NSLOT;
-        Cursor cur;
-        if (t_lo < t_hi) cur.start(a, lin0, t_lo);
-        uint32_t S = 0, L = 0;
-        // No early exit: the group meets its issuer at a named barrier every segment.
-        for (int T = t_lo; T < t_hi; ++T) {
-            for (int k = 0; k < cur.nstage; ++k, ++S) {
-                const int s = (int)(S % NS);
-                if (!warp_wait(&sign_full[s], (S / NS) & 1u, lane, abort_flag) && lane == 0) fail(a.err, abort_flag);
-                const uint8_t* stage = ring + s * SIGN_STAGE + row_off;
-                const int jn = min(4, cur.nseg - 4 * k);
-                for (int jj = g; jj < jn; jj += NGRP, ++L) {
-                    const uint32_t slot = L % NSLOT;
-                    // the segment's 32 sign bytes: 16-byte chunks 2 jj, 2 jj + 1 of this row (128B swizzle)
-                    const uint4 lo = *reinterpret_cast<const uint4*>(stage + (((2u * jj) ^ xr) << 4));
-                    const uint4 hi = *reinterpret_cast<const uint4*>(stage + (((2u * jj + 1u) ^ xr) << 4));
-                    const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-                    if (!warp_wait(&my_empty[slot], ((L / NSLOT) & 1u) ^ 1u, lane, abort_flag) && lane == 0)
-                        fail(a.err, abort_flag);
-                    ptx::tc_fence_after();
-                    const uint32_t taddr = tmem_base + lane_addr + A_COL0 + (uint32_t)(g * NSLOT + (int)slot) * A_COLS;
-                    {
-                        // columns 8 p + c: plane p (0..3) of word c as bytes 0 / 1
-                        uint32_t e[32];
-#pragma unroll
-                        for (int p = 0; p < 4; ++p)
-#pragma unroll
-                            for (int c = 0; c < 8; ++c) e[8 * p + c] = (w[c] >> p) & 0x01010101u;
-                        ptx::tmem_st_32x32b_x32(taddr, e);
-                    }
-                    {
-                        // columns 32 + 8 p + c: plane p + 4 of word c as bytes 0 / 16
-                        uint32_t e[32];
-#pragma unroll
-                        for (int p = 0; p < 4; ++p)
-#pragma unroll
-                            for (int c = 0; c < 8; ++c) e[8 * p + c] = (w[c] >> p) & 0x10101010u;
-                        ptx::tmem_st_32x32b_x32(taddr + 32, e);
-                    }
-                    ptx::tmem_st_wait();
-                    ptx::tc_fence_before();
-                    ptx::named_barrier(1 + g, 160);       // hand the segment to the group's issuer
-                }
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&sign_empty[s]);
-            }
-            cur.advance(a);
-        }
-    } else if (warp >= EPI_WARP0) {
-        // ------------------------------------------------ epilogue (one output row per thread)
-        const int q4 = warp & 3;
-        const int r = q4 * 32 + lane;
-        const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
-        const int m = a.m;
-        // this warp's copy of the current linear's per-token scalars
-        float* st_sx = stats + q4 * STAT_FLOATS;
-        int* st_sumq = reinterpret_cast<int*>(st_sx + NTOK);
-        float* st_u = st_sx + 2 * NTOK;
-        // Pointers of a linear are read once per linear, and the next tile's row parameters
-        // are loaded while the current tile is being computed.
-        struct EpiLin {
-            const float* alpha;
-            const float* sa;
-            const int8_t* wa;
-            void* y;
-            int32_t* acc;
-            int d_out;
-            bool bf16, ok;
-        };
-        auto load_lin = [&](int l) {
-            const dfssm_stack_entry& e = entry_at(a.entries, a.single, l);
-            EpiLin L;
-            L.ok = entry_ptrs_ok(e);
-            L.alpha = e.w.alpha;
-            L.sa = e.w.sa;
-            L.wa = e.w.wa;
-            L.y = e.y;
-            L.acc = e.dbg.acc;
-            L.d_out = a.desc[l].d_out;
-            L.bf16 = a.desc[l].y_dtype == DFSSM_BF16;
-            return L;
-        };
-        struct RowP {
-            float alpha, sa;
-            int4 wa;
-        };
-        auto load_row = [&](const EpiLin& L, int o) {
-            RowP p{0.f, 0.f, make_int4(0, 0, 0, 0)};
-            if (L.ok && o < L.d_out) {
-                p.alpha = L.alpha[o];
-                p.sa = L.sa[o];
-                p.wa = *reinterpret_cast<const int4*>(L.wa + (int64_t)o * kRank);
-            }
-            return p;
-        };
-        Cursor cur;
-        EpiLin lin{};
-        RowP row{0.f, 0.f, make_int4(0, 0, 0, 0)};
-        if (t_lo < t_hi) {
-            cur.start(a, lin0, t_lo);
-            lin = load_lin(cur.lin);
-            row = load_row(lin, cur.t_in * BM + r);
-        }
-        uint32_t tc = 0;
-        int prev_lin = -1;
-        bool waited = false;
-        for (int T = t_lo; T < t_hi && !*abort_flag; ++T, ++tc) {
-            if (cur.lin != prev_lin) {
-                if (!waited) { ptx::pdl_wait(); waited = true; }
-                prev_lin = cur.lin;
-                __syncwarp();
-                const TokStats* st = a.st_ws + a.desc[cur.lin].st_off;
-                for (int i = lane; i < m * 18; i += 32) {
-                    const int t = i / 18, f = i - 18 * t;
-                    if (f == 0) st_sx[t] = st[t].sx;
-                    else if (f == 1) st_sumq[t] = st[t].sumq;
-                    else st_u[t * kRank + f - 2] = st[t].u[f - 2];
-                }
-                __syncwarp();
-            }
-            const EpiLin L = lin;
-            const RowP rp = row;
-            const int o = cur.t_in * BM + r;
-            const int nseg = cur.nseg;
-            // prefetch the next tile's row parameters (and its linear's pointers)
-            if (T + 1 < t_hi) {
-                if (cur.advance(a)) lin = load_lin(cur.lin);
-                row = load_row(lin, cur.t_in * BM + r);
-            }
-            const uint32_t buf = tc & 1u;
-            if (!warp_wait(&d_full[buf], (tc >> 1) & 1u, lane, abort_flag)) {
-                if (lane == 0) fail(a.err, abort_flag);
-                break;
-            }
-            ptx::tc_fence_after();
-            // S1 = sum over groups of D_lo + D_hi / 16
-            int s_lo[NT], s_hi[NT];
-#pragma unroll
-            for (int j = 0; j < NT; ++j) s_lo[j] = s_hi[j] = 0;
-            const int ngrp = nseg < NGRP ? nseg : NGRP;
-            for (int g = 0; g < ngrp; ++g) {
-                uint32_t vl[NT], vh[NT];
-                const uint32_t col = tmem_base + lane_addr + (uint32_t)(2 * g + (int)buf) * D_COLS;
-                ptx::tmem_ld_32x32b<NT>(col, vl);
-                ptx::tmem_ld_32x32b<NT>(col + NTOK, vh);
-                ptx::tmem_ld_wait();
-#pragma unroll
-                for (int j = 0; j < NT; ++j) {
-                    s_lo[j] += (int)vl[j];
-                    s_hi[j] += (int)vh[j];
-                }
-            }
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&d_empty[buf]);
-            if (L.ok && o < L.d_out) {
-                const WaRow wa = wa_row_from_int4(rp.wa);
-#pragma unroll
-                for (int j = 0; j < NT; ++j) {
-                    if (j >= m) break;
-                    const int acc = 2 * (s_lo[j] + (s_hi[j] >> 4)) - st_sumq[j];
-                    const float y = dequant(st_sx[j], rp.alpha, rp.sa, acc, lora_dot(wa, st_u + j * kRank));
-                    const int64_t idx = (int64_t)j * L.d_out + o;
-                    if (L.bf16) reinterpret_cast<uint16_t*>(L.y)[idx] = f32_to_bf16_bits(y);
-                    else reinterpret_cast<float*>(L.y)[idx] = y;
-                    if (L.acc) L.acc[idx] = acc;
-                }
-            }
-        }
-    }
 
-    // ------------------------------------------------ teardown
-    __syncwarp();
-    ptx::tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+            // ---- epilogue after the block's last k-chunk
+            if (last_chunk) {
+                // combine the bit-position accumulators: T = sum_p D_p * 2^(7-p) = 128 * S1
+                int T[RT][NT][4];
+#pragma unroll
+                for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            int s = 0;
+                            if ((r & 1) == 0 || m > 1) {
+#pragma unroll
+                                for (int p = 0; p < 8; ++p) s += D[rt][nt][p][r] << (7 - p);
+                            }
+                            T[rt][nt][r] = s;
+                        }
+                // lane -> (row of this warp, n-tile); D fragment of (row, token t) sits in
+                // thread (row % 8) * 4 + (t % 8) / 2, register 2 * ((row / 8) % 2) + t % 2
+                constexpr int kRowsW = 16 * RT;
+                const int my_row = lane % kRowsW;
+                const int my_nt = lane / kRowsW;            // 0, or 1 when RT = 1 and NT = 2
+                const int rr = wrow0 + my_row;
+                const bool row_ok = rr < nrows;
+                const float* alpha_s = reinterpret_cast<const float*>(slot + R * kChunkBytes);
+                const float* sa_s = alpha_s + R;
+                const int4* wa_s = reinterpret_cast<const int4*>(slot + R * kChunkBytes + 8 * R);
+                const float alpha = alpha_s[rr], sa = sa_s[rr];
+                const WaRow wa = wa_row_from_int4(wa_s[rr]);
+                const int jmax = NT == 1 ? m : 8;
+                for (int j = 0; j < jmax; ++j) {
+                    const int src = (my_row & 7) * 4 + (j >> 1);
+                    int v_lo[RT][NT], v_hi[RT][NT];
+#pragma unroll
+                    for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            v_lo[rt][nt] = __shfl_sync(0xffffffffu, T[rt][nt][j & 1], src);
+                            v_hi[rt][nt] = __shfl_sync(0xffffffffu, T[rt][nt][2 + (j & 1)], src);
+                        }
+                    int val = 0;
+#pragma unroll
+                    for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt)
+                            if (rt == (my_row >> 4) && nt == my_nt) val = ((my_row >> 3) & 1) ? v_hi[rt][nt] : v_lo[rt][nt];
+                    const int t = 8 * my_nt + j;
+                    if (t < m && row_ok) {
+                        const int acc = 2 * (val >> 7) - ts.sumq[t];
+                        const float y = dequant(ts.sx[t], alpha, sa, acc, lora_dot(wa, ts.u[t]));
+                        const int64_t idx = (int64_t)t * L.d_out + row0 + rr;
+                        if (L.y_dtype == DFSSM_BF16)
+                            reinterpret_cast<uint16_t*>(L.y)[idx] = f32_to_bf16_bits(y);
+                        else
+                            reinterpret_cast<float*>(L.y)[idx] = y;
+                        if (L.dbg_acc) L.dbg_acc[idx] = acc;
+                    }
+                }
+            }
+        }
+        __syncthreads();     // slot it % kStages is refilled by the next iteration
+        cw.advance(a);
     }
+    ptx::cp_async_wait<0>();
 }
 
-size_t smem_bytes(int img_bytes, int img_bufs) {
-    return 1024 + (size_t)NS * SIGN_STAGE + (size_t)img_bufs * img_bytes + sizeof(float) * 4 * STAT_FLOATS + 128 +
-           8 * (2 * NS + NGRP * NSLOT + 8) + 32;
+struct Geometry {
+    int slot_bytes, q_region;
+    size_t smem;
+};
+
+template <int RT>
+Geometry geometry(int m, int max_d_in) {
+    constexpr int R = 16 * RT * kWarps;
+    Geometry g;
+    g.slot_bytes = (R * kChunkBytes + R * (4 + 4 + kRank) + 127) & ~127;
+    g.q_region = (m * q_stride(max_d_in) + 127) & ~127;
+    g.smem = ((sizeof(TokShared) + 127) & ~(size_t)127) + g.q_region + (size_t)kStages * g.slot_bytes;
+    return g;
 }
 
-template <int NT>
-cudaError_t launch_nt(const LaunchCtx& c, const DecodeArgs& a, size_t smem, int grid) {
+template <int RT, int NT>
+cudaError_t launch_cfg(const LaunchCtx& c) {
+    constexpr int R = 16 * RT * kWarps;
+    const Geometry geo = geometry<RT>(c.m, c.max_d_in);
+    int64_t total_bytes = 0;
+    int blocks = 0;
+    for (int i = 0; i < c.n; ++i) {
+        total_bytes += (int64_t)c.host_desc[i].d_out * (c.host_desc[i].d_in / 8);
+        blocks += (c.host_desc[i].d_out + R - 1) / R;
+    }
+    int per_sm = 0;
+    cudaError_t err =
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<RT, NT>, kThreads, geo.smem);
+    if (err != cudaSuccess) return err;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    int grid = c.sm_count * per_sm;
+    if (grid > blocks) grid = blocks;
+    DecodeArgs a{c.entries, c.single, c.desc, c.n, c.m, c.st_ws, total_bytes, geo.slot_bytes, geo.q_region};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(THREADS);
-    cfg.dynamicSmemBytes = smem;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = geo.smem;
     cfg.stream = c.stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_kernel<NT>, a);
+    return cudaLaunchKernelEx(&cfg, decode_kernel<RT, NT>, a);
 }
-
-template <int NT>
-cudaError_t set_attr_nt(int optin) {
-    return allow_dyn_smem(decode_kernel<NT>, optin);
-}
-
-int g_optin = 0;
 
 }  // namespace
 
-int decode_map_slots() { return kMapSlots; }
-int decode_tile_rows() { return BM; }
-int decode_stage_bytes() { return STAGE_ROW_BYTES; }
-
 cudaError_t launch_decode(const LaunchCtx& c) {
-    int64_t total_bytes = 0;
-    int tiles = 0, max_qrow = 0;
-    for (int i = 0; i < c.n; ++i) {
-        total_bytes += (int64_t)c.host_desc[i].d_out * (c.host_desc[i].d_in / 8);
-        tiles += (c.host_desc[i].d_out + BM - 1) / BM;
-        max_qrow = max(max_qrow, c.host_desc[i].qrow);
-    }
-    const int img_bytes = NTOK * max_qrow;
-    const int bufs = smem_bytes(img_bytes, 2) <= (size_t)g_optin ? 2 : 1;
-    const size_t smem = smem_bytes(img_bytes, bufs);
-    if (smem > (size_t)g_optin) return cudaErrorInvalidConfiguration;
-    int grid = c.sm_count < tiles ? c.sm_count : tiles;
-    if (grid > c.map_slot_ctas) grid = c.map_slot_ctas;
-    DecodeArgs a{c.entries, c.single, c.desc, reinterpret_cast<const CUtensorMap*>(c.sign_tmpl),
-                 reinterpret_cast<CUtensorMap*>(c.map_slots), c.q_ws, c.st_ws, c.err, c.n, c.m, tiles, img_bytes,
-                 bufs, total_bytes};
-    if (c.m <= 1) return launch_nt<1>(c, a, smem, grid);
-    if (c.m <= 2) return launch_nt<2>(c, a, smem, grid);
-    if (c.m <= 4) return launch_nt<4>(c, a, smem, grid);
-    if (c.m <= 8) return launch_nt<8>(c, a, smem, grid);
-    return launch_nt<16>(c, a, smem, grid);
+    if (c.m <= 8) return launch_cfg<2, 1>(c);
+    return launch_cfg<1, 2>(c);
 }
 
 cudaError_t set_decode_attr(int optin) {
-    cudaError_t e = set_attr_nt<1>(optin);
-    if (e == cudaSuccess) e = set_attr_nt<2>(optin);
-    if (e == cudaSuccess) e = set_attr_nt<4>(optin);
-    if (e == cudaSuccess) e = set_attr_nt<8>(optin);
-    if (e == cudaSuccess) e = set_attr_nt<16>(optin);
-    if (e == cudaSuccess) {
-        cudaFuncAttributes fa;
-        e = cudaFuncGetAttributes(&fa, decode_kernel<16>);
-        if (e == cudaSuccess) g_optin = optin - (int)fa.sharedSizeBytes;
-    }
-    return e;
+    cudaError_t e = allow_dyn_smem(decode_kernel<2, 1>, optin);
+    return e != cudaSuccess ? e : allow_dyn_smem(decode_kernel<1, 2>, optin);
 }
 
 }  // namespace dfssm

@@ -47,14 +47,12 @@ struct dfssm_plan_s {
     int* part = nullptr;
     unsigned int* tickets = nullptr;
     CUtensorMap* tmaps = nullptr;       // prefill: activation rows of each linear
-    CUtensorMap* sign_tmpl = nullptr;   // decode: sign rows of each linear, address set on the device
-    CUtensorMap* map_slots = nullptr;   // decode: per-CTA tensor maps edited on the device
     size_t ws_bytes = 0;
 };
 
 namespace {
 
-constexpr int kDecodeMaxM = kImgTokens;   // the quantisation kernel writes the decode image up to here
+constexpr int kDecodeMaxM = kDecodeMaxTokens;
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -105,8 +103,6 @@ void free_plan(dfssm_plan_s* p) {
     if (p->part) cudaFree(p->part);
     if (p->tickets) cudaFree(p->tickets);
     if (p->tmaps) cudaFree(p->tmaps);
-    if (p->sign_tmpl) cudaFree(p->sign_tmpl);
-    if (p->map_slots) cudaFree(p->map_slots);
     delete p;
 }
 
@@ -164,9 +160,7 @@ dfssm_status dfssm_linear_plan(const dfssm_linear_desc* descs, int n_descs, dfss
         d.y_dtype = descs[i].y_dtype;
         d.max_m = descs[i].max_m;
         d.qrow = seg_qrow(d.d_in);
-        // every region is a multiple of 256 bytes, so every offset stays 256-byte aligned
-        d.dq_off = q_bytes;
-        q_bytes += (int64_t)kImgTokens * d.qrow;
+        // activation rows only for the prefill; every region is a multiple of 256 bytes
         d.q_off = q_bytes;
         if (d.max_m > kDecodeMaxM) q_bytes += (int64_t)d.max_m * d.qrow;
         d.st_off = st_count;
@@ -176,15 +170,12 @@ dfssm_status dfssm_linear_plan(const dfssm_linear_desc* descs, int n_descs, dfss
         st_count += d.max_m;
         rt += (d.d_out + 127) / 128;
     }
-    const int n_slots = p->sm_count * decode_map_slots();
     cudaError_t e = cudaSuccess;
     e = cudaMalloc(&p->ddesc, sizeof(DevDesc) * n_descs);
-    if (e == cudaSuccess) e = cudaMalloc(&p->q_ws, (size_t)q_bytes);
+    if (e == cudaSuccess) e = cudaMalloc(&p->q_ws, (size_t)(q_bytes > 0 ? q_bytes : 256));
     if (e == cudaSuccess) e = cudaMalloc(&p->st_ws, sizeof(TokStats) * (size_t)st_count);
     if (e == cudaSuccess) e = cudaMalloc(&p->err, 16);
     if (e == cudaSuccess) e = cudaMalloc(&p->tmaps, sizeof(CUtensorMap) * n_descs);
-    if (e == cudaSuccess) e = cudaMalloc(&p->sign_tmpl, sizeof(CUtensorMap) * n_descs);
-    if (e == cudaSuccess) e = cudaMalloc(&p->map_slots, sizeof(CUtensorMap) * n_slots);
     const size_t part_bytes = sizeof(int) * (size_t)n_descs * kMaxSplits * kPartTok * 20;
     if (e == cudaSuccess) e = cudaMalloc(&p->part, part_bytes);
     if (e == cudaSuccess) e = cudaMalloc(&p->tickets, sizeof(unsigned int) * n_descs);
@@ -194,14 +185,11 @@ dfssm_status dfssm_linear_plan(const dfssm_linear_desc* descs, int n_descs, dfss
         return e == cudaErrorMemoryAllocation ? DFSSM_ERR_NO_MEMORY : DFSSM_ERR_CUDA;
     }
     p->ws_bytes = sizeof(DevDesc) * n_descs + (size_t)q_bytes + sizeof(TokStats) * st_count + 16 +
-                  sizeof(CUtensorMap) * (2 * n_descs + n_slots) + part_bytes + sizeof(unsigned int) * n_descs;
+                  sizeof(CUtensorMap) * n_descs + part_bytes + sizeof(unsigned int) * n_descs;
 
-    // prefill: tensor maps over each linear's activation rows (B operand, 128-byte swizzle);
-    // decode: tensor maps over each linear's sign rows with a placeholder address (the
-    // kernel sets the address of the call's sign tensor)
-    std::vector<CUtensorMap> tm(n_descs), sm(n_descs);
+    // prefill: tensor maps over each linear's activation rows (B operand, 128-byte swizzle)
+    std::vector<CUtensorMap> tm(n_descs);
     std::memset(tm.data(), 0, sizeof(CUtensorMap) * n_descs);
-    std::memset(sm.data(), 0, sizeof(CUtensorMap) * n_descs);
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) { free_plan(p); return DFSSM_ERR_CUDA; }
     for (int i = 0; i < n_descs; ++i) {
@@ -216,13 +204,8 @@ dfssm_status dfssm_linear_plan(const dfssm_linear_desc* descs, int n_descs, dfss
                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
             if (r != CUDA_SUCCESS) { free_plan(p); return DFSSM_ERR_CUDA; }
         }
-        if (encode_sign_map(enc, &sm[i], p->q_ws, d.d_in, d.d_out) != CUDA_SUCCESS) {
-            free_plan(p);
-            return DFSSM_ERR_CUDA;
-        }
     }
     e = cudaMemcpy(p->tmaps, tm.data(), sizeof(CUtensorMap) * n_descs, cudaMemcpyHostToDevice);
-    if (e == cudaSuccess) e = cudaMemcpy(p->sign_tmpl, sm.data(), sizeof(CUtensorMap) * n_descs, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(p->ddesc, p->hdesc.data(), sizeof(DevDesc) * n_descs, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemset(p->err, 0, 16);
     if (e == cudaSuccess) e = cudaMemset(p->tickets, 0, sizeof(unsigned int) * n_descs);
@@ -284,9 +267,6 @@ dfssm_status dfssm_linear_fwd(dfssm_plan plan, int32_t desc_index, const dfssm_l
     c.part = plan->part + (size_t)desc_index * kMaxSplits * kPartTok * 20;
     c.tickets = plan->tickets + desc_index;
     c.tmaps = plan->tmaps + desc_index;
-    c.sign_tmpl = plan->sign_tmpl + desc_index;
-    c.map_slots = plan->map_slots;
-    c.map_slot_ctas = plan->sm_count;
     c.max_d_in = hd.d_in;
     c.total_rows = hd.d_out;
     c.sm_count = plan->sm_count;
@@ -320,9 +300,6 @@ dfssm_status dfssm_linear_stack_fwd(dfssm_plan plan, const dfssm_stack_entry* en
     c.part = plan->part;
     c.tickets = plan->tickets;
     c.tmaps = plan->tmaps;
-    c.sign_tmpl = plan->sign_tmpl;
-    c.map_slots = plan->map_slots;
-    c.map_slot_ctas = plan->sm_count;
     c.max_d_in = max_d_in;
     c.total_rows = rows;
     c.sm_count = plan->sm_count;

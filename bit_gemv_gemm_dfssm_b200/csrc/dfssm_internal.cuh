@@ -22,8 +22,7 @@ struct DevDesc {
     int32_t d_out;
     int32_t y_dtype;
     int32_t max_m;
-    int64_t q_off;      // byte offset of this linear's activation rows (prefill layout) in the q workspace
-    int64_t dq_off;     // byte offset of its 16-token activation image (decode layout)
+    int64_t q_off;      // byte offset of this linear's activation rows (prefill) in the q workspace
     int64_t st_off;     // index of its first TokStats record
     int32_t qrow;       // activation bytes per token: d_in rounded up to a whole 256-column segment
     int32_t rt_begin;   // first 128-row tile of this linear in the flattened stack order
@@ -44,21 +43,16 @@ struct alignas(16) TokStats {
 static_assert(sizeof(TokStats) == 80, "TokStats layout");
 static_assert(sizeof(dfssm_stack_entry) == 104, "dfssm_stack_entry layout");
 
-// Activation layouts in the q workspace. The columns of a row are taken in
-// segments of 256 (a final half segment is padded to 256 with zeros); inside a
-// segment the int8 value of column 32c + 8i + p (c = 0..7: 32-bit word of the
-// sign row, i = 0..3: byte of that word, p = 0..7: bit of that byte) sits at
-// K position 32p + 4c + i. With this plane-major order the four bytes that
-// w_c & (0x01010101 << p) selects from sign word c meet four consecutive
-// activation bytes of plane p, and the 32 bytes of plane p form one K = 32 step
-// of an int8 MMA.
-//  * prefill rows: token t, segment s at q_off + t * qrow + 256 s (K-major rows,
-//    loaded by TMA with 128-byte swizzle);
-//  * decode image (always 16 tokens): the 512-byte unit u = 8 s + p holds K step
-//    (s, p) for the 16 tokens as 8-row x 16-byte core matrices: token t, K byte k
-//    at dq_off + 512 u + 256 (t / 8) + 128 (k / 16) + 16 (t % 8) + k % 16.
+// Activation layout in the q workspace (the prefill's B operand). The columns of
+// a row are taken in segments of 256 (a final half segment is padded to 256);
+// inside a segment the int8 value of column 32c + 8i + p (c = 0..7: 32-bit word
+// of the sign row, i = 0..3: byte of that word, p = 0..7: bit of that byte) sits
+// at K position 32p + 4c + i. With this plane-major order the four bytes of
+// bit plane p of sign word c meet four consecutive activation bytes, and the 32
+// bytes of plane p form one K = 32 step of an int8 MMA. Token t, segment s is at
+// q_off + t * qrow + 256 s (K-major rows, loaded by TMA with 128-byte swizzle).
 constexpr int kSegCols = 256;
-constexpr int kImgTokens = 16;
+constexpr int kDecodeMaxTokens = 16;   // m up to this runs the decode kernel
 __host__ __device__ inline int seg_qrow(int d_in) { return (d_in + kSegCols - 1) / kSegCols * kSegCols; }
 
 // ---- launch wrappers implemented in the .cu files ---------------------------------
@@ -76,9 +70,6 @@ struct LaunchCtx {
     int* part;                         // split partials: n x kMaxSplits x 16 tokens x 20 ints
     unsigned int* tickets;             // n split tickets, zero between calls
     const void* tmaps;                 // device array of CUtensorMap (prefill activation rows), one per desc
-    const void* sign_tmpl;             // device array of CUtensorMap (sign rows, placeholder address), one per desc
-    void* map_slots;                   // device scratch: decode_map_slots() tensor maps per decode CTA
-    int map_slot_ctas;                 // CTAs the slots cover
     int max_d_in;                      // largest d_in among the n linears
     int64_t total_rows;                // sum of d_out over the n linears
     int sm_count;
@@ -90,9 +81,6 @@ cudaError_t launch_pack_sign(const void* src, int src_dtype, int d_out, int d_in
 cudaError_t launch_quant(const LaunchCtx& c);
 cudaError_t launch_decode(const LaunchCtx& c);
 cudaError_t launch_prefill(const LaunchCtx& c);
-int decode_map_slots();      // tensor-map slots per decode CTA
-int decode_tile_rows();      // rows per sign TMA box (and per decode tile)
-int decode_stage_bytes();    // bytes per row of a sign TMA box
 
 // ---- tensor maps (host side) ----------------------------------------------------------
 
@@ -111,20 +99,6 @@ inline EncodeTiledFn get_encode_fn() {
         return nullptr;
     fn = reinterpret_cast<EncodeTiledFn>(p);
     return fn;
-}
-
-// Sign rows of one linear (d_out rows of d_in / 8 bytes) as the decode kernel loads them:
-// boxes of decode_tile_rows() rows x decode_stage_bytes() bytes, 128-byte swizzle, zero fill
-// outside the tensor. `base` is the tensor's address (any 16-byte aligned placeholder when
-// the kernel sets the address itself).
-inline CUresult encode_sign_map(EncodeTiledFn enc, CUtensorMap* map, const void* base, int d_in, int d_out) {
-    cuuint64_t dims[2] = {(cuuint64_t)(d_in / 8), (cuuint64_t)d_out};
-    cuuint64_t strides[1] = {(cuuint64_t)(d_in / 8)};
-    cuuint32_t box[2] = {(cuuint32_t)decode_stage_bytes(), (cuuint32_t)decode_tile_rows()};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
 // Allow `kernel` the opt-in dynamic shared memory (minus its static shared memory).

@@ -5,9 +5,8 @@
 // captured, allocators that must not be re-entered, or embedders whose memory
 // budget is fixed up front. This entry point needs no plan: the quantisation
 // and decode kernels run exactly as for dfssm_linear_fwd, with their scratch
-// (per-token scalars, split partials and their ticket, the int8 activation
-// image, the linear's descriptor and sign tensor map, the decode kernel's
-// tensor-map slots and the error word) in the file-scope device array
+// (per-token scalars, split partials and their ticket, the linear's
+// descriptor and the error word) in the file-scope device array
 // below, which every GPU that loads this library keeps until the process exits.
 //
 // Limits: 1 <= m <= DFSSM_NOALLOC_MAX_M (16) tokens, 128 <= d_in <= 8192.
@@ -15,7 +14,6 @@
 // without ordering) race on it. The first call on a device looks up the array's
 // device address (cudaGetSymbolAddress) and sets the kernels' shared-memory
 // limits; make that first call before any stream capture.
-#include <cstddef>
 #include <cstring>
 #include <mutex>
 
@@ -31,30 +29,16 @@ namespace {
 constexpr int kNoAllocMaxM = DFSSM_NOALLOC_MAX_M;
 constexpr int kMaxDevices = 64;
 
-constexpr int kMaxCtas = 256;          // decode CTAs the tensor-map slots cover
-
 // scratch layout (byte offsets, 256-byte aligned pieces)
 constexpr size_t kOffDesc = 0;                                                      // DevDesc
-constexpr size_t kOffTmpl = 256;                                                    // sign tensor map (128 B)
-constexpr size_t kOffErr = 512;                                                     // uint32 error word
-constexpr size_t kOffTicket = 768;                                                  // split ticket
-constexpr size_t kOffStats = 1024;                                                  // TokStats[16]
+constexpr size_t kOffErr = 256;                                                     // uint32 error word
+constexpr size_t kOffTicket = 512;                                                  // split ticket
+constexpr size_t kOffStats = 768;                                                   // TokStats[16]
 constexpr size_t kOffPart = kOffStats + ((sizeof(TokStats) * kNoAllocMaxM + 255) & ~(size_t)255);
 constexpr size_t kPartBytes = sizeof(int) * kMaxSplits * kPartTok * 20;
-constexpr size_t kOffQ = kOffPart + ((kPartBytes + 255) & ~(size_t)255);          // 16-token activation image
-constexpr size_t kOffSlots = kOffQ + (size_t)kImgTokens * kMaxDIn;                // decode tensor-map slots
-constexpr size_t kScratchBytes = kOffSlots + (size_t)kMaxCtas * 4 * sizeof(CUtensorMap);   // about 270 KB
+constexpr size_t kScratchBytes = kOffPart + ((kPartBytes + 255) & ~(size_t)255);  // about 8 KB
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kScratchBytes];
-
-// what each call copies to the head of the scratch
-struct HostHead {
-    DevDesc desc;
-    uint8_t pad[kOffTmpl - sizeof(DevDesc)];
-    CUtensorMap tmpl;
-};
-static_assert(sizeof(DevDesc) <= kOffTmpl, "scratch head layout");
-static_assert(offsetof(HostHead, tmpl) == kOffTmpl, "scratch head layout");
 
 struct DeviceSetup {
     uint8_t* scratch = nullptr;   // device address of g_noalloc_scratch on this device
@@ -111,21 +95,16 @@ extern "C" dfssm_status dfssm_linear_fwd_noalloc(const dfssm_linear_desc* desc, 
     dfssm_status st = setup_device(dev, &s);
     if (st != DFSSM_OK) return st;
 
-    EncodeTiledFn enc = get_encode_fn();
-    if (!enc) return DFSSM_ERR_CUDA;
-    HostHead head;
-    std::memset(&head, 0, sizeof(head));
-    DevDesc& hd = head.desc;
+    DevDesc hd;
+    std::memset(&hd, 0, sizeof(hd));
     hd.d_in = desc->d_in;
     hd.d_out = desc->d_out;
     hd.y_dtype = desc->y_dtype;
     hd.max_m = kNoAllocMaxM;
     hd.qrow = seg_qrow(desc->d_in);
-    // the sign map gets this call's address here; the kernel sets the same address again
-    if (encode_sign_map(enc, &head.tmpl, w->sign, desc->d_in, desc->d_out) != CUDA_SUCCESS) return DFSSM_ERR_CUDA;
     DevDesc* ddesc = reinterpret_cast<DevDesc*>(s->scratch + kOffDesc);
-    // descriptor and sign map go into the scratch on the stream (a small host-to-device copy, no allocation)
-    if (cudaMemcpyAsync(s->scratch, &head, sizeof(head), cudaMemcpyHostToDevice, (cudaStream_t)stream) != cudaSuccess)
+    // the descriptor goes into the scratch on the stream (a small host-to-device copy, no allocation)
+    if (cudaMemcpyAsync(ddesc, &hd, sizeof(hd), cudaMemcpyHostToDevice, (cudaStream_t)stream) != cudaSuccess)
         return DFSSM_ERR_CUDA;
 
     LaunchCtx c{};
@@ -138,15 +117,12 @@ extern "C" dfssm_status dfssm_linear_fwd_noalloc(const dfssm_linear_desc* desc, 
     c.m = m;
     c.desc = ddesc;
     c.host_desc = &hd;
-    c.q_ws = reinterpret_cast<int8_t*>(s->scratch + kOffQ);
+    c.q_ws = nullptr;     // the decode kernel quantises into shared memory; no activation rows are stored
     c.st_ws = reinterpret_cast<TokStats*>(s->scratch + kOffStats);
     c.err = reinterpret_cast<uint32_t*>(s->scratch + kOffErr);
     c.part = reinterpret_cast<int*>(s->scratch + kOffPart);
     c.tickets = reinterpret_cast<unsigned int*>(s->scratch + kOffTicket);   // zero at load, reset by each call
     c.tmaps = nullptr;
-    c.sign_tmpl = s->scratch + kOffTmpl;
-    c.map_slots = s->scratch + kOffSlots;
-    c.map_slot_ctas = kMaxCtas;
     c.max_d_in = desc->d_in;
     c.total_rows = desc->d_out;
     c.sm_count = s->sm_count;

@@ -11,9 +11,8 @@
 //   sumq   = sum_j q[t,j]                          (int32)
 //   h[t,k] = sum_j W_B[k,j] q[t,j]                 (int32, warp MMA s8 x s8)
 //   u[t,k] = s_B[k] * h[t,k]                       (fp32)
-// and stores q in the plane-major int8 layouts the scaffold kernels read (the
-// 16-token decode image for m <= 16, token rows for the prefill otherwise),
-// plus s_x, sumq and u.
+// and, for the prefill (m > 16), stores q in the plane-major int8 rows its
+// tensor-core kernel reads, plus s_x, sumq and u.
 //
 // A block owns one linear and up to kTokPerBlock tokens, processed in rounds of
 // 16 tokens (one MMA tile). The 8 warps split the 32-column k-blocks of d_in
@@ -271,27 +270,28 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__
         // (columns 32c + 8i + p, i = 0..3) as byte p % 4 of W[p / 4], W[2 + p / 4], W[4 + p / 4],
         // W[6 + p / 4]; the four groups' words of plane p form one 16-byte piece.
         const int npc = pc_hi - pc_lo;
-        const bool to_image = m <= kImgTokens;
+        // the decode kernel (m <= 16) quantises into its own shared memory; only the prefill reads rows
+        const bool rows = m > kDecodeMaxTokens;
         for (int i = tid; i < nt * npc; i += kThreads) {
             const int tk = i / npc, pc = pc_lo + (i - tk * npc);
             const int sg = pc >> 1, hc = pc & 1, t = t0 + tk;
             const uint32_t* src = reinterpret_cast<const uint32_t*>(q_s + tk * d_in + 128 * pc);
-            uint32_t P[8][4];
+            if (rows) {
+                uint32_t P[8][4];
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                const uint32_t* W = src + 8 * c4;
-                const uint4 lo = transpose4x4(W[0], W[2], W[4], W[6]);   // planes 0..3
-                const uint4 hi = transpose4x4(W[1], W[3], W[5], W[7]);   // planes 4..7
-                P[0][c4] = lo.x; P[1][c4] = lo.y; P[2][c4] = lo.z; P[3][c4] = lo.w;
-                P[4][c4] = hi.x; P[5][c4] = hi.y; P[6][c4] = hi.z; P[7][c4] = hi.w;
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const uint32_t* W = src + 8 * c4;
+                    const uint4 lo = transpose4x4(W[0], W[2], W[4], W[6]);   // planes 0..3
+                    const uint4 hi = transpose4x4(W[1], W[3], W[5], W[7]);   // planes 4..7
+                    P[0][c4] = lo.x; P[1][c4] = lo.y; P[2][c4] = lo.z; P[3][c4] = lo.w;
+                    P[4][c4] = hi.x; P[5][c4] = hi.y; P[6][c4] = hi.z; P[7][c4] = hi.w;
+                }
+                // plane p of segment sg, K half hc: 16 bytes at 256 sg + 32 p + 16 hc of the token row
+                int8_t* base = q_ws + d.q_off + (int64_t)t * d.qrow + 256 * sg + 16 * hc;
+#pragma unroll
+                for (int p = 0; p < 8; ++p)
+                    *reinterpret_cast<uint4*>(base + 32 * p) = make_uint4(P[p][0], P[p][1], P[p][2], P[p][3]);
             }
-            // decode image: unit 8 sg + p, token group t / 8, K half hc, row t % 8; prefill rows: 32 p + 16 hc
-            int8_t* base = to_image ? q_ws + d.dq_off + 4096 * sg + 256 * (t >> 3) + 128 * hc + 16 * (t & 7)
-                                    : q_ws + d.q_off + (int64_t)t * d.qrow + 256 * sg + 16 * hc;
-            const int pstride = to_image ? 512 : 32;
-#pragma unroll
-            for (int p = 0; p < 8; ++p)
-                *reinterpret_cast<uint4*>(base + p * pstride) = make_uint4(P[p][0], P[p][1], P[p][2], P[p][3]);
             if (e.dbg.q) {
                 const uint4* sq = reinterpret_cast<const uint4*>(src);
                 uint4* dq = reinterpret_cast<uint4*>(e.dbg.q + (int64_t)t * d_in + 128 * pc);
