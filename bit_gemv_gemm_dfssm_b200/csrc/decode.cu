@@ -423,7 +423,10 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
                 const float alpha = alpha_s[rr], sa = sa_s[rr];
                 const WaRow wa = wa_row_from_int4(wa_s[rr]);
                 const int jmax = NT == 1 ? m : 8;
-                for (int j = 0; j < jmax; ++j) {
+                // j unrolled so every register index is a constant (no local-memory copy of T)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (j >= jmax) break;
                     const int src = (my_row & 7) * 4 + (j >> 1);
                     int v_lo[RT][NT], v_hi[RT][NT];
 #pragma unroll
