@@ -159,16 +159,21 @@ __device__ __forceinline__ void issue_step(const Cursor& c, const Lin& L, uint8_
     const int row0 = c.b * R;
     const int nrows = min(R, L.d_out - row0);
     const int nch = min(kChunkBytes, L.rb - kChunkBytes * c.kc) >> 4;   // 16-byte pieces in this chunk
-    const uint8_t* src = L.sign + (int64_t)row0 * L.rb + kChunkBytes * c.kc;
-    // thread t copies 16-byte piece j = t % kChunkJ of rows t / kChunkJ + k * kRowStep
+    // thread t copies 16-byte piece j = t % kChunkJ of rows r0 + k * kRowStep (r0 = t / kChunkJ),
+    // each to its rotated position (j + r) mod kChunkJ
     constexpr int kRowStep = kThreads / kChunkJ;
+    static_assert(R % kRowStep == 0, "copy pattern");
     const int j = threadIdx.x % kChunkJ;
-    int r = threadIdx.x / kChunkJ;
+    const int r0 = threadIdx.x / kChunkJ;
     if (j < nch) {
-        const uint8_t* s0 = src + (int64_t)r * L.rb + 16 * j;
+        const uint8_t* s0 = L.sign + (int64_t)(row0 + r0) * L.rb + kChunkBytes * c.kc + 16 * j;
         const int64_t sstep = (int64_t)kRowStep * L.rb;
-        for (; r < nrows; r += kRowStep, s0 += sstep)
-            ptx::cp_async16(slot + r * kChunkBytes + 16 * ((j + r) % kChunkJ), s0);
+        const uint32_t d0 = ptx::smem_u32(slot) + r0 * kChunkBytes;
+#pragma unroll
+        for (int k = 0; k < R / kRowStep; ++k)
+            if (r0 + k * kRowStep < nrows)
+                ptx::cp_async16_s(d0 + k * kRowStep * kChunkBytes + 16 * ((j + r0 + k * kRowStep) & (kChunkJ - 1)),
+                                  s0 + k * sstep);
     }
     if (c.kc == L.nchunks - 1) {
         uint8_t* par = slot + R * kChunkBytes;
@@ -292,6 +297,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
     const int lm_row = (lane & 7) + 8 * ((lane >> 3) & 1);
     const int lm_hi = lane >> 4;
     const int wrow0 = warp * 16 * RT;             // first row of this warp in a block
+    const int q_off = (int)(q_s - smem);          // staged q, as an offset into the shared array
 
     for (int it = 0; cw.valid(a, hi); ++it) {
         const Lin& L = cw.L;
@@ -335,8 +341,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
             const int cb = min(kChunkBytes, L.rb - kChunkBytes * cw.c.kc);
             const uint32_t slot_s = ptx::smem_u32(slot);
             // ldmatrix row addresses: row r's 16-byte piece j sits at (j + r) mod kChunkJ; rows
-            // of a tile are 8-aligned, so the rotation depends on (lane % 8) only
-            const int rot = (lm_row & 7) + lm_hi;
+            // of a tile start at multiples of 16, so the rotation depends on the lane only
+            const int rot = (lm_row & (kChunkJ - 1)) + lm_hi;
             uint32_t a_addr[RT][kGroups];
 #pragma unroll
             for (int rt = 0; rt < RT; ++rt)
@@ -344,11 +350,12 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
                 for (int G = 0; G < kGroups; ++G)
                     a_addr[rt][G] = slot_s + (wrow0 + 16 * rt + lm_row) * kChunkBytes + 16 * ((2 * G + rot) % kChunkJ);
             // B rows: tokens nt * 8 + g; lanes past m read token 0 (their MMA columns are never stored)
-            const uint8_t* qk[NT][4];
+            // (32-bit offsets into the shared array, so the loads need no 64-bit address math)
+            int qk[NT][4];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 const int tk = nt * 8 + g;
-                const uint8_t* qrow = q_s + (tk < m ? tk : 0) * qstride + 256 * (kGroups * cw.c.kc) + 64 * c;
+                const int qrow = q_off + (tk < m ? tk : 0) * qstride + 256 * (kGroups * cw.c.kc) + 64 * c;
 #pragma unroll
                 for (int k = 0; k < 4; ++k) qk[nt][k] = qrow + 16 * ((k + c) & 3);
             }
@@ -365,7 +372,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) bq[nt][k] = *reinterpret_cast<const uint4*>(qk[nt][k] + 256 * G);
+                    for (int k = 0; k < 4; ++k) bq[nt][k] = *reinterpret_cast<const uint4*>(smem + qk[nt][k] + 256 * G);
 #pragma unroll
                 for (int p = 0; p < 8; ++p) {
                     const uint32_t msk = 0x01010101u << p;

@@ -132,7 +132,7 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__
     const int g = lane >> 2, c = lane & 3;
 
     QuantRed& red = *reinterpret_cast<QuantRed*>(smem_raw);
-    int8_t* q_s = reinterpret_cast<int8_t*>(smem_raw + ((sizeof(QuantRed) + 127) & ~(size_t)127));  // [kTok][d_in]
+    int8_t* q_s = reinterpret_cast<int8_t*>(smem_raw + ((sizeof(QuantRed) + 127) & ~(size_t)127));  // [min(m, kTok)][d_in]
 
     const uint16_t* xg = reinterpret_cast<const uint16_t*>(e.x);
     const uint8_t* wb = reinterpret_cast<const uint8_t*>(e.w.wb);
@@ -195,10 +195,15 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__
             const uint32_t b11 = *reinterpret_cast<const uint32_t*>(wb + (int64_t)(g + 8) * d_in + col + 16 + 4 * c);
             mma_s8s8(D0, a0, a1, a2, a3, b00, b01);
             mma_s8s8(D1, a0, a1, a2, a3, b10, b11);
-            *reinterpret_cast<uint32_t*>(q_s + g * d_in + col + 4 * c) = a0;
-            *reinterpret_cast<uint32_t*>(q_s + g * d_in + col + 16 + 4 * c) = a2;
-            *reinterpret_cast<uint32_t*>(q_s + (g + 8) * d_in + col + 4 * c) = a1;
-            *reinterpret_cast<uint32_t*>(q_s + (g + 8) * d_in + col + 16 + 4 * c) = a3;
+            // the shared tile holds the round's nt tokens only
+            if (hasA) {
+                *reinterpret_cast<uint32_t*>(q_s + g * d_in + col + 4 * c) = a0;
+                *reinterpret_cast<uint32_t*>(q_s + g * d_in + col + 16 + 4 * c) = a2;
+            }
+            if (hasB) {
+                *reinterpret_cast<uint32_t*>(q_s + (g + 8) * d_in + col + 4 * c) = a1;
+                *reinterpret_cast<uint32_t*>(q_s + (g + 8) * d_in + col + 16 + 4 * c) = a3;
+            }
         }
         // quad reduction of the token sums
         sA += __shfl_xor_sync(0xffffffffu, sA, 1);
