@@ -14,8 +14,8 @@
 // and, for the prefill (m > 16), stores q in the plane-major int8 rows its
 // tensor-core kernel reads, plus s_x, sumq and u.
 //
-// A block owns one linear and up to kTokPerBlock tokens, processed in rounds of
-// 16 tokens (one MMA tile). The 8 warps split the 32-column k-blocks of d_in
+// A block owns one linear and up to kTokPerBlock = 16 tokens (one MMA tile;
+// many small blocks keep enough loads in flight). The 8 warps split the 32-column k-blocks of d_in
 // between them: pass 1 finds each token's amax, pass 2 quantises x straight
 // into MMA A fragments (16 tokens x 32 columns), runs h += q * W_B^T on the
 // warp MMA (m16n8k32, two n-tiles for the 16 LoRA rows) and writes q to a
@@ -40,10 +40,10 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kTok = 16;              // tokens per round
-constexpr int kTokPerBlock = 64;      // rounds per block: 4
+constexpr int kTokPerBlock = 16;      // one round per block: more blocks in flight hide the loads
 
 struct QuantRed {
-    unsigned int amax[kTok];     // fp32 bits of a non-negative max (order-preserving as unsigned)
+    unsigned int amax[kTok];     // fp32 bits of max |x| (order-preserving as unsigned; NaN above Inf)
     int sumq[kWarps][kTok];
     int h[kWarps][kTok][kRank];
     float inv[kTok];
@@ -61,12 +61,14 @@ __device__ __forceinline__ uint32_t quant4(uint2 raw, float inv, bool zero, int&
            ((uint32_t)(q3 & 0xFF) << 24);
 }
 
-__device__ __forceinline__ float absmax8(uint4 v, float m) {
+// running max of |x| over 8 bf16 values, as fp32 bit patterns: for |x| the unsigned order is
+// the numeric order, and a NaN (bits above Inf) wins, so a non-finite row is still seen
+__device__ __forceinline__ uint32_t absmax8_bits(uint4 v, uint32_t m) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        m = fmaxf(m, fabsf(bf16_bits_to_float(w[i] & 0xFFFFu)));
-        m = fmaxf(m, fabsf(bf16_bits_to_float(w[i] >> 16)));
+        m = max(m, (w[i] << 16) & 0x7FFFFFFFu);
+        m = max(m, w[i] & 0x7FFF0000u);
     }
     return m;
 }
@@ -146,19 +148,17 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__
     for (int t0 = tb0; t0 < tb1; t0 += kTok) {
         const int nt = min(kTok, tb1 - t0);
 
-        // ---- pass 1: amax over (token, 16-column piece) items spread over all threads
-        if (tid < kTok) red.amax[tid] = 0u;
-        __syncthreads();
-        {
-            const int pieces = d_in >> 4;
-#pragma unroll 4
-            for (int it = tid; it < nt * pieces; it += kThreads) {
-                const int tk = it / pieces, pc = it - tk * pieces;
-                const uint4* p = reinterpret_cast<const uint4*>(xg + (int64_t)(t0 + tk) * d_in + 16 * pc);
-                const float am = absmax8(p[1], absmax8(p[0], 0.0f));
-                atomicMax(&red.amax[tk], __float_as_uint(am));
-            }
+        // ---- pass 1: amax of each token's row, one warp per token, lanes across the row
+        for (int tk = warp; tk < nt; tk += kWarps) {
+            const uint4* p = reinterpret_cast<const uint4*>(xg + (int64_t)(t0 + tk) * d_in);
+            uint32_t am = 0u;
+#pragma unroll 8
+            for (int i = lane; i < (d_in >> 3); i += 32) am = absmax8_bits(p[i], am);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) am = max(am, __shfl_xor_sync(0xffffffffu, am, o));
+            if (lane == 0) red.amax[tk] = am;
         }
+        if (tid >= nt && tid < kTok) red.amax[tid] = 0u;    // tokens past the round: q = 0
         __syncthreads();
         if (tid < kTok) {
             const float am = __uint_as_float(red.amax[tid]);
@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__
         const uint16_t* xB = xg + (int64_t)(t0 + g + 8) * d_in + 4 * c;
         int D0[4] = {0, 0, 0, 0}, D1[4] = {0, 0, 0, 0};
         int sA = 0, sB = 0;
-#pragma unroll 2
+#pragma unroll 4
         for (int kb = kb_lo + warp; kb < kb_hi; kb += kWarps) {
             const int col = 32 * kb;
             const uint2 zero2 = make_uint2(0u, 0u);
@@ -240,10 +240,14 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__
                 int* mine = qa.part + ((int64_t)lin * qa.splits + split) * kTok * kPartInts + tk * kPartInts;
                 mine[k] = h;
                 if (k == 0) mine[16] = sq;
-                __threadfence();
+                // the block's partials are ordered before its ticket by the barrier and one
+                // device-scope fence (cumulative over what the barrier made visible to thread 0)
                 __syncthreads();
                 __shared__ unsigned int ticket;
-                if (tid == 0) ticket = atomicAdd(qa.tickets + lin, 1u);
+                if (tid == 0) {
+                    __threadfence();
+                    ticket = atomicAdd(qa.tickets + lin, 1u);
+                }
                 __syncthreads();
                 final_block = ticket == (unsigned int)(qa.splits - 1);
                 if (final_block) {
