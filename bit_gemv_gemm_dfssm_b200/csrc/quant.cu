@@ -40,6 +40,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kTok = 16;              // tokens per round
+constexpr int kQsPad = 16;            // bytes of padding per shared q row
 constexpr int kTokPerBlock = 16;      // one round per block: more blocks in flight hide the loads
 
 struct QuantRed {
@@ -134,7 +135,9 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__
     const int g = lane >> 2, c = lane & 3;
 
     QuantRed& red = *reinterpret_cast<QuantRed*>(smem_raw);
-    int8_t* q_s = reinterpret_cast<int8_t*>(smem_raw + ((sizeof(QuantRed) + 127) & ~(size_t)127));  // [min(m, kTok)][d_in]
+    // [kTok][qs_row]: rows padded by 16 bytes so the 8 token rows of an MMA fragment hit 8 bank groups
+    const int qs_row = d_in + kQsPad;
+    int8_t* q_s = reinterpret_cast<int8_t*>(smem_raw + ((sizeof(QuantRed) + 127) & ~(size_t)127));
 
     const uint16_t* xg = reinterpret_cast<const uint16_t*>(e.x);
     const uint8_t* wb = reinterpret_cast<const uint8_t*>(e.w.wb);
@@ -197,12 +200,12 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__
             mma_s8s8(D1, a0, a1, a2, a3, b10, b11);
             // the shared tile holds the round's nt tokens only
             if (hasA) {
-                *reinterpret_cast<uint32_t*>(q_s + g * d_in + col + 4 * c) = a0;
-                *reinterpret_cast<uint32_t*>(q_s + g * d_in + col + 16 + 4 * c) = a2;
+                *reinterpret_cast<uint32_t*>(q_s + g * qs_row + col + 4 * c) = a0;
+                *reinterpret_cast<uint32_t*>(q_s + g * qs_row + col + 16 + 4 * c) = a2;
             }
             if (hasB) {
-                *reinterpret_cast<uint32_t*>(q_s + (g + 8) * d_in + col + 4 * c) = a1;
-                *reinterpret_cast<uint32_t*>(q_s + (g + 8) * d_in + col + 16 + 4 * c) = a3;
+                *reinterpret_cast<uint32_t*>(q_s + (g + 8) * qs_row + col + 4 * c) = a1;
+                *reinterpret_cast<uint32_t*>(q_s + (g + 8) * qs_row + col + 16 + 4 * c) = a3;
             }
         }
         // quad reduction of the token sums
@@ -284,7 +287,7 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__
         for (int i = tid; i < nt * npc; i += kThreads) {
             const int tk = i / npc, pc = pc_lo + (i - tk * npc);
             const int sg = pc >> 1, hc = pc & 1, t = t0 + tk;
-            const uint32_t* src = reinterpret_cast<const uint32_t*>(q_s + tk * d_in + 128 * pc);
+            const uint32_t* src = reinterpret_cast<const uint32_t*>(q_s + tk * qs_row + 128 * pc);
             if (rows) {
                 uint32_t P[8][4];
 #pragma unroll
@@ -325,7 +328,7 @@ cudaError_t launch_quant(const LaunchCtx& c) {
         splits = max(1, min(splits, min(kMaxSplits, min_pc / 2)));
     }
     dim3 grid(splits > 1 ? splits : (c.m + kTokPerBlock - 1) / kTokPerBlock, c.n);
-    const size_t smem = ((sizeof(QuantRed) + 127) & ~(size_t)127) + (size_t)kTok * c.max_d_in;
+    const size_t smem = ((sizeof(QuantRed) + 127) & ~(size_t)127) + (size_t)kTok * (c.max_d_in + kQsPad);
     QuantArgs qa{c.entries, c.single, c.desc, c.m, splits, c.q_ws, c.st_ws, c.part, c.tickets, c.err};
     quant_kernel<<<grid, kThreads, smem, c.stream>>>(qa);
     return cudaGetLastError();
