@@ -84,6 +84,23 @@ __device__ __forceinline__ float lora_dot(const WaRow& wa, const float* __restri
     return __fadd_rn(acc.x, acc.y);
 }
 
+// two int8 (low byte = lower k) -> two bf16 (exact: |v| <= 128), low half = lower k
+__device__ __forceinline__ uint32_t int8_pair_to_bf16x2(uint32_t w) {
+    const uint32_t b0 = __float_as_uint(small_int_to_float((int)(int8_t)(w & 0xFFu))) >> 16;
+    const uint32_t b1 = __float_as_uint(small_int_to_float((int)(int8_t)((w >> 8) & 0xFFu))) & 0xFFFF0000u;
+    return b0 | b1;
+}
+
+// (a, b) as bf16 pairs hi = bf16(x) and lo = bf16(x - hi), low half = a: hi + lo is x to
+// within 2^-18 |x| (x - hi is exact in fp32)
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    const float ha = __uint_as_float(hi << 16), hb = __uint_as_float(hi & 0xFFFF0000u);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(__fsub_rn(a, ha), __fsub_rn(b, hb));
+    lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
 __device__ __forceinline__ float dequant(float sx, float alpha, float sa, int acc, float dot) {
     return __fmul_rn(sx, __fmaf_rn(alpha, small_int_to_float(acc), __fmul_rn(sa, dot)));
 }

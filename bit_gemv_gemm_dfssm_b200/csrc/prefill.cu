@@ -22,11 +22,15 @@
 //               128-byte k-block (four bit planes of that segment, the activation
 //               order of dfssm_internal.cuh), 128 0/1 bytes into the K-major
 //               SWIZZLE_128B layout the MMA reads
-//   warps 8-15  epilogue: tcgen05.ld of its 32 TMEM lanes (= output rows) and
-//               half of the 256 token columns, acc = 2D - sum q, LoRA
-//               up-projection and dequantisation, coalesced stores of y along
-//               the output dimension; the per-token scalars of each 16-token
-//               chunk are staged in a warp-private, double-buffered smem slice
+//   warps 8-15  epilogue over its 32 TMEM lanes (= output rows) and half of the
+//               256 token columns, 16 tokens at a time: tcgen05.ld in the
+//               16x256b shape, which is the register layout of an mma.sync
+//               m16n8 accumulator, acc = 2D - sum q; the LoRA up-projection
+//               W_A u as bf16 warp MMAs in that same layout (W_A exact in bf16,
+//               u split into bf16 hi + lo, fp32 accumulation); dequantisation
+//               and stores. The per-token scalars and the hi/lo u of each
+//               16-token chunk are staged in a warp-private, double-buffered
+//               smem slice
 // 4-stage shared-memory ring (mbarriers), two TMEM accumulator buffers of 256
 // columns so the epilogue of one tile overlaps the main loop of the next.
 // Every mbarrier wait is bounded; a timeout sets the plan's error word.
@@ -49,7 +53,10 @@ constexpr int B_STAGE = BN * BK;   // 32 KB
 constexpr int NUM_THREADS = 16 * 32;
 constexpr int EPI_WARPS = 8;                         // warps 8..15
 constexpr int EPI_THREADS = EPI_WARPS * 32;
-constexpr int STAT_CHUNK = 16 * (int)sizeof(TokStats);  // per-token scalars of 16 tokens (1280 B)
+// staged per 16-token chunk: s_x[16], sum q[16], then u as bf16 pairs (k = 2j, 2j + 1), hi and lo,
+// in rows of 12 words so the B-fragment loads of a warp hit distinct banks
+constexpr int U_ROW = 12;                                 // words per token row (8 used)
+constexpr int STAT_CHUNK = 128 + 2 * 16 * U_ROW * 4;      // 1664 B
 constexpr int STAT_BYTES = EPI_WARPS * 2 * STAT_CHUNK;  // double-buffered, one pair per epilogue warp
 constexpr int SMEM_BYTES = STAGES * (A_STAGE + B_STAGE) + STAT_BYTES + 256 + 1024;
 constexpr uint32_t TMEM_COLS = 512;
@@ -258,52 +265,96 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
         }
     } else if (warp >= 8) {
         // ------------------------------------------------ epilogue
-        // warp 8 + 4h + q handles TMEM lanes 32q.. (output rows) and token columns [128h, 128h + 128)
+        // warp 8 + 4h + q4 handles TMEM lanes 32 q4 .. (output rows) and token columns
+        // [128h, 128h + 128); lane (g, c) = (lane / 4, lane % 4) holds, in mma-fragment order,
+        // rows 32 q4 + 16 rt + g + 8 hh (rt, hh = 0, 1) and tokens 8 tt + 2c + e (tt, e = 0, 1)
         ptx::pdl_wait();
         const int q4 = warp & 3;
         const int half = (warp - 8) >> 2;
-        const int r = q4 * 32 + lane;
+        const int g = lane >> 2, cq = lane & 3;
         uint8_t* stat_buf = sStat + (warp - 8) * 2 * STAT_CHUNK;
         int tcount = 0;
         for (int tile = blockIdx.x; tile < a.n_tiles && !*abort_flag; tile += gridDim.x, ++tcount) {
             const TileCoord tc = tile_coord(a.desc, a.n, n_tt, tile);
             const DevDesc d = a.desc[tc.lin];
             const dfssm_stack_entry& e = entry_at(a.entries, a.single, tc.lin);
-            const int o = tc.row0 + r;
-            const bool valid = o < d.d_out && entry_ptrs_ok(e);
+            const bool lin_ok = entry_ptrs_ok(e);
             // entry fields in registers: the stores below must not force reloads
             void* const y_ptr = e.y;
             int32_t* const dbg_acc = e.dbg.acc;
             const bool y_bf16 = d.y_dtype == DFSSM_BF16;
             const int d_out = d.d_out;
-            float alpha = 0.f, sa = 0.f;
-            WaRow wa = wa_row_from_int4(make_int4(0, 0, 0, 0));
-            if (valid) {
-                alpha = e.w.alpha[o];
-                sa = e.w.sa[o];
-                wa = wa_row_from_int4(*reinterpret_cast<const int4*>(e.w.wa + (int64_t)o * kRank));
-            }
-            // per-token scalars: chunk ch covers tokens tok_base + 16 ch .. + 15 (80 x 16 bytes)
-            const int tok_base = tc.tok0 + half * (BN / 2);
-            const uint4* st_src = reinterpret_cast<const uint4*>(a.st_ws + d.st_off);
-            auto load_chunk = [&](int ch, uint4 (&rg)[3]) {
+            // this thread's 4 rows: alpha, s_A, and the W_A rows as bf16 A fragments
+            int orow[2][2];
+            bool rok[2][2];
+            float alpha[2][2], sa[2][2];
+            uint32_t afr[2][4];
 #pragma unroll
-                for (int u = 0; u < 3; ++u) {
-                    const int idx = lane + 32 * u;                  // uint4 index inside the chunk
-                    const int tok = tok_base + 16 * ch + idx / 5;
-                    rg[u] = (idx < 80 && tok < a.m) ? st_src[(int64_t)(tok_base + 16 * ch) * 5 + idx]
-                                                    : make_uint4(0u, 0u, 0u, 0u);
+            for (int rt = 0; rt < 2; ++rt) {
+                uint32_t wlo[2], whi[2];     // k = 2c, 2c+1 and 2c+8, 2c+9 of rows g, g + 8 (int8 pairs)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int o = tc.row0 + 32 * q4 + 16 * rt + g + 8 * hh;
+                    orow[rt][hh] = o;
+                    rok[rt][hh] = lin_ok && o < d_out;
+                    alpha[rt][hh] = 0.f;
+                    sa[rt][hh] = 0.f;
+                    wlo[hh] = whi[hh] = 0u;
+                    if (rok[rt][hh]) {
+                        alpha[rt][hh] = e.w.alpha[o];
+                        sa[rt][hh] = e.w.sa[o];
+                        const uint16_t* wrow = reinterpret_cast<const uint16_t*>(e.w.wa + (int64_t)o * kRank);
+                        wlo[hh] = wrow[cq];
+                        whi[hh] = wrow[4 + cq];
+                    }
+                }
+                afr[rt][0] = int8_pair_to_bf16x2(wlo[0]);
+                afr[rt][1] = int8_pair_to_bf16x2(wlo[1]);
+                afr[rt][2] = int8_pair_to_bf16x2(whi[0]);
+                afr[rt][3] = int8_pair_to_bf16x2(whi[1]);
+            }
+            // per-token scalars and u of chunk ch (tokens tok_base + 16 ch ..): lane l takes token
+            // l / 2 and u[8 (l % 2) ..]; s_x and sum q from the even lanes
+            const int tok_base = tc.tok0 + half * (BN / 2);
+            const TokStats* st_src = a.st_ws + d.st_off;
+            const int tl = lane >> 1, kh = lane & 1;
+            struct Staged {
+                float4 u0, u1;
+                float sx;
+                int sumq;
+            };
+            auto load_chunk = [&](int ch, Staged& sg) {
+                const int tok = tok_base + 16 * ch + tl;
+                sg.u0 = sg.u1 = make_float4(0.f, 0.f, 0.f, 0.f);
+                sg.sx = 0.f;
+                sg.sumq = 0;
+                if (tok < a.m) {
+                    const TokStats* st = st_src + tok;
+                    sg.u0 = *reinterpret_cast<const float4*>(st->u + 8 * kh);
+                    sg.u1 = *reinterpret_cast<const float4*>(st->u + 8 * kh + 4);
+                    sg.sx = st->sx;
+                    sg.sumq = st->sumq;
                 }
             };
-            auto store_chunk = [&](int buf_i, const uint4 (&rg)[3]) {
-                uint4* dst = reinterpret_cast<uint4*>(stat_buf + buf_i * STAT_CHUNK);
-#pragma unroll
-                for (int u = 0; u < 3; ++u)
-                    if (lane + 32 * u < 80) dst[lane + 32 * u] = rg[u];
+            auto store_chunk = [&](int buf_i, const Staged& sg) {
+                uint8_t* base = stat_buf + buf_i * STAT_CHUNK;
+                uint32_t h[4], l[4];
+                split_bf16x2(sg.u0.x, sg.u0.y, h[0], l[0]);
+                split_bf16x2(sg.u0.z, sg.u0.w, h[1], l[1]);
+                split_bf16x2(sg.u1.x, sg.u1.y, h[2], l[2]);
+                split_bf16x2(sg.u1.z, sg.u1.w, h[3], l[3]);
+                uint32_t* uhi = reinterpret_cast<uint32_t*>(base + 128);
+                uint32_t* ulo = uhi + 16 * U_ROW;
+                *reinterpret_cast<uint4*>(uhi + tl * U_ROW + 4 * kh) = make_uint4(h[0], h[1], h[2], h[3]);
+                *reinterpret_cast<uint4*>(ulo + tl * U_ROW + 4 * kh) = make_uint4(l[0], l[1], l[2], l[3]);
+                if (kh == 0) {
+                    reinterpret_cast<float*>(base)[tl] = sg.sx;
+                    reinterpret_cast<int*>(base + 64)[tl] = sg.sumq;
+                }
             };
-            uint4 rg[3];
-            load_chunk(0, rg);
-            store_chunk(0, rg);
+            Staged sg;
+            load_chunk(0, sg);
+            store_chunk(0, sg);
 
             const int buf = tcount & 1;
             const uint32_t acc_ph = (uint32_t)(tcount >> 1) & 1u;
@@ -316,47 +367,64 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
                 break;
             }
             ptx::tc_fence_after();
-            const uint32_t taddr = tmem_base + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(buf * BN + half * (BN / 2));
+            const uint32_t tcol = tmem_base + (uint32_t)(buf * BN + half * (BN / 2));
             constexpr int NCH = BN / 2 / 16;
             for (int ch = 0; ch < NCH; ++ch) {
                 __syncwarp();
-                const bool more = ch + 1 < NCH && tok_base + 16 * (ch + 1) < a.m;
-                if (more) load_chunk(ch + 1, rg);
-                uint32_t v[16];
-                ptx::tmem_ld_32x32b_x16(taddr + (uint32_t)(16 * ch), v);
-                ptx::tmem_ld_wait();
-                const TokStats* stc = reinterpret_cast<const TokStats*>(stat_buf + (ch & 1) * STAT_CHUNK);
                 const int t0c = tok_base + 16 * ch;
-                if (t0c < a.m && valid) {
-                    const int nj = min(16, a.m - t0c);
-                    // element (t0c + j, o) of y / acc: base + j * d_out (32-bit offsets inside a chunk)
-                    const int64_t base_idx = (int64_t)t0c * d_out + o;
-                    if (y_bf16) {
-                        uint16_t* yb = reinterpret_cast<uint16_t*>(y_ptr) + base_idx;
-                        int32_t* ab = dbg_acc ? dbg_acc + base_idx : nullptr;
+                const bool more = ch + 1 < NCH && t0c + 16 < a.m;
+                if (more) load_chunk(ch + 1, sg);
+                uint32_t v[2][8];
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            if (j >= nj) break;
-                            const TokStats& st = stc[j];
-                            const int acc = 2 * (int)v[j] - st.sumq;
-                            yb[j * d_out] = f32_to_bf16_bits(dequant(st.sx, alpha, sa, acc, lora_dot(wa, st.u)));
-                            if (ab) ab[j * d_out] = acc;
+                for (int rt = 0; rt < 2; ++rt)
+                    ptx::tmem_ld_16x256b_x2(tcol + ((uint32_t)(32 * q4 + 16 * rt) << 16) + (uint32_t)(16 * ch), v[rt]);
+                ptx::tmem_ld_wait();
+                if (t0c < a.m) {
+                    const uint8_t* base = stat_buf + (ch & 1) * STAT_CHUNK;
+                    const uint32_t* uhi = reinterpret_cast<const uint32_t*>(base + 128);
+                    const uint32_t* ulo = uhi + 16 * U_ROW;
+                    // W_A u for the 32 rows x 16 tokens of the chunk: hi then lo, fp32 accumulation
+                    float lora[2][2][4];
+#pragma unroll
+                    for (int tt = 0; tt < 2; ++tt) {
+                        const int tk = 8 * tt + g;
+                        const uint32_t bh0 = uhi[tk * U_ROW + cq], bh1 = uhi[tk * U_ROW + 4 + cq];
+                        const uint32_t bl0 = ulo[tk * U_ROW + cq], bl1 = ulo[tk * U_ROW + 4 + cq];
+#pragma unroll
+                        for (int rt = 0; rt < 2; ++rt) {
+                            float* dd = lora[rt][tt];
+                            dd[0] = dd[1] = dd[2] = dd[3] = 0.f;
+                            ptx::mma_bf16_16816(lora[rt][tt], afr[rt][0], afr[rt][1], afr[rt][2], afr[rt][3], bh0, bh1);
+                            ptx::mma_bf16_16816(lora[rt][tt], afr[rt][0], afr[rt][1], afr[rt][2], afr[rt][3], bl0, bl1);
                         }
-                    } else {
-                        float* yf = reinterpret_cast<float*>(y_ptr) + base_idx;
-                        int32_t* ab = dbg_acc ? dbg_acc + base_idx : nullptr;
+                    }
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            if (j >= nj) break;
-                            const TokStats& st = stc[j];
-                            const int acc = 2 * (int)v[j] - st.sumq;
-                            yf[j * d_out] = dequant(st.sx, alpha, sa, acc, lora_dot(wa, st.u));
-                            if (ab) ab[j * d_out] = acc;
+                    for (int tt = 0; tt < 2; ++tt) {
+#pragma unroll
+                        for (int ee = 0; ee < 2; ++ee) {
+                            const int tj = 8 * tt + 2 * cq + ee;          // token within the chunk
+                            const int t = t0c + tj;
+                            if (t >= a.m) continue;
+                            const float sxt = reinterpret_cast<const float*>(base)[tj];
+                            const int sqt = reinterpret_cast<const int*>(base + 64)[tj];
+#pragma unroll
+                            for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+                                for (int hh = 0; hh < 2; ++hh) {
+                                    if (!rok[rt][hh]) continue;
+                                    const int acc = 2 * (int)v[rt][4 * tt + 2 * hh + ee] - sqt;
+                                    const float y = __fmul_rn(sxt, __fmaf_rn(alpha[rt][hh], small_int_to_float(acc),
+                                                                            __fmul_rn(sa[rt][hh], lora[rt][tt][2 * hh + ee])));
+                                    const int64_t idx = (int64_t)t * d_out + orow[rt][hh];
+                                    if (y_bf16) reinterpret_cast<uint16_t*>(y_ptr)[idx] = f32_to_bf16_bits(y);
+                                    else reinterpret_cast<float*>(y_ptr)[idx] = y;
+                                    if (dbg_acc) dbg_acc[idx] = acc;
+                                }
                         }
                     }
                 }
                 __syncwarp();
-                if (more) store_chunk((ch + 1) & 1, rg);
+                if (more) store_chunk((ch + 1) & 1, sg);
             }
             ptx::tc_fence_before();
             ptx::mbar_arrive(&acc_empty[buf]);

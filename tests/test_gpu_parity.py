@@ -13,7 +13,7 @@ import torch
 import bit_gemv_gemm_dfssm_b200 as dfssm
 import dfssm_synth as synth
 import oracle
-from gpu_util import Linear, check_linear_full, check_linear_sampled, dev, entries_device
+from gpu_util import Linear, check_linear_full, check_linear_sampled, check_y, dev, entries_device, term_bound
 
 pytestmark = pytest.mark.gpu
 
@@ -81,8 +81,10 @@ def test_max_m_larger_than_m():
         check_linear_full(lin)
 
 
-def test_decode_and_prefill_agree_bit_for_bit():
-    # the first 16 tokens: m = 16 runs the decode kernel, m = 17 the tcgen05 kernel
+def test_decode_and_prefill_agree():
+    # the first 16 tokens: m = 16 runs the decode kernel, m = 17 the tcgen05 kernel. The
+    # integer sums agree bit for bit; y is computed in different fp32 orders (the prefill runs
+    # the LoRA up-projection on bf16 hi/lo warp MMAs), so each is held to the oracle's bound.
     d_in, d_out = 2048, 640
     x = synth.activations(SEED, 9, 5, 17, d_in)
     a = Linear(SEED, 9, 5, d_in, d_out, 16, F32, x=np.ascontiguousarray(x[:16]))
@@ -90,7 +92,10 @@ def test_decode_and_prefill_agree_bit_for_bit():
     run_one(a)
     run_one(b)
     np.testing.assert_array_equal(a.dacc.cpu().numpy(), b.dacc.cpu().numpy()[:16])
-    np.testing.assert_array_equal(a.dy.cpu().numpy(), b.dy.cpu().numpy()[:16])
+    ref = oracle.linear(b.x, b.w, 17, d_in, d_out)
+    check_y(b.y_host(), ref["y"], term_bound(ref, b.w), F32)
+    ref16 = oracle.linear(a.x, a.w, 16, d_in, d_out)
+    check_y(a.y_host(), ref16["y"], term_bound(ref16, a.w), F32)
 
 
 def test_zero_and_single_channel_inputs():
