@@ -398,29 +398,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
                             ptx::mma_bf16_16816(lora[rt][tt], afr[rt][0], afr[rt][1], afr[rt][2], afr[rt][3], bl0, bl1);
                         }
                     }
+                    // element (rt, hh, tt, ee): row orow[rt][hh], token t0c + 8 tt + 2 cq + ee; branch-free,
+                    // with the validity of row and token as store predicates
+                    auto elements = [&](auto store_y) {
 #pragma unroll
-                    for (int tt = 0; tt < 2; ++tt) {
+                        for (int tt = 0; tt < 2; ++tt) {
 #pragma unroll
-                        for (int ee = 0; ee < 2; ++ee) {
-                            const int tj = 8 * tt + 2 * cq + ee;          // token within the chunk
-                            const int t = t0c + tj;
-                            if (t >= a.m) continue;
-                            const float sxt = reinterpret_cast<const float*>(base)[tj];
-                            const int sqt = reinterpret_cast<const int*>(base + 64)[tj];
+                            for (int ee = 0; ee < 2; ++ee) {
+                                const int tj = 8 * tt + 2 * cq + ee;      // token within the chunk
+                                const int t = t0c + tj;
+                                const bool tok_ok = t < a.m;
+                                const float sxt = reinterpret_cast<const float*>(base)[tj];
+                                const int sqt = reinterpret_cast<const int*>(base + 64)[tj];
 #pragma unroll
-                            for (int rt = 0; rt < 2; ++rt)
+                                for (int rt = 0; rt < 2; ++rt)
 #pragma unroll
-                                for (int hh = 0; hh < 2; ++hh) {
-                                    if (!rok[rt][hh]) continue;
-                                    const int acc = 2 * (int)v[rt][4 * tt + 2 * hh + ee] - sqt;
-                                    const float y = __fmul_rn(sxt, __fmaf_rn(alpha[rt][hh], small_int_to_float(acc),
-                                                                            __fmul_rn(sa[rt][hh], lora[rt][tt][2 * hh + ee])));
-                                    const int64_t idx = (int64_t)t * d_out + orow[rt][hh];
-                                    if (y_bf16) reinterpret_cast<uint16_t*>(y_ptr)[idx] = f32_to_bf16_bits(y);
-                                    else reinterpret_cast<float*>(y_ptr)[idx] = y;
-                                    if (dbg_acc) dbg_acc[idx] = acc;
-                                }
+                                    for (int hh = 0; hh < 2; ++hh) {
+                                        const int acc = 2 * (int)v[rt][4 * tt + 2 * hh + ee] - sqt;
+                                        const float y = __fmul_rn(
+                                            sxt, __fmaf_rn(alpha[rt][hh], small_int_to_float(acc),
+                                                           __fmul_rn(sa[rt][hh], lora[rt][tt][2 * hh + ee])));
+                                        const bool ok = tok_ok && rok[rt][hh];
+                                        const int64_t idx = (int64_t)t * d_out + orow[rt][hh];
+                                        store_y(ok, idx, y);
+                                        if (ok && dbg_acc != nullptr) dbg_acc[idx] = acc;
+                                    }
+                            }
                         }
+                    };
+                    if (y_bf16) {
+                        uint16_t* yb = reinterpret_cast<uint16_t*>(y_ptr);
+                        elements([&](bool ok, int64_t idx, float y) {
+                            const uint16_t b = f32_to_bf16_bits(y);
+                            if (ok) yb[idx] = b;
+                        });
+                    } else {
+                        float* yf = reinterpret_cast<float*>(y_ptr);
+                        elements([&](bool ok, int64_t idx, float y) {
+                            if (ok) yf[idx] = y;
+                        });
                     }
                 }
                 __syncwarp();
