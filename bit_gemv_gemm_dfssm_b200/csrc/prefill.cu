@@ -36,6 +36,8 @@
 // Every mbarrier wait is bounded; a timeout sets the plan's error word.
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "dfssm_internal.cuh"
 #include "epilogue.cuh"
 #include "ptx.cuh"
@@ -400,7 +402,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
                     }
                     // element (rt, hh, tt, ee): row orow[rt][hh], token t0c + 8 tt + 2 cq + ee; branch-free,
                     // with the validity of row and token as store predicates
-                    auto elements = [&](auto store_y) {
+                    auto elements = [&](auto store_y, auto dbg_tag) {
+                        constexpr bool kDbg = decltype(dbg_tag)::value;
 #pragma unroll
                         for (int tt = 0; tt < 2; ++tt) {
 #pragma unroll
@@ -421,22 +424,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
                                         const bool ok = tok_ok && rok[rt][hh];
                                         const int64_t idx = (int64_t)t * d_out + orow[rt][hh];
                                         store_y(ok, idx, y);
-                                        if (ok && dbg_acc != nullptr) dbg_acc[idx] = acc;
+                                        if constexpr (kDbg) {
+                                            if (ok) dbg_acc[idx] = acc;
+                                        }
                                     }
                             }
                         }
                     };
-                    if (y_bf16) {
-                        uint16_t* yb = reinterpret_cast<uint16_t*>(y_ptr);
-                        elements([&](bool ok, int64_t idx, float y) {
-                            const uint16_t b = f32_to_bf16_bits(y);
-                            if (ok) yb[idx] = b;
-                        });
+                    // the output type and the debug export are fixed per call: one code path each
+                    uint16_t* yb = reinterpret_cast<uint16_t*>(y_ptr);
+                    float* yf = reinterpret_cast<float*>(y_ptr);
+                    auto st_bf16 = [&](bool ok, int64_t idx, float y) {
+                        const uint16_t b = f32_to_bf16_bits(y);
+                        if (ok) yb[idx] = b;
+                    };
+                    auto st_f32 = [&](bool ok, int64_t idx, float y) {
+                        if (ok) yf[idx] = y;
+                    };
+                    using kNo = std::integral_constant<bool, false>;
+                    using kYes = std::integral_constant<bool, true>;
+                    if (dbg_acc == nullptr) {
+                        if (y_bf16) elements(st_bf16, kNo{}); else elements(st_f32, kNo{});
                     } else {
-                        float* yf = reinterpret_cast<float*>(y_ptr);
-                        elements([&](bool ok, int64_t idx, float y) {
-                            if (ok) yf[idx] = y;
-                        });
+                        if (y_bf16) elements(st_bf16, kYes{}); else elements(st_f32, kYes{});
                     }
                 }
                 __syncwarp();
