@@ -21,6 +21,7 @@ using namespace dfssm;
 
 namespace dfssm {
 cudaError_t set_quant_attr(int optin);
+cudaError_t set_quant_rows_attr(int optin);
 cudaError_t set_decode_attr(int optin);
 cudaError_t set_prefill_attr(int optin);
 int prefill_box_tokens();
@@ -29,6 +30,7 @@ int prefill_box_bytes();
 // Allow each kernel the opt-in shared memory size (a permission, not a reservation).
 static cudaError_t set_kernel_attributes(int optin) {
     cudaError_t e = set_quant_attr(optin);
+    if (e == cudaSuccess) e = set_quant_rows_attr(optin);
     if (e == cudaSuccess) e = set_decode_attr(optin);
     if (e == cudaSuccess) e = set_prefill_attr(optin);
     return e;

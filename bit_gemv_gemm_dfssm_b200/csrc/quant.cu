@@ -317,7 +317,10 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__
 
 }  // namespace
 
+cudaError_t launch_quant_rows(const LaunchCtx& c);
+
 cudaError_t launch_quant(const LaunchCtx& c) {
+    if (c.m > kDecodeMaxTokens) return launch_quant_rows(c);
     int splits = 1;
     if (c.m <= kTok) {
         // enough blocks to cover the SMs twice, at least two 128-column pieces (8 k-blocks,
