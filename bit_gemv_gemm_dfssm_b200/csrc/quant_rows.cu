@@ -6,32 +6,36 @@
 // per-row scales; §2.C: int8 activations for the int8 x int8 -> int32
 // scaffold matmul), arranged for throughput over a large activation matrix.
 //
-// Persistent kernel, one block per SM: 16 consumer warps and one producer warp.
-// Work items are T tokens of one linear, T = min(16, 16384 / d_in), so an
-// item is at most 32 KB of bf16; the items of a linear are numbered in token
-// order and the linears follow each other.
-//   producer   per item: looks up the linear, writes the item's descriptor
-//              (shape, offsets, pointers, s_B) to a shared ring, and fetches
-//              the item's rows (one contiguous range of x) with a single bulk
-//              copy (TMA engine, no tensor map, no multicast) into one of three
-//              shared x tiles. x is read from HBM once; two items stream in
-//              while one is processed.
-//   consumers  per item, with three barriers among the 16 warps:
-//     1. amax per token from the shared tile: a 16-bit SIMD max over the |x|
-//        bit patterns (the unsigned order of |bf16| bits is the numeric
-//        order, NaN above Inf, so a non-finite row is still seen);
-//     2. each thread quantises one 32-column group of one token.
-//        rint(x * inv) is taken by adding 1.5 * 2^23 in round-to-nearest-even,
-//        exact here because |x * inv| <= 127 * (1 + 2^-23); the low byte of
-//        the sum is q. The group is written twice: in natural order to a
-//        shared q tile, and in the plane-major order of the prefill's
-//        activation rows straight to global memory (eight 4-byte plane words;
-//        eight lanes fill one 32-byte sector);
-//     3. h = q W_B^T and sum q on the warp MMA (m16n8k32, s8 x s8 -> s32)
-//        from the shared q tile, a third n-tile of ones giving sum q; warp w
-//        takes k-blocks w, w + 16, ... and keeps their W_B fragments in
-//        registers for as long as the linear stays the same;
-//     4. the 16 partials are added in shared memory; u = s_B h, s_x, sum q.
+// Persistent kernel, one block of 16 warps per SM. Work items are T tokens of
+// one linear, T = min(16, 32768 / d_in), so an item is at most 64 KB of bf16;
+// the items of a linear are numbered in token order, the linears follow each
+// other, and each block takes one contiguous range of items (so it meets few
+// linears and keeps their W_B fragments in registers). Per item:
+//   issue (warp 0, two items ahead, as soon as the tile is free): the item's
+//     descriptor (shape, offsets, pointers, s_B; looked up in global memory
+//     only when the linear changes) goes to a shared ring, and its rows (one
+//     contiguous range of x) come in by a single bulk copy (TMA engine, no
+//     tensor map, no multicast) into one of two shared x tiles: x is read from
+//     HBM once, and the next item streams in while one is processed;
+//   1. each thread loads its (up to two) 32-column groups of the tile into
+//      registers and takes their max |x| as a 16-bit SIMD max over the bit
+//      patterns (the unsigned order of |bf16| bits is the numeric order, NaN
+//      above Inf, so a non-finite row is still seen); per token the maximum
+//      is gathered by shuffles and a shared atomic max;
+//   2. rint(x * inv) by adding 1.5 * 2^23 in round-to-nearest-even, exact here
+//      because |x * inv| <= 127 * (1 + 2^-23); the low byte of the sum is q.
+//      Each group's eight plane words (the plane-major order of the prefill's
+//      activation rows) go to global memory (eight lanes fill one 32-byte
+//      sector) and to a shared q tile in the same order;
+//   3. h^T = W_B q^T on the warp MMA (m16n8k32, s8 x s8 -> s32): the 16 LoRA
+//      rows are M and 8 tokens N, so T <= 8 takes one MMA per 32 bytes of K
+//      and T = 16 two; the K order is the plane-major one of the shared tile,
+//      so the W_B fragments are gathered in that order. sum q comes from dp4a
+//      on the same q fragments. Warp w takes k-blocks w, w + 16, ...;
+//   4. the 16 warp partials are added in shared memory; u = s_B h, s_x, sum q.
+// Three barriers per item. No integer division per item: token and group of a
+// thread come from an fp32 reciprocal of d_in / 32, exact at these sizes (the
+// quotient's fractional part stays at least 1/512 away from an integer).
 #include "dfssm_internal.cuh"
 #include "epilogue.cuh"
 #include "ptx.cuh"
@@ -40,22 +44,29 @@ namespace dfssm {
 
 namespace {
 
-constexpr int kConsumers = 512;
+constexpr int kConsumers = 512;             // all threads of the block
 constexpr int kCWarps = kConsumers / 32;     // 16
-constexpr int kThreads = kConsumers + 32;    // + the producer warp
-constexpr int kItemElems = 16384;            // bf16 values of one item at most (32 KB)
-constexpr int kMaxT = 16;                    // tokens per item at most (the MMA's M)
-constexpr int kBufs = 3;                     // x tiles
-constexpr int kInfos = kBufs + 1;            // item descriptors (a descriptor outlives its tile)
-constexpr int kQsPad = 16;                   // bytes of padding per shared q row (ldmatrix rows on distinct banks)
+constexpr int kThreads = kConsumers;
+constexpr int kItemElems = 32768;            // bf16 values of one item at most (64 KB)
+constexpr int kGroupsPerThread = kItemElems / 32 / kConsumers;   // 2
+constexpr int kMaxT = 16;                    // tokens per item at most (two MMA n-tiles)
+constexpr int kBufs = 2;                     // x tiles
+constexpr int kInfos = kBufs + 1;            // item descriptors (a descriptor outlives its tile by one item)
+// shared q rows: plane-major like the global rows, but segments 288 bytes apart (the plane words of
+// the 4 segments a warp writes land on distinct banks) and rows 16 bytes longer than that (the 8
+// token rows an ldmatrix reads land on distinct banks)
+constexpr int kQsSegStride = kSegCols + 32;
+constexpr int kQsRowPad = 16;
 constexpr int kHCols = kRank + 1;            // h[0..15] and sum q
-constexpr int kQsBytes = kItemElems + kMaxT * kQsPad;
+// largest T * (segments * 288 + 16) over d_in (T * d_in <= 32768)
+constexpr int kQsBytes = 41984;
 constexpr int kWbRegKb = 8;                  // k-blocks per warp whose W_B fragments stay in registers (d_in <= 4096)
-constexpr uint32_t kBarConsumers = 1;        // named barrier of the 16 consumer warps
+constexpr uint32_t kBarConsumers = 1;        // named barrier of the 16 warps
 
 struct ItemInfo {
     int lin, t0, nt, d_in;
-    int qrow, usable, pad0, pad1;
+    int T, qrow, usable, pad0;
+    float rgpt, pad1;                        // 1 / (d_in / 32)
     int64_t q_off, st_off;
     const int8_t* wb;
     int8_t* dbg_q;
@@ -64,15 +75,22 @@ struct ItemInfo {
     float sb[kRank];
 };
 
+// Position in the item sequence and the linear of the last descriptor written.
+struct Cursor {
+    int lin, begin, count, tpi, info_lin;
+    const uint16_t* x;
+    int d_in, usable;
+};
+
 struct RowsShared {
     uint16_t x[kBufs][kItemElems];           // bf16 tiles, bulk-copy destinations
-    int8_t q[kQsBytes];                      // natural-order q of the item, rows of d_in + 16 bytes
+    int8_t q[kQsBytes];                      // q of the item, plane-major rows (see kQsSegStride)
     int h[kCWarps][kMaxT][kHCols];           // per-warp partial h and sum q
     ItemInfo info[kInfos];
-    uint32_t amax[kCWarps];                  // per-warp partial max |x| (fp32 bit pattern)
+    uint32_t amax_tok[kMaxT];                // max |x| per token (fp32 bit pattern), zero between items
     float sx[kMaxT];
-    uint64_t full[kBufs];                    // producer -> consumers: tile and descriptor ready
-    uint64_t empty[kBufs];                   // consumers -> producer: tile read
+    Cursor cur;
+    uint64_t full[kBufs];                    // tile and descriptor ready
 };
 
 __host__ __device__ inline int tokens_per_item(int d_in) {
@@ -116,25 +134,18 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
     return d;
 }
 
-// four bf16 (two words) -> four int8 (one word, little-endian), q = rint(x * inv). The
-// rounding add is the scalar __fadd_rn, which is never merged with the product into an FMA
-// (a fused x * inv + 1.5 * 2^23 would skip the product's own rounding and can move a tie).
-__device__ __forceinline__ uint32_t quant_pack4(uint32_t wa, uint32_t wb, float inv) {
-    constexpr float kRound = 12582912.0f;   // 1.5 * 2^23: ulp 1, low byte q
-    const float2 iv = make_float2(inv, inv);
-    const float2 pa = fmul2(make_float2(bf16_lo(wa), bf16_hi(wa)), iv);
-    const float2 pb = fmul2(make_float2(bf16_lo(wb), bf16_hi(wb)), iv);
-    const uint32_t y0 = __float_as_uint(__fadd_rn(pa.x, kRound)), y1 = __float_as_uint(__fadd_rn(pa.y, kRound));
-    const uint32_t y2 = __float_as_uint(__fadd_rn(pb.x, kRound)), y3 = __float_as_uint(__fadd_rn(pb.y, kRound));
-    return __byte_perm(__byte_perm(y0, y1, 0x0040u), __byte_perm(y2, y3, 0x4000u), 0x7610u);
+// two bf16 (one word) -> y = rint(x * inv) + 1.5 * 2^23 as fp32 bits, whose low byte is q. The
+// rounding add is the scalar __fadd_rn, which is never merged with the product into an FMA (a fused
+// x * inv + 1.5 * 2^23 would skip the product's own rounding and can move a tie).
+__device__ __forceinline__ void quant_pair(uint32_t w, float inv, uint32_t& y_lo, uint32_t& y_hi) {
+    constexpr float kRound = 12582912.0f;   // 1.5 * 2^23: ulp 1
+    const float2 p = fmul2(make_float2(bf16_lo(w), bf16_hi(w)), make_float2(inv, inv));
+    y_lo = __float_as_uint(__fadd_rn(p.x, kRound));
+    y_hi = __float_as_uint(__fadd_rn(p.y, kRound));
 }
 
-// word r of the result = byte r of a, b, c, d (4x4 byte transpose)
-__device__ __forceinline__ uint4 transpose4x4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    const uint32_t t0 = __byte_perm(a, b, 0x5140), t1 = __byte_perm(a, b, 0x7362);
-    const uint32_t t2 = __byte_perm(c, d, 0x5140), t3 = __byte_perm(c, d, 0x7362);
-    return make_uint4(__byte_perm(t0, t2, 0x5410), __byte_perm(t0, t2, 0x7632), __byte_perm(t1, t3, 0x5410),
-                      __byte_perm(t1, t3, 0x7632));
+__device__ __forceinline__ uint32_t word_of(const uint4& v, int h) {
+    return h == 0 ? v.x : h == 1 ? v.y : h == 2 ? v.z : v.w;
 }
 
 __device__ __forceinline__ void mma_s8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -146,63 +157,128 @@ __device__ __forceinline__ void mma_s8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// ------------------------------------------------------------------ producer warp
-__device__ void produce(const RowsArgs& a, RowsShared& sh) {
-    const int lane = threadIdx.x & 31;
-    int lin = 0, begin = 0, tpi = tokens_per_item(a.descs[0].d_in);
-    int count = (a.m + tpi - 1) / tpi;
-    for (int kk = 0;; ++kk) {
-        const int item = blockIdx.x + kk * gridDim.x;
-        if (item >= a.total) break;
-        while (item >= begin + count && lin + 1 < a.n) {   // items arrive in increasing order
-            begin += count;
-            ++lin;
-            tpi = tokens_per_item(a.descs[lin].d_in);
-            count = (a.m + tpi - 1) / tpi;
+__device__ __forceinline__ void ldmatrix_x2(uint32_t saddr, uint32_t& r0, uint32_t& r1) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(saddr));
+}
+
+// A fragment (m16n8k32: rows = LoRA rows g, g + 8) of k-block kb in the plane-major K order of
+// the shared q tile: K position 32 p + 4 c' + i of segment s is column 256 s + 32 c' + 8 i + p
+// (p = kb % 8, s = kb / 8); columns past d_in (the absent half of a final half segment) are zero.
+// f[0] = row g, c' = cq; f[1] = row g + 8, c' = cq; f[2] = row g, c' = cq + 4; f[3] = row g + 8, c' = cq + 4.
+__device__ __forceinline__ void wb_fragment(const int8_t* wb, int d_in, int kb, int g, int cq, uint32_t (&f)[4]) {
+    const int s = kb >> 3, p = kb & 7;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int row = g + 8 * (r & 1);
+        const int col0 = 256 * s + 32 * (cq + 4 * (r >> 1)) + p;
+        uint32_t v = 0u;
+        if (col0 < d_in) {
+            const uint8_t* src = reinterpret_cast<const uint8_t*>(wb) + (int64_t)row * d_in + col0;
+            v = (uint32_t)__ldg(src) | ((uint32_t)__ldg(src + 8) << 8) | ((uint32_t)__ldg(src + 16) << 16) |
+                ((uint32_t)__ldg(src + 24) << 24);
         }
-        const int slot = kk % kBufs;
-        bool ok = true;
-        if (lane == 0) ok = ptx::mbar_wait(&sh.empty[slot], ((uint32_t)(kk / kBufs) & 1u) ^ 1u);
-        if (!__shfl_sync(0xffffffffu, ok, 0)) {
-            if (lane == 0) atomicOr(a.err, DFSSM_DEVERR_TIMEOUT);
-            return;
+        f[r] = v;
+    }
+}
+
+// the fragments of k-blocks warp + 16 j, j < kWbRegKb
+__device__ __forceinline__ void load_wb_fragments(const int8_t* wb, int d_in, int warp, int g, int cq,
+                                                  uint32_t (&wbf)[kWbRegKb][4]) {
+    const int nkb = (d_in + kSegCols - 1) / kSegCols * 8;
+#pragma unroll
+    for (int j = 0; j < kWbRegKb; ++j) {
+        const int kb = warp + kCWarps * j;
+        if (kb < nkb) wb_fragment(wb, d_in, kb, g, cq, wbf[j]);
+    }
+}
+
+// (token, group) of group index G: token = G / gpt by the fp32 reciprocal (exact here)
+__device__ __forceinline__ int div_by_recip(int G, float r) { return __float2int_rz(((float)G + 0.5f) * r); }
+
+// this block's contiguous range of items
+__device__ __forceinline__ void item_range(const RowsArgs& a, int& lo, int& hi) {
+    lo = (int)((int64_t)blockIdx.x * a.total / gridDim.x);
+    hi = (int)((int64_t)(blockIdx.x + 1) * a.total / gridDim.x);
+}
+
+// ------------------------------------------------------------------ item issue (warp 0)
+__device__ __forceinline__ void cursor_start(const RowsArgs& a, Cursor& cur) {
+    cur.lin = 0;
+    cur.begin = 0;
+    cur.tpi = tokens_per_item(a.descs[0].d_in);
+    cur.count = (a.m + cur.tpi - 1) / cur.tpi;
+    cur.info_lin = -1;
+    cur.x = nullptr;
+    cur.d_in = 0;
+    cur.usable = 0;
+}
+
+// Warp 0, all lanes: write the descriptor of the block's kk-th item (global index `item`) and
+// start its bulk copy into tile kk % kBufs, which no thread still reads. Items arrive in
+// increasing order; a descriptor repeats its predecessor's linear fields unless the linear changed.
+__device__ void issue_item(const RowsArgs& a, RowsShared& sh, Cursor& cur, int kk, int item, int lane) {
+    if (lane == 0) {
+        while (item >= cur.begin + cur.count && cur.lin + 1 < a.n) {
+            cur.begin += cur.count;
+            ++cur.lin;
+            cur.tpi = tokens_per_item(a.descs[cur.lin].d_in);
+            cur.count = (a.m + cur.tpi - 1) / cur.tpi;
         }
-        const dfssm_stack_entry& e = entry_at(a.entries, a.single, lin);
-        const DevDesc d = a.descs[lin];
-        const bool desc_ok = a.entries == nullptr || e.desc_index == lin;
+    }
+    __syncwarp();
+    ItemInfo& inf = sh.info[kk % kInfos];
+    if (cur.lin != cur.info_lin) {
+        const dfssm_stack_entry& e = entry_at(a.entries, a.single, cur.lin);
+        const DevDesc d = a.descs[cur.lin];
+        const bool desc_ok = a.entries == nullptr || e.desc_index == cur.lin;
         const bool usable = desc_ok && entry_ptrs_ok(e);
-        const int t0 = (item - begin) * tpi;
-        const int nt = min(tpi, a.m - t0);
-        ItemInfo& inf = sh.info[kk % kInfos];
         if (lane < kRank) inf.sb[lane] = usable ? e.w.sb[lane] : 0.0f;
         if (lane == 0) {
-            inf.lin = lin;
-            inf.t0 = t0;
-            inf.nt = nt;
+            inf.lin = cur.lin;
             inf.d_in = d.d_in;
+            inf.T = cur.tpi;
             inf.qrow = d.qrow;
             inf.usable = usable;
+            inf.rgpt = 1.0f / (float)(d.d_in >> 5);
             inf.q_off = d.q_off;
             inf.st_off = d.st_off;
             inf.wb = reinterpret_cast<const int8_t*>(e.w.wb);
             inf.dbg_q = e.dbg.q;
             inf.dbg_h = e.dbg.h;
             inf.dbg_sx = e.dbg.sx;
+            if (!usable) atomicOr(a.err, desc_ok ? DFSSM_DEVERR_ENTRY_PTR : DFSSM_DEVERR_ENTRY_DESC);
         }
         __syncwarp();
         if (lane == 0) {
-            uint64_t* bar = &sh.full[slot];
-            if (usable) {
-                const uint32_t bytes = (uint32_t)nt * (uint32_t)d.d_in * 2u;
-                ptx::mbar_arrive_expect_tx(bar, bytes);   // release: the descriptor above is visible
-                ptx::bulk_g2s(sh.x[slot], reinterpret_cast<const uint16_t*>(e.x) + (int64_t)t0 * d.d_in, bytes,
-                              bar);
-            } else {
-                atomicOr(a.err, desc_ok ? DFSSM_DEVERR_ENTRY_PTR : DFSSM_DEVERR_ENTRY_DESC);
-                ptx::mbar_arrive(bar);                    // nothing to copy: complete the phase
-            }
+            cur.info_lin = cur.lin;
+            cur.x = reinterpret_cast<const uint16_t*>(e.x);
+            cur.d_in = d.d_in;
+            cur.usable = usable;
+        }
+    } else {
+        // the same linear: copy the previous descriptor (still intact: it is rewritten two items later)
+        static_assert(sizeof(ItemInfo) % 4 == 0 && sizeof(ItemInfo) / 4 <= 64, "descriptor copy");
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(&sh.info[(kk + kInfos - 1) % kInfos]);
+        uint32_t* dst = reinterpret_cast<uint32_t*>(&inf);
+        for (int i = lane; i < (int)(sizeof(ItemInfo) / 4); i += 32) dst[i] = src[i];
+    }
+    __syncwarp();
+    if (lane == 0) {
+        const int t0 = (item - cur.begin) * cur.tpi;
+        const int nt = min(cur.tpi, a.m - t0);
+        inf.t0 = t0;
+        inf.nt = nt;
+        const int slot = kk % kBufs;
+        uint64_t* bar = &sh.full[slot];
+        if (cur.usable) {
+            const uint32_t bytes = (uint32_t)nt * (uint32_t)cur.d_in * 2u;
+            ptx::mbar_arrive_expect_tx(bar, bytes);   // release: the descriptor above is visible
+            ptx::bulk_g2s(sh.x[slot], cur.x + (int64_t)t0 * cur.d_in, bytes, bar);
+        } else {
+            ptx::mbar_arrive(bar);                    // nothing to copy: complete the phase
         }
     }
+    __syncwarp();
 }
 
 __global__ void __launch_bounds__(kThreads, 1) quant_rows_kernel(const __grid_constant__ RowsArgs a) {
@@ -211,178 +287,218 @@ __global__ void __launch_bounds__(kThreads, 1) quant_rows_kernel(const __grid_co
     // let the dependent prefill kernel start streaming weights; it waits for this grid before reading q
     ptx::pdl_launch_dependents();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid < kMaxT) sh.amax_tok[tid] = 0u;
     if (tid == 0) {
-        for (int b = 0; b < kBufs; ++b) {
-            ptx::mbar_init(&sh.full[b], 1);
-            ptx::mbar_init(&sh.empty[b], 1);
-        }
+        for (int b = 0; b < kBufs; ++b) ptx::mbar_init(&sh.full[b], 1);
         ptx::fence_mbar_init();
     }
     __syncthreads();
-    if (warp == kCWarps) {
-        produce(a, sh);
-        return;
+    int lo, hi;
+    item_range(a, lo, hi);
+    Cursor& cur = sh.cur;     // warp 0's issue state (shared memory: no registers in the other warps)
+    if (warp == 0) {
+        if (lane == 0) cursor_start(a, cur);
+        __syncwarp();
+        for (int kk = 0; kk < kBufs && lo + kk < hi; ++kk) issue_item(a, sh, cur, kk, lo + kk, lane);
     }
 
     // ------------------------------------------------------------------ consumers
     const int g = lane >> 2, cq = lane & 3;
+    // the 16-byte x loads in a lane-dependent order (chunk kk_j = (j + rot_r) % 4 at load j):
+    // 8 consecutive lanes then read distinct banks
+    const int rot_r = ((lane >> 1) ^ (lane >> 3)) & 3;
+    // byte selector that puts the bytes of loads 0..3 (gathered as t01.b0, t01.b1, t23.b2, t23.b3)
+    // at byte positions kk_0..kk_3 of a plane word
+    const uint32_t plane_sel = (0u << (4 * (rot_r & 3))) | (1u << (4 * ((rot_r + 1) & 3))) |
+                               (6u << (4 * ((rot_r + 2) & 3))) | (7u << (4 * ((rot_r + 3) & 3)));
+    // ldmatrix (q as the B operand): this lane addresses token (lane & 7) + 8 (lane >> 4), bytes 16 ((lane >> 3) & 1)
+    const int lm_tok = (lane & 7) + 8 * (lane >> 4), lm_off = 16 * ((lane >> 3) & 1);
     int wb_lin = -1;                       // linear whose W_B fragments are in wbf
-    uint32_t wbf[kWbRegKb][4];
+    uint32_t wbf[kWbRegKb][4];             // A fragments of this warp's k-blocks (plane-major K order)
 #pragma unroll
     for (int j = 0; j < kWbRegKb; ++j) wbf[j][0] = wbf[j][1] = wbf[j][2] = wbf[j][3] = 0u;
-    for (int kk = 0;; ++kk) {
-        const int item = blockIdx.x + kk * gridDim.x;
-        if (item >= a.total) break;
+    for (int item = lo, kk = 0; item < hi; ++item, ++kk) {
         const int slot = kk % kBufs;
         const bool got = ptx::mbar_wait(&sh.full[slot], (uint32_t)(kk / kBufs) & 1u);
         const ItemInfo& inf = sh.info[kk % kInfos];
         const int usable = got ? inf.usable : 0;
         const int d_in = inf.d_in, nt = inf.nt, t0 = inf.t0;
-        const int T = tokens_per_item(d_in);
-        const int nkb = d_in >> 5;
+        const int gpt = d_in >> 5;                   // 32-column groups per token
+        const int nseg = (d_in + kSegCols - 1) / kSegCols;
+        const int qs_row = nseg * kQsSegStride + kQsRowPad;
         const uint16_t* xt = sh.x[slot];
 
-        // W_B fragments of this warp's k-blocks (b00, b01: rank g; b10, b11: rank g + 8), on a change of linear
         if (usable && inf.lin != wb_lin) {
             wb_lin = inf.lin;
-            const uint8_t* w0 = reinterpret_cast<const uint8_t*>(inf.wb) + (int64_t)g * d_in + 4 * cq;
-            const uint8_t* w1 = w0 + (int64_t)8 * d_in;
-#pragma unroll
-            for (int j = 0; j < kWbRegKb; ++j) {
-                const int col = 32 * (warp + kCWarps * j);
-                if (col < d_in) {
-                    wbf[j][0] = __ldg(reinterpret_cast<const uint32_t*>(w0 + col));
-                    wbf[j][1] = __ldg(reinterpret_cast<const uint32_t*>(w0 + col + 16));
-                    wbf[j][2] = __ldg(reinterpret_cast<const uint32_t*>(w1 + col));
-                    wbf[j][3] = __ldg(reinterpret_cast<const uint32_t*>(w1 + col + 16));
-                }
-            }
+            load_wb_fragments(inf.wb, d_in, warp, g, cq, wbf);
         }
 
-        // ---- 1: partial amax, warp w takes part w % parts of token w / parts
-        const int parts = kCWarps / T;
+        // ---- 1: load this thread's groups G = tid, tid + 512 (token G / gpt, group G % gpt) and
+        //         their partial max |x|; per token the maximum goes to amax_tok
+        uint4 xv[kGroupsPerThread][4];
+        int tkg[kGroupsPerThread], cg[kGroupsPerThread];
         if (usable) {
-            const int tk = warp / parts, part = warp - tk * parts;
-            uint32_t m2 = 0u;
-            if (tk < nt) {
-                const uint4* row = reinterpret_cast<const uint4*>(xt + tk * d_in);
-#pragma unroll 4
-                for (int i = part * 32 + lane; i < (d_in >> 3); i += parts * 32) {
-                    const uint4 v = row[i];
-                    m2 = __vmaxu2(m2, v.x & 0x7FFF7FFFu);
-                    m2 = __vmaxu2(m2, v.y & 0x7FFF7FFFu);
-                    m2 = __vmaxu2(m2, v.z & 0x7FFF7FFFu);
-                    m2 = __vmaxu2(m2, v.w & 0x7FFF7FFFu);
+#pragma unroll
+            for (int gi = 0; gi < kGroupsPerThread; ++gi) {
+                const int G = tid + kConsumers * gi;
+                const int tk = div_by_recip(G, inf.rgpt);
+                tkg[gi] = tk;
+                cg[gi] = G - tk * gpt;
+                uint32_t m2 = 0u;
+                if (tk < nt) {
+                    const uint8_t* src = reinterpret_cast<const uint8_t*>(xt + tk * d_in + 32 * cg[gi]);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        xv[gi][j] = *reinterpret_cast<const uint4*>(src + 16 * ((j + rot_r) & 3));
+                        m2 = __vmaxu2(m2, xv[gi][j].x & 0x7FFF7FFFu);
+                        m2 = __vmaxu2(m2, xv[gi][j].y & 0x7FFF7FFFu);
+                        m2 = __vmaxu2(m2, xv[gi][j].z & 0x7FFF7FFFu);
+                        m2 = __vmaxu2(m2, xv[gi][j].w & 0x7FFF7FFFu);
+                    }
+                }
+                uint32_t am = max(m2 & 0xFFFFu, m2 >> 16) << 16;
+                if ((gpt & 31) == 0) {             // the warp's 32 groups belong to one token
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) am = max(am, __shfl_xor_sync(0xffffffffu, am, o));
+                    if (lane == 0 && tk < nt) atomicMax(&sh.amax_tok[tk], am);
+                } else if (tk < nt) {
+                    atomicMax(&sh.amax_tok[tk], am);
                 }
             }
-            uint32_t am = max(m2 & 0xFFFFu, m2 >> 16) << 16;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) am = max(am, __shfl_xor_sync(0xffffffffu, am, o));
-            if (lane == 0) sh.amax[warp] = am;
         }
         if (consumer_sync_or(!got)) {
             if (tid == 0) atomicOr(a.err, DFSSM_DEVERR_TIMEOUT);
             break;
         }
-        if (!usable) {                     // the producer recorded the error; just free the tile
-            if (tid == 0) ptx::mbar_arrive(&sh.empty[slot]);
+        if (!usable) {                     // the issuing warp recorded the error
+            if (warp == 0 && item + kBufs < hi) issue_item(a, sh, cur, kk + kBufs, item + kBufs, lane);
             continue;
         }
 
-        // ---- 2: quantise one 32-column group per thread
-        const int qs_row = d_in + kQsPad;
-        {
-            const int gpt = d_in >> 5;                 // groups per token
-            const int tk = tid / gpt, c = tid - tk * gpt;
+        // ---- 2: quantise the groups held in registers
+#pragma unroll
+        for (int gi = 0; gi < kGroupsPerThread; ++gi) {
+            const int tk = tkg[gi], c = cg[gi];
             if (tk < nt) {
-                uint32_t amb = 0u;
-                for (int p = 0; p < parts; ++p) amb = max(amb, sh.amax[tk * parts + p]);
+                const uint32_t amb = sh.amax_tok[tk];
                 const float am = __uint_as_float(amb);
-                const float inv = quant_inv(am);
-                // amax 0: q = 0; Inf or NaN: q = 0 and the error bit (output undefined)
-                const uint32_t keep = (amb != 0u && amb < 0x7F800000u) ? 0xFFFFFFFFu : 0u;
                 if (c == 0) {
                     sh.sx[tk] = quant_sx(am);
                     if (amb >= 0x7F800000u) atomicOr(a.err, DFSSM_DEVERR_NONFINITE);
                 }
-                // the four 16-byte loads in a lane-dependent order: 8 (and 16) consecutive lanes
-                // then touch distinct banks in the loads below and in the 8-byte q stores
-                const int r = ((lane >> 1) ^ (lane >> 3)) & 3;
-                const uint8_t* src = reinterpret_cast<const uint8_t*>(xt + tk * d_in + 32 * c);
-                int8_t* qs = sh.q + tk * qs_row + 32 * c;
-                int8_t* dq = inf.dbg_q ? inf.dbg_q + (int64_t)(t0 + tk) * d_in + 32 * c : nullptr;
-                uint32_t w0[4], w1[4];       // load j: columns 8 kk .. 8 kk + 3 and 8 kk + 4 .. 8 kk + 7
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int kk8 = 8 * ((j + r) & 3);
-                    const uint4 v = *reinterpret_cast<const uint4*>(src + 2 * kk8);
-                    w0[j] = quant_pack4(v.x, v.y, inv) & keep;
-                    w1[j] = quant_pack4(v.z, v.w, inv) & keep;
-                    *reinterpret_cast<uint2*>(qs + kk8) = make_uint2(w0[j], w1[j]);
-                    if (dq) *reinterpret_cast<uint2*>(dq + kk8) = make_uint2(w0[j], w1[j]);
-                }
-                // plane p of the group: columns 8 i + p (i = 0..3) as bytes i. The transposes give
-                // byte j = load j; rotating left by r bytes puts it at i = (j + r) % 4.
-                const uint4 lo = transpose4x4(w0[0], w0[1], w0[2], w0[3]);   // planes 0..3
-                const uint4 hi = transpose4x4(w1[0], w1[1], w1[2], w1[3]);   // planes 4..7
-                const uint32_t rot = 8u * (uint32_t)r;
-                const uint32_t P[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-                // plane p of segment c / 8: 4 bytes at 256 (c / 8) + 32 p + 4 (c % 8) of the token's row
+                // plane p of this group: 4 bytes at 256 (c / 8) + 32 p + 4 (c % 8) of the token's row
+                // (global), at 288 (c / 8) + 32 p + 4 (c % 8) of its shared row
                 int8_t* dst = a.q_ws + inf.q_off + (int64_t)(t0 + tk) * inf.qrow + 256 * (c >> 3) + 4 * (c & 7);
+                int8_t* qs = sh.q + tk * qs_row + kQsSegStride * (c >> 3) + 4 * (c & 7);
+                uint32_t P[8];
+                if (amb != 0u && amb < 0x7F800000u) {
+                    const float inv = quant_inv(am);
+                    // word h of every load: elements 2h, 2h + 1, i.e. planes 2h and 2h + 1 (the low
+                    // byte of each y is q)
 #pragma unroll
-                for (int p = 0; p < 8; ++p)
-                    *reinterpret_cast<uint32_t*>(dst + 32 * p) = __funnelshift_l(P[p], P[p], rot);
+                    for (int h = 0; h < 4; ++h) {
+                        uint32_t ylo[4], yhi[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) quant_pair(word_of(xv[gi][j], h), inv, ylo[j], yhi[j]);
+                        P[2 * h] = __byte_perm(__byte_perm(ylo[0], ylo[1], 0x0040u), __byte_perm(ylo[2], ylo[3], 0x4000u),
+                                               plane_sel);
+                        P[2 * h + 1] = __byte_perm(__byte_perm(yhi[0], yhi[1], 0x0040u),
+                                                   __byte_perm(yhi[2], yhi[3], 0x4000u), plane_sel);
+                    }
+                    if (inf.dbg_q) {           // natural order: element e of load j is column 8 kk_j + e
+                        int8_t* dq = inf.dbg_q + (int64_t)(t0 + tk) * d_in + 32 * c;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            uint32_t y[8];
+#pragma unroll
+                            for (int h = 0; h < 4; ++h) quant_pair(word_of(xv[gi][j], h), inv, y[2 * h], y[2 * h + 1]);
+                            const uint32_t lo4 = __byte_perm(__byte_perm(y[0], y[1], 0x0040u),
+                                                             __byte_perm(y[2], y[3], 0x4000u), 0x7610u);
+                            const uint32_t hi4 = __byte_perm(__byte_perm(y[4], y[5], 0x0040u),
+                                                             __byte_perm(y[6], y[7], 0x4000u), 0x7610u);
+                            *reinterpret_cast<uint2*>(dq + 8 * ((j + rot_r) & 3)) = make_uint2(lo4, hi4);
+                        }
+                    }
+                } else {                       // amax 0: q = 0; Inf or NaN: q = 0 and the error bit
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) P[p] = 0u;
+                    if (inf.dbg_q) {
+                        int8_t* dq = inf.dbg_q + (int64_t)(t0 + tk) * d_in + 32 * c;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) *reinterpret_cast<uint2*>(dq + 8 * j) = make_uint2(0u, 0u);
+                    }
+                }
+#pragma unroll
+                for (int p = 0; p < 8; ++p) {
+                    *reinterpret_cast<uint32_t*>(dst + 32 * p) = P[p];
+                    *reinterpret_cast<uint32_t*>(qs + 32 * p) = P[p];
+                }
+                // a final half segment: its absent half is zero in the shared tile (the MMA and
+                // the dp4a sums read whole 32-byte k-blocks)
+                if ((c >> 3) == nseg - 1 && (d_in & (kSegCols - 1)) != 0) {
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) *reinterpret_cast<uint32_t*>(qs + 32 * p + 16) = 0u;
+                }
             }
         }
         consumer_sync();
-        if (tid == 0) ptx::mbar_arrive(&sh.empty[slot]);   // the tile has been read
+        // the tile has been read: it takes the item after next
+        if (warp == 0 && item + kBufs < hi) issue_item(a, sh, cur, kk + kBufs, item + kBufs, lane);
 
-        // ---- 3: h = q W_B^T (two n-tiles) and sum q (n-tile of ones)
+        // ---- 3: h^T = W_B q^T (M = 16 LoRA rows, N = 8 tokens per n-tile) and sum q by dp4a;
+        //         k-block kb = (segment kb / 8, plane kb % 8), 32 bytes of the shared row
+        if (tid < kMaxT) sh.amax_tok[tid] = 0u;        // for the next item (read before the last barrier)
         {
-            int D0[4] = {0, 0, 0, 0}, D1[4] = {0, 0, 0, 0}, D2[4] = {0, 0, 0, 0};
-            const int mi = lane >> 3;                  // ldmatrix: this lane addresses row (lane & 7) of matrix mi
-            const int row = min((lane & 7) + 8 * (mi & 1), nt - 1);
-            const uint32_t a_base = ptx::smem_u32(sh.q) + (uint32_t)(row * qs_row + 16 * (mi >> 1));
-            const uint32_t mA = g < nt ? 0xFFFFFFFFu : 0u, mB = g + 8 < nt ? 0xFFFFFFFFu : 0u;
+            const bool two = inf.T > 8;                // a second n-tile (tokens 8..15)
+            const int nkb = nseg * 8;
+            int D0[4] = {0, 0, 0, 0}, D1[4] = {0, 0, 0, 0};
+            int s0 = 0, s1 = 0;                        // sum q of tokens g and g + 8, this lane's k slices
+            const uint32_t b_base =
+                ptx::smem_u32(sh.q) + (uint32_t)(min(lm_tok, nt - 1) * qs_row + lm_off);
+            const uint32_t m0 = g < nt ? 0xFFFFFFFFu : 0u, m1 = g + 8 < nt ? 0xFFFFFFFFu : 0u;
+            auto kblock = [&](int kb, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
+                const uint32_t off = (uint32_t)(kQsSegStride * (kb >> 3) + 32 * (kb & 7));
+                uint32_t b0, b1, b2, b3;
+                if (two) {
+                    ptx::ldmatrix_x4(b_base + off, b0, b1, b2, b3);
+                    b2 &= m1; b3 &= m1;
+                    mma_s8s8(D1, a0, a1, a2, a3, b2, b3);
+                    s1 = __dp4a((int)b2, 0x01010101, __dp4a((int)b3, 0x01010101, s1));
+                } else {
+                    ldmatrix_x2(b_base + off, b0, b1);
+                }
+                b0 &= m0; b1 &= m0;
+                mma_s8s8(D0, a0, a1, a2, a3, b0, b1);
+                s0 = __dp4a((int)b0, 0x01010101, __dp4a((int)b1, 0x01010101, s0));
+            };
 #pragma unroll
             for (int j = 0; j < kWbRegKb; ++j) {
                 const int kb = warp + kCWarps * j;
-                if (kb < nkb) {
-                    uint32_t a0, a1, a2, a3;
-                    ptx::ldmatrix_x4(a_base + 32u * (uint32_t)kb, a0, a1, a2, a3);
-                    a0 &= mA; a2 &= mA; a1 &= mB; a3 &= mB;
-                    mma_s8s8(D0, a0, a1, a2, a3, wbf[j][0], wbf[j][1]);
-                    mma_s8s8(D1, a0, a1, a2, a3, wbf[j][2], wbf[j][3]);
-                    mma_s8s8(D2, a0, a1, a2, a3, 0x01010101u, 0x01010101u);
-                }
+                if (kb < nkb) kblock(kb, wbf[j][0], wbf[j][1], wbf[j][2], wbf[j][3]);
             }
-            // d_in > 4096: the remaining k-blocks read W_B from global memory
-            const uint8_t* w0 = reinterpret_cast<const uint8_t*>(inf.wb) + (int64_t)g * d_in + 4 * cq;
-            const uint8_t* w1 = w0 + (int64_t)8 * d_in;
+            // d_in > 4096: the remaining k-blocks gather W_B from global memory
             for (int kb = warp + kCWarps * kWbRegKb; kb < nkb; kb += kCWarps) {
-                uint32_t a0, a1, a2, a3;
-                ptx::ldmatrix_x4(a_base + 32u * (uint32_t)kb, a0, a1, a2, a3);
-                a0 &= mA; a2 &= mA; a1 &= mB; a3 &= mB;
-                const int col = 32 * kb;
-                mma_s8s8(D0, a0, a1, a2, a3, __ldg(reinterpret_cast<const uint32_t*>(w0 + col)),
-                         __ldg(reinterpret_cast<const uint32_t*>(w0 + col + 16)));
-                mma_s8s8(D1, a0, a1, a2, a3, __ldg(reinterpret_cast<const uint32_t*>(w1 + col)),
-                         __ldg(reinterpret_cast<const uint32_t*>(w1 + col + 16)));
-                mma_s8s8(D2, a0, a1, a2, a3, 0x01010101u, 0x01010101u);
+                uint32_t f[4];
+                wb_fragment(inf.wb, d_in, kb, g, cq, f);
+                kblock(kb, f[0], f[1], f[2], f[3]);
             }
-            // D: (token g, n 2cq), (g, 2cq + 1), (g + 8, 2cq), (g + 8, 2cq + 1)
+            s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+            s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+            s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+            s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+            // D: (LoRA row g, token 2cq), (g, 2cq + 1), (g + 8, 2cq), (g + 8, 2cq + 1); D1 for tokens + 8
             int (*hw)[kHCols] = sh.h[warp];
-            hw[g][2 * cq] = D0[0];
-            hw[g][2 * cq + 1] = D0[1];
-            hw[g + 8][2 * cq] = D0[2];
-            hw[g + 8][2 * cq + 1] = D0[3];
-            hw[g][8 + 2 * cq] = D1[0];
-            hw[g][8 + 2 * cq + 1] = D1[1];
-            hw[g + 8][8 + 2 * cq] = D1[2];
-            hw[g + 8][8 + 2 * cq + 1] = D1[3];
+            hw[2 * cq][g] = D0[0];
+            hw[2 * cq + 1][g] = D0[1];
+            hw[2 * cq][g + 8] = D0[2];
+            hw[2 * cq + 1][g + 8] = D0[3];
+            hw[8 + 2 * cq][g] = D1[0];
+            hw[8 + 2 * cq + 1][g] = D1[1];
+            hw[8 + 2 * cq][g + 8] = D1[2];
+            hw[8 + 2 * cq + 1][g + 8] = D1[3];
             if (cq == 0) {
-                hw[g][kRank] = D2[0];
-                hw[g + 8][kRank] = D2[2];
+                hw[g][kRank] = s0;
+                hw[g + 8][kRank] = s1;
             }
         }
         consumer_sync();
