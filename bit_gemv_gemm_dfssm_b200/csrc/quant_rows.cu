@@ -51,7 +51,8 @@ constexpr int kItemElems = 32768;            // bf16 values of one item at most 
 constexpr int kGroupsPerThread = kItemElems / 32 / kConsumers;   // 2
 constexpr int kMaxT = 16;                    // tokens per item at most (two MMA n-tiles)
 constexpr int kBufs = 2;                     // x tiles
-constexpr int kInfos = kBufs + 1;            // item descriptors (a descriptor outlives its tile by one item)
+constexpr int kInfos = kBufs + 2;            // item descriptors (stage 4 of item k runs beside the issue of k + 3)
+constexpr int kIssueWarp = 15;               // issues items (stage 4 runs on warps 0..8)
 // shared q rows: plane-major like the global rows, but segments 288 bytes apart (the plane words of
 // the 4 segments a warp writes land on distinct banks) and rows 16 bytes longer than that (the 8
 // token rows an ldmatrix reads land on distinct banks)
@@ -87,8 +88,8 @@ struct RowsShared {
     int8_t q[kQsBytes];                      // q of the item, plane-major rows (see kQsSegStride)
     int h[kCWarps][kMaxT][kHCols];           // per-warp partial h and sum q
     ItemInfo info[kInfos];
-    uint32_t amax_tok[kMaxT];                // max |x| per token (fp32 bit pattern), zero between items
-    float sx[kMaxT];
+    uint32_t amax_tok[2][kMaxT];             // max |x| per token (fp32 bit pattern), by item parity
+    float sx[2][kMaxT];                      // s_x per token, by item parity
     Cursor cur;
     uint64_t full[kBufs];                    // tile and descriptor ready
 };
@@ -287,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1) quant_rows_kernel(const __grid_co
     // let the dependent prefill kernel start streaming weights; it waits for this grid before reading q
     ptx::pdl_launch_dependents();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (tid < kMaxT) sh.amax_tok[tid] = 0u;
+    if (tid < 2 * kMaxT) sh.amax_tok[tid >> 4][tid & 15] = 0u;
     if (tid == 0) {
         for (int b = 0; b < kBufs; ++b) ptx::mbar_init(&sh.full[b], 1);
         ptx::fence_mbar_init();
@@ -295,14 +296,15 @@ __global__ void __launch_bounds__(kThreads, 1) quant_rows_kernel(const __grid_co
     __syncthreads();
     int lo, hi;
     item_range(a, lo, hi);
-    Cursor& cur = sh.cur;     // warp 0's issue state (shared memory: no registers in the other warps)
-    if (warp == 0) {
+    const int n_items = hi - lo;
+    if (n_items <= 0) return;
+    Cursor& cur = sh.cur;     // the issuing warp's state (shared memory: no registers in the other warps)
+    if (warp == kIssueWarp) {
         if (lane == 0) cursor_start(a, cur);
         __syncwarp();
-        for (int kk = 0; kk < kBufs && lo + kk < hi; ++kk) issue_item(a, sh, cur, kk, lo + kk, lane);
+        for (int k = 0; k < kBufs && k < n_items; ++k) issue_item(a, sh, cur, k, lo + k, lane);
     }
 
-    // ------------------------------------------------------------------ consumers
     const int g = lane >> 2, cq = lane & 3;
     // the 16-byte x loads in a lane-dependent order (chunk kk_j = (j + rot_r) % 4 at load j):
     // 8 consecutive lanes then read distinct banks
@@ -317,73 +319,67 @@ __global__ void __launch_bounds__(kThreads, 1) quant_rows_kernel(const __grid_co
     uint32_t wbf[kWbRegKb][4];             // A fragments of this warp's k-blocks (plane-major K order)
 #pragma unroll
     for (int j = 0; j < kWbRegKb; ++j) wbf[j][0] = wbf[j][1] = wbf[j][2] = wbf[j][3] = 0u;
-    for (int item = lo, kk = 0; item < hi; ++item, ++kk) {
-        const int slot = kk % kBufs;
-        const bool got = ptx::mbar_wait(&sh.full[slot], (uint32_t)(kk / kBufs) & 1u);
-        const ItemInfo& inf = sh.info[kk % kInfos];
-        const int usable = got ? inf.usable : 0;
-        const int d_in = inf.d_in, nt = inf.nt, t0 = inf.t0;
-        const int gpt = d_in >> 5;                   // 32-column groups per token
-        const int nseg = (d_in + kSegCols - 1) / kSegCols;
-        const int qs_row = nseg * kQsSegStride + kQsRowPad;
-        const uint16_t* xt = sh.x[slot];
+    uint4 xv[kGroupsPerThread][4];         // this thread's groups of the item in flight
+    int tkg[kGroupsPerThread], cg[kGroupsPerThread];
 
-        if (usable && inf.lin != wb_lin) {
+    // ---- 1 (item k): wait for the tile, W_B fragments on a change of linear, load this thread's
+    //      groups G = tid, tid + 512 (token G / gpt, group G % gpt) and gather max |x| per token
+    auto stage1 = [&](int k) -> bool {
+        const bool got = ptx::mbar_wait(&sh.full[k % kBufs], (uint32_t)(k / kBufs) & 1u);
+        const ItemInfo& inf = sh.info[k % kInfos];
+        if (!got || !inf.usable) return got;
+        const int d_in = inf.d_in, nt = inf.nt, gpt = d_in >> 5;
+        if (inf.lin != wb_lin) {
             wb_lin = inf.lin;
             load_wb_fragments(inf.wb, d_in, warp, g, cq, wbf);
         }
-
-        // ---- 1: load this thread's groups G = tid, tid + 512 (token G / gpt, group G % gpt) and
-        //         their partial max |x|; per token the maximum goes to amax_tok
-        uint4 xv[kGroupsPerThread][4];
-        int tkg[kGroupsPerThread], cg[kGroupsPerThread];
-        if (usable) {
+        const uint16_t* xt = sh.x[k % kBufs];
+        uint32_t* amax_tok = sh.amax_tok[k & 1];
 #pragma unroll
-            for (int gi = 0; gi < kGroupsPerThread; ++gi) {
-                const int G = tid + kConsumers * gi;
-                const int tk = div_by_recip(G, inf.rgpt);
-                tkg[gi] = tk;
-                cg[gi] = G - tk * gpt;
-                uint32_t m2 = 0u;
-                if (tk < nt) {
-                    const uint8_t* src = reinterpret_cast<const uint8_t*>(xt + tk * d_in + 32 * cg[gi]);
+        for (int gi = 0; gi < kGroupsPerThread; ++gi) {
+            const int G = tid + kConsumers * gi;
+            const int tk = div_by_recip(G, inf.rgpt);
+            tkg[gi] = tk;
+            cg[gi] = G - tk * gpt;
+            uint32_t ma = 0u, mb = 0u;         // two chains
+            if (tk < nt) {
+                const uint8_t* src = reinterpret_cast<const uint8_t*>(xt + tk * d_in + 32 * cg[gi]);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        xv[gi][j] = *reinterpret_cast<const uint4*>(src + 16 * ((j + rot_r) & 3));
-                        m2 = __vmaxu2(m2, xv[gi][j].x & 0x7FFF7FFFu);
-                        m2 = __vmaxu2(m2, xv[gi][j].y & 0x7FFF7FFFu);
-                        m2 = __vmaxu2(m2, xv[gi][j].z & 0x7FFF7FFFu);
-                        m2 = __vmaxu2(m2, xv[gi][j].w & 0x7FFF7FFFu);
-                    }
-                }
-                uint32_t am = max(m2 & 0xFFFFu, m2 >> 16) << 16;
-                if ((gpt & 31) == 0) {             // the warp's 32 groups belong to one token
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) am = max(am, __shfl_xor_sync(0xffffffffu, am, o));
-                    if (lane == 0 && tk < nt) atomicMax(&sh.amax_tok[tk], am);
-                } else if (tk < nt) {
-                    atomicMax(&sh.amax_tok[tk], am);
+                for (int j = 0; j < 4; ++j) {
+                    xv[gi][j] = *reinterpret_cast<const uint4*>(src + 16 * ((j + rot_r) & 3));
+                    ma = __vmaxu2(ma, xv[gi][j].x & 0x7FFF7FFFu);
+                    mb = __vmaxu2(mb, xv[gi][j].y & 0x7FFF7FFFu);
+                    ma = __vmaxu2(ma, xv[gi][j].z & 0x7FFF7FFFu);
+                    mb = __vmaxu2(mb, xv[gi][j].w & 0x7FFF7FFFu);
                 }
             }
+            const uint32_t m2 = __vmaxu2(ma, mb);
+            uint32_t am = max(m2 & 0xFFFFu, m2 >> 16) << 16;
+            if ((gpt & 31) == 0) {             // the warp's 32 groups belong to one token
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) am = max(am, __shfl_xor_sync(0xffffffffu, am, o));
+                if (lane == 0 && tk < nt) atomicMax(&amax_tok[tk], am);
+            } else if (tk < nt) {
+                atomicMax(&amax_tok[tk], am);
+            }
         }
-        if (consumer_sync_or(!got)) {
-            if (tid == 0) atomicOr(a.err, DFSSM_DEVERR_TIMEOUT);
-            break;
-        }
-        if (!usable) {                     // the issuing warp recorded the error
-            if (warp == 0 && item + kBufs < hi) issue_item(a, sh, cur, kk + kBufs, item + kBufs, lane);
-            continue;
-        }
+        return true;
+    };
 
-        // ---- 2: quantise the groups held in registers
+    // ---- 2 (item k): quantise the groups held in registers
+    auto stage2 = [&](int k) {
+        const ItemInfo& inf = sh.info[k % kInfos];
+        const int d_in = inf.d_in, nt = inf.nt, t0 = inf.t0;
+        const int nseg = (d_in + kSegCols - 1) / kSegCols;
+        const int qs_row = nseg * kQsSegStride + kQsRowPad;
 #pragma unroll
         for (int gi = 0; gi < kGroupsPerThread; ++gi) {
             const int tk = tkg[gi], c = cg[gi];
             if (tk < nt) {
-                const uint32_t amb = sh.amax_tok[tk];
+                const uint32_t amb = sh.amax_tok[k & 1][tk];
                 const float am = __uint_as_float(amb);
                 if (c == 0) {
-                    sh.sx[tk] = quant_sx(am);
+                    sh.sx[k & 1][tk] = quant_sx(am);
                     if (amb >= 0x7F800000u) atomicOr(a.err, DFSSM_DEVERR_NONFINITE);
                 }
                 // plane p of this group: 4 bytes at 256 (c / 8) + 32 p + 4 (c % 8) of the token's row
@@ -441,86 +437,111 @@ __global__ void __launch_bounds__(kThreads, 1) quant_rows_kernel(const __grid_co
                 }
             }
         }
-        consumer_sync();
-        // the tile has been read: it takes the item after next
-        if (warp == 0 && item + kBufs < hi) issue_item(a, sh, cur, kk + kBufs, item + kBufs, lane);
+    };
 
-        // ---- 3: h^T = W_B q^T (M = 16 LoRA rows, N = 8 tokens per n-tile) and sum q by dp4a;
-        //         k-block kb = (segment kb / 8, plane kb % 8), 32 bytes of the shared row
-        if (tid < kMaxT) sh.amax_tok[tid] = 0u;        // for the next item (read before the last barrier)
-        {
-            const bool two = inf.T > 8;                // a second n-tile (tokens 8..15)
-            const int nkb = nseg * 8;
-            int D0[4] = {0, 0, 0, 0}, D1[4] = {0, 0, 0, 0};
-            int s0 = 0, s1 = 0;                        // sum q of tokens g and g + 8, this lane's k slices
-            const uint32_t b_base =
-                ptx::smem_u32(sh.q) + (uint32_t)(min(lm_tok, nt - 1) * qs_row + lm_off);
-            const uint32_t m0 = g < nt ? 0xFFFFFFFFu : 0u, m1 = g + 8 < nt ? 0xFFFFFFFFu : 0u;
-            auto kblock = [&](int kb, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
-                const uint32_t off = (uint32_t)(kQsSegStride * (kb >> 3) + 32 * (kb & 7));
-                uint32_t b0, b1, b2, b3;
-                if (two) {
-                    ptx::ldmatrix_x4(b_base + off, b0, b1, b2, b3);
-                    b2 &= m1; b3 &= m1;
-                    mma_s8s8(D1, a0, a1, a2, a3, b2, b3);
-                    s1 = __dp4a((int)b2, 0x01010101, __dp4a((int)b3, 0x01010101, s1));
-                } else {
-                    ldmatrix_x2(b_base + off, b0, b1);
-                }
-                b0 &= m0; b1 &= m0;
-                mma_s8s8(D0, a0, a1, a2, a3, b0, b1);
-                s0 = __dp4a((int)b0, 0x01010101, __dp4a((int)b1, 0x01010101, s0));
-            };
+    // ---- 3 (item k): h^T = W_B q^T (M = 16 LoRA rows, N = 8 tokens per n-tile) and sum q by dp4a;
+    //      k-block kb = (segment kb / 8, plane kb % 8), 32 bytes of the shared row
+    auto stage3 = [&](int k) {
+        const ItemInfo& inf = sh.info[k % kInfos];
+        const int d_in = inf.d_in, nt = inf.nt;
+        const int nseg = (d_in + kSegCols - 1) / kSegCols;
+        const int qs_row = nseg * kQsSegStride + kQsRowPad;
+        const bool two = inf.T > 8;                // a second n-tile (tokens 8..15)
+        const int nkb = nseg * 8;
+        int D0[4] = {0, 0, 0, 0}, D1[4] = {0, 0, 0, 0};
+        int s0 = 0, s1 = 0;                        // sum q of tokens g and g + 8, this lane's k slices
+        const uint32_t b_base = ptx::smem_u32(sh.q) + (uint32_t)(min(lm_tok, nt - 1) * qs_row + lm_off);
+        const uint32_t m0 = g < nt ? 0xFFFFFFFFu : 0u, m1 = g + 8 < nt ? 0xFFFFFFFFu : 0u;
+        auto kblock = [&](int kb, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
+            const uint32_t off = (uint32_t)(kQsSegStride * (kb >> 3) + 32 * (kb & 7));
+            uint32_t b0, b1, b2, b3;
+            if (two) {
+                ptx::ldmatrix_x4(b_base + off, b0, b1, b2, b3);
+                b2 &= m1; b3 &= m1;
+                mma_s8s8(D1, a0, a1, a2, a3, b2, b3);
+                s1 = __dp4a((int)b2, 0x01010101, __dp4a((int)b3, 0x01010101, s1));
+            } else {
+                ldmatrix_x2(b_base + off, b0, b1);
+            }
+            b0 &= m0; b1 &= m0;
+            mma_s8s8(D0, a0, a1, a2, a3, b0, b1);
+            s0 = __dp4a((int)b0, 0x01010101, __dp4a((int)b1, 0x01010101, s0));
+        };
 #pragma unroll
-            for (int j = 0; j < kWbRegKb; ++j) {
-                const int kb = warp + kCWarps * j;
-                if (kb < nkb) kblock(kb, wbf[j][0], wbf[j][1], wbf[j][2], wbf[j][3]);
-            }
-            // d_in > 4096: the remaining k-blocks gather W_B from global memory
-            for (int kb = warp + kCWarps * kWbRegKb; kb < nkb; kb += kCWarps) {
-                uint32_t f[4];
-                wb_fragment(inf.wb, d_in, kb, g, cq, f);
-                kblock(kb, f[0], f[1], f[2], f[3]);
-            }
-            s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
-            s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
-            s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
-            s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
-            // D: (LoRA row g, token 2cq), (g, 2cq + 1), (g + 8, 2cq), (g + 8, 2cq + 1); D1 for tokens + 8
-            int (*hw)[kHCols] = sh.h[warp];
-            hw[2 * cq][g] = D0[0];
-            hw[2 * cq + 1][g] = D0[1];
-            hw[2 * cq][g + 8] = D0[2];
-            hw[2 * cq + 1][g + 8] = D0[3];
-            hw[8 + 2 * cq][g] = D1[0];
-            hw[8 + 2 * cq + 1][g] = D1[1];
-            hw[8 + 2 * cq][g + 8] = D1[2];
-            hw[8 + 2 * cq + 1][g + 8] = D1[3];
-            if (cq == 0) {
-                hw[g][kRank] = s0;
-                hw[g + 8][kRank] = s1;
-            }
+        for (int j = 0; j < kWbRegKb; ++j) {
+            const int kb = warp + kCWarps * j;
+            if (kb < nkb) kblock(kb, wbf[j][0], wbf[j][1], wbf[j][2], wbf[j][3]);
         }
-        consumer_sync();
+        // d_in > 4096: the remaining k-blocks gather W_B from global memory
+        for (int kb = warp + kCWarps * kWbRegKb; kb < nkb; kb += kCWarps) {
+            uint32_t f[4];
+            wb_fragment(inf.wb, d_in, kb, g, cq, f);
+            kblock(kb, f[0], f[1], f[2], f[3]);
+        }
+        s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+        s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+        // D: (LoRA row g, token 2cq), (g, 2cq + 1), (g + 8, 2cq), (g + 8, 2cq + 1); D1 for tokens + 8
+        int (*hw)[kHCols] = sh.h[warp];
+        hw[2 * cq][g] = D0[0];
+        hw[2 * cq + 1][g] = D0[1];
+        hw[2 * cq][g + 8] = D0[2];
+        hw[2 * cq + 1][g + 8] = D0[3];
+        hw[8 + 2 * cq][g] = D1[0];
+        hw[8 + 2 * cq + 1][g] = D1[1];
+        hw[8 + 2 * cq][g + 8] = D1[2];
+        hw[8 + 2 * cq + 1][g + 8] = D1[3];
+        if (cq == 0) {
+            hw[g][kRank] = s0;
+            hw[g + 8][kRank] = s1;
+        }
+    };
 
-        // ---- 4: per-token results: thread (token tid / 17, column tid % 17)
+    // ---- 4 (item k): per-token results, thread (token tid / 17, column tid % 17)
+    auto stage4 = [&](int k) {
+        const ItemInfo& inf = sh.info[k % kInfos];
+        const int nt = inf.nt;
         if (tid < nt * kHCols) {
             const int tk = tid / kHCols, col = tid - tk * kHCols;
             int s = 0;
 #pragma unroll
             for (int w = 0; w < kCWarps; ++w) s += sh.h[w][tk][col];
-            const int t = t0 + tk;
+            const int t = inf.t0 + tk;
             TokStats* st = a.st_ws + inf.st_off + t;
             if (col < kRank) {
                 st->u[col] = __fmul_rn(inf.sb[col], (float)s);
                 if (inf.dbg_h) inf.dbg_h[(int64_t)t * kRank + col] = s;
             } else {
-                st->sx = sh.sx[tk];
+                const float sx = sh.sx[k & 1][tk];
+                st->sx = sx;
                 st->sumq = s;
-                if (inf.dbg_sx) inf.dbg_sx[t] = sh.sx[tk];
+                if (inf.dbg_sx) inf.dbg_sx[t] = sx;
             }
         }
+    };
+
+    // Two barriers per item. Phase X(k): stage 2 of item k, stage 4 of item k - 1, issue of
+    // item k + 2 (its tile was last read in stage 1 of item k). Phase Y(k): stage 3 of item k,
+    // stage 1 of item k + 1.
+    if (consumer_sync_or(!stage1(0))) {
+        if (tid == 0) atomicOr(a.err, DFSSM_DEVERR_TIMEOUT);
+        return;
     }
+    for (int k = 0; k < n_items; ++k) {
+        if (sh.info[k % kInfos].usable) stage2(k);
+        if (k >= 1 && sh.info[(k - 1) % kInfos].usable) stage4(k - 1);
+        if (warp == kIssueWarp && k + kBufs < n_items) issue_item(a, sh, cur, k + kBufs, lo + k + kBufs, lane);
+        consumer_sync();
+        if (sh.info[k % kInfos].usable) stage3(k);
+        if (tid < kMaxT) sh.amax_tok[k & 1][tid] = 0u;   // item k + 2 gathers into it
+        const bool got = k + 1 < n_items ? stage1(k + 1) : true;
+        if (consumer_sync_or(!got)) {
+            if (tid == 0) atomicOr(a.err, DFSSM_DEVERR_TIMEOUT);
+            return;
+        }
+    }
+    if (sh.info[(n_items - 1) % kInfos].usable) stage4(n_items - 1);
 }
 
 }  // namespace
