@@ -315,6 +315,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
                 afr[rt][2] = int8_pair_to_bf16x2(whi[0]);
                 afr[rt][3] = int8_pair_to_bf16x2(whi[1]);
             }
+            float2 alpha2[2][2], sa2[2][2];
+#pragma unroll
+            for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    alpha2[rt][hh] = make_float2(alpha[rt][hh], alpha[rt][hh]);
+                    sa2[rt][hh] = make_float2(sa[rt][hh], sa[rt][hh]);
+                }
+            uint16_t* const yb = reinterpret_cast<uint16_t*>(y_ptr);
+            float* const yf = reinterpret_cast<float*>(y_ptr);
+            // this warp's 32 rows as 16-byte row pieces per token: bf16, no debug export, all 32 rows
+            // inside d_out and d_out a multiple of 8 (16-byte aligned token rows)
+            const int orow_base = tc.row0 + 32 * q4;
+            const bool vec_store = lin_ok && y_bf16 && dbg_acc == nullptr && (d_out & 7) == 0 &&
+                                   orow_base + 32 <= d_out;
             // per-token scalars and u of chunk ch (tokens tok_base + 16 ch ..): lane l takes token
             // l / 2 and u[8 (l % 2) ..]; s_x and sum q from the even lanes
             const int tok_base = tc.tok0 + half * (BN / 2);
@@ -400,53 +415,97 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
                             ptx::mma_bf16_16816(lora[rt][tt], afr[rt][0], afr[rt][1], afr[rt][2], afr[rt][3], bl0, bl1);
                         }
                     }
-                    // element (rt, hh, tt, ee): row orow[rt][hh], token t0c + 8 tt + 2 cq + ee; branch-free,
-                    // with the validity of row and token as store predicates
-                    auto elements = [&](auto store_y, auto dbg_tag) {
-                        constexpr bool kDbg = decltype(dbg_tag)::value;
+                    // y for rows (rt, hh) and the token pair (2 cq, 2 cq + 1) of n-tile tt, in packed fp32
+                    // pairs: acc = 2 D - sum q as fp32 (the 1.5 * 2^23 bias, exact below 2^22), then
+                    // y = s_x (alpha acc + s_A (W_A u)) with the same roundings as the scalar form
+                    const float* sx_s = reinterpret_cast<const float*>(base);
+                    const int* sq_s = reinterpret_cast<const int*>(base + 64);
+                    float2 sx2[2];
+                    int kq[2][2];                              // 0x4B400000 - sum q per token
+#pragma unroll
+                    for (int tt = 0; tt < 2; ++tt) {
+                        const int tj = 8 * tt + 2 * cq;
+                        sx2[tt] = make_float2(sx_s[tj], sx_s[tj + 1]);
+                        kq[tt][0] = 0x4B400000 - sq_s[tj];
+                        kq[tt][1] = 0x4B400000 - sq_s[tj + 1];
+                    }
+                    float2 y2[2][2][2];                        // [rt][hh][tt]
+#pragma unroll
+                    for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                            for (int tt = 0; tt < 2; ++tt) {
+                                const int i0 = 4 * tt + 2 * hh;
+                                const float2 accf = fadd2(
+                                    make_float2(__int_as_float(2 * (int)v[rt][i0] + kq[tt][0]),
+                                                __int_as_float(2 * (int)v[rt][i0 + 1] + kq[tt][1])),
+                                    make_float2(-12582912.0f, -12582912.0f));
+                                const float2 l2 = make_float2(lora[rt][tt][2 * hh], lora[rt][tt][2 * hh + 1]);
+                                y2[rt][hh][tt] = fmul2(sx2[tt], ffma2(alpha2[rt][hh], accf, fmul2(sa2[rt][hh], l2)));
+                            }
+                    __syncwarp();                              // every lane is done with this chunk's staged values
+                    if (vec_store) {
+                        // bf16 pairs in the mma C layout -> stmatrix.trans into the chunk's (now free) staging
+                        // buffer as [16 tokens][32 rows], 16-byte pieces swizzled by (token / 2) % 4; then each
+                        // lane stores two 16-byte row pieces of one token
+                        const uint32_t stg = ptx::smem_u32(base);
 #pragma unroll
                         for (int tt = 0; tt < 2; ++tt) {
-#pragma unroll
-                            for (int ee = 0; ee < 2; ++ee) {
-                                const int tj = 8 * tt + 2 * cq + ee;      // token within the chunk
-                                const int t = t0c + tj;
-                                const bool tok_ok = t < a.m;
-                                const float sxt = reinterpret_cast<const float*>(base)[tj];
-                                const int sqt = reinterpret_cast<const int*>(base + 64)[tj];
-#pragma unroll
-                                for (int rt = 0; rt < 2; ++rt)
-#pragma unroll
-                                    for (int hh = 0; hh < 2; ++hh) {
-                                        const int acc = 2 * (int)v[rt][4 * tt + 2 * hh + ee] - sqt;
-                                        const float y = __fmul_rn(
-                                            sxt, __fmaf_rn(alpha[rt][hh], small_int_to_float(acc),
-                                                           __fmul_rn(sa[rt][hh], lora[rt][tt][2 * hh + ee])));
-                                        const bool ok = tok_ok && rok[rt][hh];
-                                        const int64_t idx = (int64_t)t * d_out + orow[rt][hh];
-                                        store_y(ok, idx, y);
-                                        if constexpr (kDbg) {
-                                            if (ok) dbg_acc[idx] = acc;
-                                        }
-                                    }
-                            }
+                            const int r = lane & 7, mi = lane >> 3;      // this lane addresses row r of matrix mi
+                            const uint32_t addr = stg + (uint32_t)((8 * tt + r) * 64 + 16 * (mi ^ ((r >> 1) & 3)));
+                            ptx::stmatrix_x4_trans(addr, bf16x2_of(y2[0][0][tt]), bf16x2_of(y2[0][1][tt]),
+                                                   bf16x2_of(y2[1][0][tt]), bf16x2_of(y2[1][1][tt]));
                         }
-                    };
-                    // the output type and the debug export are fixed per call: one code path each
-                    uint16_t* yb = reinterpret_cast<uint16_t*>(y_ptr);
-                    float* yf = reinterpret_cast<float*>(y_ptr);
-                    auto st_bf16 = [&](bool ok, int64_t idx, float y) {
-                        const uint16_t b = f32_to_bf16_bits(y);
-                        if (ok) yb[idx] = b;
-                    };
-                    auto st_f32 = [&](bool ok, int64_t idx, float y) {
-                        if (ok) yf[idx] = y;
-                    };
-                    using kNo = std::integral_constant<bool, false>;
-                    using kYes = std::integral_constant<bool, true>;
-                    if (dbg_acc == nullptr) {
-                        if (y_bf16) elements(st_bf16, kNo{}); else elements(st_f32, kNo{});
+                        __syncwarp();
+#pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            const int j = (lane >> 2) + 8 * i, c = lane & 3;
+                            const uint4 piece = ptx::lds128(stg + (uint32_t)(j * 64 + 16 * (c ^ ((j >> 1) & 3))));
+                            if (t0c + j < a.m)
+                                *reinterpret_cast<uint4*>(yb + (int64_t)(t0c + j) * d_out + orow_base + 8 * c) = piece;
+                        }
                     } else {
-                        if (y_bf16) elements(st_bf16, kYes{}); else elements(st_f32, kYes{});
+                        // element (rt, hh, tt, ee): row orow[rt][hh], token t0c + 8 tt + 2 cq + ee, with the
+                        // validity of row and token as store predicates
+                        auto elements = [&](auto store_y, auto dbg_tag) {
+                            constexpr bool kDbg = decltype(dbg_tag)::value;
+#pragma unroll
+                            for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+                                for (int ee = 0; ee < 2; ++ee) {
+                                    const int t = t0c + 8 * tt + 2 * cq + ee;
+                                    const bool tok_ok = t < a.m;
+#pragma unroll
+                                    for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+                                        for (int hh = 0; hh < 2; ++hh) {
+                                            const float y = ee ? y2[rt][hh][tt].y : y2[rt][hh][tt].x;
+                                            const bool ok = tok_ok && rok[rt][hh];
+                                            const int64_t idx = (int64_t)t * d_out + orow[rt][hh];
+                                            store_y(ok, idx, y);
+                                            if constexpr (kDbg) {
+                                                const int acc = 2 * (int)v[rt][4 * tt + 2 * hh + ee] -
+                                                                (0x4B400000 - kq[tt][ee]);
+                                                if (ok) dbg_acc[idx] = acc;
+                                            }
+                                        }
+                                }
+                        };
+                        auto st_bf16 = [&](bool ok, int64_t idx, float y) {
+                            const uint16_t b = f32_to_bf16_bits(y);
+                            if (ok) yb[idx] = b;
+                        };
+                        auto st_f32 = [&](bool ok, int64_t idx, float y) {
+                            if (ok) yf[idx] = y;
+                        };
+                        using kNo = std::integral_constant<bool, false>;
+                        using kYes = std::integral_constant<bool, true>;
+                        if (dbg_acc == nullptr) {
+                            if (y_bf16) elements(st_bf16, kNo{}); else elements(st_f32, kNo{});
+                        } else {
+                            if (y_bf16) elements(st_bf16, kYes{}); else elements(st_f32, kYes{});
+                        }
                     }
                 }
                 __syncwarp();

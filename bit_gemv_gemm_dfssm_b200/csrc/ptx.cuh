@@ -119,6 +119,13 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 
 // ---- ldmatrix: four 8x8 b16 matrices (= 8 rows x 16 bytes each); lane l addresses row l % 8 of matrix l / 8
+// four 8x8 b16 matrices from the mma C-fragment layout, stored transposed (a matrix row in shared
+// memory is a fragment column); lane l gives the address of row l % 8 of matrix l / 8
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t saddr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1,%2,%3,%4};"
+                 ::"r"(saddr), "r"(r0), "r"(r1), "r"(r2), "r"(r3) : "memory");
+}
+
 __device__ __forceinline__ void ldmatrix_x4(uint32_t saddr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(saddr));

@@ -125,16 +125,6 @@ __device__ __forceinline__ bool consumer_sync_or(bool p) {
     return r != 0;
 }
 
-// two fp32 products in one instruction, each rounded like the scalar __fmul_rn
-__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
-
 // two bf16 (one word) -> y = rint(x * inv) + 1.5 * 2^23 as fp32 bits, whose low byte is q. The
 // rounding add is the scalar __fadd_rn, which is never merged with the product into an FMA (a fused
 // x * inv + 1.5 * 2^23 would skip the product's own rounding and can move a tie).
