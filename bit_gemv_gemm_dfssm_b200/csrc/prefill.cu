@@ -6,24 +6,26 @@
 // packed 1-bit scaffold weights are expanded on the fly to int8 and multiplied
 // on INT8 tensor cores. With many tokens the contraction is a dense GEMM
 // (2 * d_in ops per token per output row), so here the expansion happens in
-// shared memory, once per 128-row x 128-column weight block, and the block is
-// reused by 256 tokens:
+// registers and tensor memory, once per 128-row x 128-column weight block, and
+// the block is reused by 192 tokens:
 //
 //   D[o, t] = sum_k b[o, k] * q[t, k]    (b = sign bit as 0/1, int32 in TMEM)
 //   acc     = 2 * D - sum_k q[t, k]       (a +-1 weight is 2b - 1)
 //
 // Persistent kernel, one CTA per SM, 16 warps with fixed roles:
-//   warp 0      TMA producer: 256-token x 128-byte tiles of the int8
+//   warp 0      TMA producer: 192-token x 128-byte tiles of the int8
 //               activations (permuted column order, 128B swizzle), no multicast
-//   warp 1      TMEM owner and MMA issuer: tcgen05.mma.kind::i8, M=128 rows,
-//               N=256 tokens, K=32 per instruction, 4 per 128-column block
-//   warps 4-7   bit expansion: each thread owns one weight row of the tile,
-//               loads the 32 sign bytes of a 256-column segment and writes, per
-//               128-byte k-block (four bit planes of that segment, the activation
-//               order of dfssm_internal.cuh), 128 0/1 bytes into the K-major
-//               SWIZZLE_128B layout the MMA reads
+//   warp 1      TMEM owner and MMA issuer: tcgen05.mma.kind::i8 with A in TMEM,
+//               M=128 rows, N=192 tokens, K=32 per instruction, 4 per 128-column
+//               block
+//   warps 4-7   bit expansion: each thread owns one weight row of the tile (its
+//               TMEM lane), loads the 32 sign bytes of a 256-column segment and
+//               stores, per 128-byte k-block (four bit planes of that segment, the
+//               activation order of dfssm_internal.cuh), 128 0/1 bytes into the
+//               k-block's TMEM stage with one tcgen05.st (no shared-memory traffic
+//               for the weights: shared memory carries only the activation tiles)
 //   warps 8-15  epilogue over its 32 TMEM lanes (= output rows) and half of the
-//               256 token columns, 16 tokens at a time: tcgen05.ld in the
+//               192 token columns, 16 tokens at a time: tcgen05.ld in the
 //               16x256b shape, which is the register layout of an mma.sync
 //               m16n8 accumulator, acc = 2D - sum q; the LoRA up-projection
 //               W_A u as bf16 warp MMAs in that same layout (W_A exact in bf16,
@@ -31,8 +33,9 @@
 //               and stores. The per-token scalars and the hi/lo u of each
 //               16-token chunk are staged in a warp-private, double-buffered
 //               smem slice
-// 4-stage shared-memory ring (mbarriers), two TMEM accumulator buffers of 256
-// columns so the epilogue of one tile overlaps the main loop of the next.
+// 4-stage ring (activation tiles in shared memory, expanded weights in TMEM,
+// mbarriers), two TMEM accumulator buffers of 192 columns so the epilogue of one
+// tile overlaps the main loop of the next (2 x 192 + 4 x 32 = 512 columns).
 // Every mbarrier wait is bounded; a timeout sets the plan's error word.
 #include <cuda.h>
 
@@ -47,11 +50,17 @@ namespace dfssm {
 namespace {
 
 constexpr int BM = 128;            // output rows per tile (MMA M, TMEM lanes)
-constexpr int BN = 256;            // tokens per tile (MMA N, TMEM columns)
-constexpr int BK = 128;            // k (bytes) per stage
-constexpr int STAGES = 4;
-constexpr int A_STAGE = BM * BK;   // 16 KB
-constexpr int B_STAGE = BN * BK;   // 32 KB
+constexpr int BN = 192;            // tokens per tile (MMA N, TMEM columns)
+constexpr int BK = 128;            // k (bytes) per TMA box (the 128-byte swizzle span)
+constexpr int SEG = kSegCols;      // k (bytes) per pipeline stage: one 256-column segment, 8 MMAs
+constexpr int A_STAGES = 2;        // expanded-weight stages (TMEM)
+constexpr int B_STAGES = 3;        // activation stages (shared memory)
+constexpr int B_HALF = BN * BK;    // 24 KB: one TMA box, K bytes 128 h .. of the segment
+constexpr int B_STAGE = 2 * B_HALF;
+// TMEM: two accumulator buffers of BN columns, then the A stages, SEG / 4 columns each
+// (4 int8 per 32-bit column, one weight row per lane)
+constexpr uint32_t A_COL0 = 2 * BN;
+constexpr uint32_t A_COLS = SEG / 4;
 constexpr int NUM_THREADS = 16 * 32;
 constexpr int EPI_WARPS = 8;                         // warps 8..15
 constexpr int EPI_THREADS = EPI_WARPS * 32;
@@ -60,8 +69,19 @@ constexpr int EPI_THREADS = EPI_WARPS * 32;
 constexpr int U_ROW = 12;                                 // words per token row (8 used)
 constexpr int STAT_CHUNK = 128 + 2 * 16 * U_ROW * 4;      // 1664 B
 constexpr int STAT_BYTES = EPI_WARPS * 2 * STAT_CHUNK;  // double-buffered, one pair per epilogue warp
-constexpr int SMEM_BYTES = STAGES * (A_STAGE + B_STAGE) + STAT_BYTES + 256 + 1024;
+// descriptor and stack entry of the first kLinCache linears, copied to shared memory at the
+// start: every role looks up each tile's linear, and chains of dependent global loads there
+// would stall the pipeline at every tile boundary
+constexpr int kLinCache = 256;
+struct LinCache {
+    DevDesc d;
+    dfssm_stack_entry e;
+};
+constexpr int LIN_CACHE_BYTES = kLinCache * (int)sizeof(LinCache);
+constexpr int SMEM_BYTES = B_STAGES * B_STAGE + STAT_BYTES + 256 + LIN_CACHE_BYTES + 1024;
 constexpr uint32_t TMEM_COLS = 512;
+static_assert(A_COL0 + A_STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
+static_assert(B_HALF % 1024 == 0, "SWIZZLE_128B atoms");
 
 struct PrefillArgs {
     const dfssm_stack_entry* entries;
@@ -91,49 +111,76 @@ struct TileCoord {
     int lin, row0, tok0;
 };
 
-__device__ __forceinline__ TileCoord tile_coord(const DevDesc* desc, int n, int n_tt, int tile) {
+__device__ __forceinline__ const DevDesc& lin_desc(const PrefillArgs& a, const LinCache* lc, int l) {
+    return l < kLinCache ? lc[l].d : a.desc[l];
+}
+__device__ __forceinline__ const dfssm_stack_entry& lin_entry(const PrefillArgs& a, const LinCache* lc, int l) {
+    return l < kLinCache ? lc[l].e : entry_at(a.entries, a.single, l);
+}
+
+__device__ __forceinline__ TileCoord tile_coord(const PrefillArgs& a, const LinCache* lc, int n_tt, int tile) {
     const int rt = tile / n_tt;                 // global 128-row tile index
     const int tt = tile - rt * n_tt;
-    const int base = desc[0].rt_begin;
-    int lo = 0, hi = n - 1;
+    const int base = lin_desc(a, lc, 0).rt_begin;
+    int lo = 0, hi = a.n - 1;
     while (lo < hi) {
         int mid = (lo + hi + 1) >> 1;
-        if (desc[mid].rt_begin - base <= rt) lo = mid; else hi = mid - 1;
+        if (lin_desc(a, lc, mid).rt_begin - base <= rt) lo = mid; else hi = mid - 1;
     }
     TileCoord c;
     c.lin = lo;
-    c.row0 = (rt - (desc[lo].rt_begin - base)) * BM;
+    c.row0 = (rt - (lin_desc(a, lc, lo).rt_begin - base)) * BM;
     c.tok0 = tt * BN;
     return c;
 }
 
 __device__ __forceinline__ void set_err(uint32_t* err, uint32_t bit) { atomicOr(err, bit); }
 
+__device__ __forceinline__ uint64_t globaltimer_elapsed(uint64_t t0) { return ptx::globaltimer() - t0; }
+
+// Wait for two mbarrier phases at once: the two probes go out back to back, so their latencies
+// overlap. Bounded like ptx::mbar_wait; false on timeout.
+__device__ __forceinline__ bool mbar_wait2(uint64_t* b0, uint32_t p0, uint64_t* b1, uint32_t p1) {
+    bool r0 = ptx::mbar_try_wait(b0, p0), r1 = ptx::mbar_try_wait(b1, p1);
+    if (r0 && r1) return true;
+    const uint64_t t0 = ptx::globaltimer();
+    while (!(r0 && r1)) {
+        if (!r0) r0 = ptx::mbar_try_wait(b0, p0);
+        if (!r1) r1 = ptx::mbar_try_wait(b1, p1);
+        if (globaltimer_elapsed(t0) > 1000000000ull) return false;
+    }
+    return true;
+}
+
 __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_constant__ PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned base (SWIZZLE_128B atoms), offset from the __shared__ array so the
     // compiler keeps shared-memory addressing
     uint8_t* smem = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint8_t* sA = smem;
-    uint8_t* sB = smem + STAGES * A_STAGE;
-    uint8_t* sStat = sB + STAGES * B_STAGE;
+    uint8_t* sB = smem;
+    uint8_t* sStat = sB + B_STAGES * B_STAGE;
     uint64_t* bars = reinterpret_cast<uint64_t*>(sStat + STAT_BYTES);
-    uint64_t* full_a = bars;               // [STAGES], 128 arrivals (expansion threads)
-    uint64_t* full_b = bars + STAGES;      // [STAGES], TMA transaction bytes
-    uint64_t* empty = bars + 2 * STAGES;   // [STAGES], MMA commit
-    uint64_t* acc_full = bars + 3 * STAGES;       // [2], MMA commit
-    uint64_t* acc_empty = bars + 3 * STAGES + 2;  // [2], EPI_THREADS epilogue arrivals
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 4);
+    LinCache* lc = reinterpret_cast<LinCache*>(sStat + STAT_BYTES + 256);
+    uint64_t* full_a = bars;                         // [A_STAGES], 128 arrivals (TMEM stores done)
+    uint64_t* empty_a = full_a + A_STAGES;           // [A_STAGES], MMA commit
+    uint64_t* full_b = empty_a + A_STAGES;           // [B_STAGES], TMA transaction bytes
+    uint64_t* empty_b = full_b + B_STAGES;           // [B_STAGES], MMA commit
+    uint64_t* acc_full = empty_b + B_STAGES;         // [2], MMA commit
+    uint64_t* acc_empty = acc_full + 2;              // [2], EPI_THREADS epilogue arrivals
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
     volatile uint32_t* abort_flag = tmem_slot + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_tt = (a.m + BN - 1) / BN;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < A_STAGES; ++s) {
             ptx::mbar_init(&full_a[s], 128);
+            ptx::mbar_init(&empty_a[s], 1);
+        }
+        for (int s = 0; s < B_STAGES; ++s) {
             ptx::mbar_init(&full_b[s], 1);
-            ptx::mbar_init(&empty[s], 1);
+            ptx::mbar_init(&empty_b[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(&acc_full[b], 1);
@@ -146,6 +193,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
         ptx::tmem_alloc(tmem_slot, TMEM_COLS);
         ptx::tmem_relinquish();
     }
+    for (int l = threadIdx.x; l < a.n && l < kLinCache; l += NUM_THREADS) {
+        lc[l].d = a.desc[l];
+        lc[l].e = entry_at(a.entries, a.single, l);
+    }
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
@@ -157,44 +208,51 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
             ptx::pdl_wait();
             int it = 0;
             for (int tile = blockIdx.x; tile < a.n_tiles && !*abort_flag; tile += gridDim.x) {
-                const TileCoord tc = tile_coord(a.desc, a.n, n_tt, tile);
+                const TileCoord tc = tile_coord(a, lc, n_tt, tile);
                 const CUtensorMap* tm = a.tmaps + tc.lin;
-                const int nkb = a.desc[tc.lin].qrow / BK;
-                for (int kb = 0; kb < nkb; ++kb, ++it) {
-                    const int s = it % STAGES;
-                    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                    if (!ptx::mbar_wait(&empty[s], ph ^ 1u)) { set_err(a.err, DFSSM_DEVERR_TIMEOUT); *abort_flag = 1; break; }
+                const int nseg = lin_desc(a, lc, tc.lin).qrow / SEG;
+                for (int sg = 0; sg < nseg; ++sg, ++it) {
+                    const int s = it % B_STAGES;
+                    const uint32_t ph = (uint32_t)(it / B_STAGES) & 1u;
+                    if (!ptx::mbar_wait(&empty_b[s], ph ^ 1u)) { set_err(a.err, DFSSM_DEVERR_TIMEOUT); *abort_flag = 1; break; }
                     ptx::mbar_arrive_expect_tx(&full_b[s], B_STAGE);
-                    ptx::tma_load_2d(sB + s * B_STAGE, tm, kb * BK, tc.tok0, &full_b[s]);
+                    ptx::tma_load_2d(sB + s * B_STAGE, tm, sg * SEG, tc.tok0, &full_b[s]);
+                    ptx::tma_load_2d(sB + s * B_STAGE + B_HALF, tm, sg * SEG + BK, tc.tok0, &full_b[s]);
                 }
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            int it = 0, tcount = 0;
+            int ita = 0, itb = 0, tcount = 0;
             for (int tile = blockIdx.x; tile < a.n_tiles && !*abort_flag; tile += gridDim.x, ++tcount) {
-                const TileCoord tc = tile_coord(a.desc, a.n, n_tt, tile);
-                const int nkb = a.desc[tc.lin].qrow / BK;
+                const TileCoord tc = tile_coord(a, lc, n_tt, tile);
+                const int nseg = lin_desc(a, lc, tc.lin).qrow / SEG;
                 const int buf = tcount & 1;
                 const uint32_t acc_ph = (uint32_t)(tcount >> 1) & 1u;
                 if (!ptx::mbar_wait(&acc_empty[buf], acc_ph ^ 1u)) { set_err(a.err, DFSSM_DEVERR_TIMEOUT); *abort_flag = 1; break; }
                 ptx::tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
                 bool ok = true;
-                for (int kb = 0; kb < nkb; ++kb, ++it) {
-                    const int s = it % STAGES;
-                    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                    if (!ptx::mbar_wait(&full_a[s], ph) || !ptx::mbar_wait(&full_b[s], ph)) {
+                for (int sg = 0; sg < nseg; ++sg, ++ita, ++itb) {
+                    const int sa = ita % A_STAGES, sb = itb % B_STAGES;
+                    if (!mbar_wait2(&full_a[sa], (uint32_t)(ita / A_STAGES) & 1u, &full_b[sb],
+                                    (uint32_t)(itb / B_STAGES) & 1u)) {
                         set_err(a.err, DFSSM_DEVERR_TIMEOUT); *abort_flag = 1; ok = false; break;
                     }
                     ptx::tc_fence_after();
-                    const uint64_t adesc = sw128_desc(ptx::smem_u32(sA + s * A_STAGE));
-                    const uint64_t bdesc = sw128_desc(ptx::smem_u32(sB + s * B_STAGE));
+                    const uint32_t a_tmem = tmem_base + A_COL0 + (uint32_t)sa * A_COLS;
+                    // segment half h = B box h; +32 bytes along K: +8 TMEM columns for A, +2 in the
+                    // 16-byte address field for B
 #pragma unroll
-                    for (int kk = 0; kk < BK / 32; ++kk)   // +32 bytes along K = +2 in the 16-byte address field
-                        ptx::mma_i8(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, kIdesc, (kb | kk) != 0);
-                    ptx::mma_commit(&empty[s]);
+                    for (int h = 0; h < 2; ++h) {
+                        const uint64_t bdesc = sw128_desc(ptx::smem_u32(sB + sb * B_STAGE + h * B_HALF));
+#pragma unroll
+                        for (int kk = 0; kk < BK / 32; ++kk)
+                            ptx::mma_i8_ts(d_tmem, a_tmem + 32 * h + 8 * kk, bdesc + 2 * kk, kIdesc, (sg | h | kk) != 0);
+                    }
+                    ptx::mma_commit(&empty_a[sa]);
+                    ptx::mma_commit(&empty_b[sb]);
                 }
                 if (!ok) break;
                 ptx::mma_commit(&acc_full[buf]);
@@ -202,68 +260,84 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
         }
     } else if (warp >= 4 && warp < 8) {
         // ------------------------------------------------ bit expansion (one weight row per thread)
+        // The sign bytes of this thread's row are loaded two segments ahead, across tile
+        // boundaries too: the first segments of the next tile are in flight while the last ones
+        // of this tile are expanded.
         const int r = threadIdx.x - 128;
+        struct RowSrc {
+            const uint8_t* src;
+            int nseg, rb;
+            bool valid;
+        };
+        auto row_src = [&](int tile) {
+            RowSrc rs{nullptr, 0, 0, false};
+            if (tile < a.n_tiles) {
+                const TileCoord tc = tile_coord(a, lc, n_tt, tile);
+                const DevDesc& d = lin_desc(a, lc, tc.lin);
+                const dfssm_stack_entry& e = lin_entry(a, lc, tc.lin);
+                rs.nseg = d.qrow / kSegCols;
+                rs.rb = d.d_in >> 3;
+                const int o = tc.row0 + r;
+                rs.valid = o < d.d_out && entry_ptrs_ok(e);
+                rs.src = e.w.sign + (int64_t)(rs.valid ? o : 0) * rs.rb;
+            }
+            return rs;
+        };
+        // segment sg of a row: words 0..3 and 4..7 (the second half is absent in a final half segment)
+        auto load_seg = [&](const RowSrc& rs, int sg, uint4& lo, uint4& hi) {
+            lo = make_uint4(0, 0, 0, 0);
+            hi = make_uint4(0, 0, 0, 0);
+            if (rs.valid && sg < rs.nseg) {
+                lo = __ldg(reinterpret_cast<const uint4*>(rs.src + 32 * sg));
+                if (32 * sg + 16 < rs.rb) hi = __ldg(reinterpret_cast<const uint4*>(rs.src + 32 * sg + 16));
+            }
+        };
+        // this row is TMEM lane r (the warp's lane quarter 32 (warp - 4) .. + 31)
+        const uint32_t a_lane = tmem_base + ((uint32_t)(32 * (warp - 4)) << 16) + A_COL0;
         int it = 0;
+        RowSrc cur = row_src(blockIdx.x), nxt = row_src(blockIdx.x + gridDim.x);
+        uint4 c_lo, c_hi, n_lo, n_hi;          // the next two segments of the stream
+        int have = 0;                          // how many of them belong to `cur` and are loaded
         for (int tile = blockIdx.x; tile < a.n_tiles && !*abort_flag; tile += gridDim.x) {
-            const TileCoord tc = tile_coord(a.desc, a.n, n_tt, tile);
-            const DevDesc d = a.desc[tc.lin];
-            const dfssm_stack_entry& e = entry_at(a.entries, a.single, tc.lin);
-            const int nseg = d.qrow / kSegCols;
-            const int rb = d.d_in >> 3;                 // sign bytes per row
-            const int o = tc.row0 + r;
-            const bool valid = o < d.d_out && entry_ptrs_ok(e);
-            const uint8_t* src = e.w.sign + (int64_t)(valid ? o : 0) * rb;
-            // segment sg of this row: words 0..3 and 4..7 (the second half is absent in a final half segment)
-            auto load_seg = [&](int sg, uint4& lo, uint4& hi) {
-                lo = make_uint4(0, 0, 0, 0);
-                hi = make_uint4(0, 0, 0, 0);
-                if (valid && sg < nseg) {
-                    lo = __ldg(reinterpret_cast<const uint4*>(src + 32 * sg));
-                    if (32 * sg + 16 < rb) hi = __ldg(reinterpret_cast<const uint4*>(src + 32 * sg + 16));
-                }
-            };
-            // two segments of look-ahead
-            uint4 c_lo, c_hi, n_lo, n_hi;
-            load_seg(0, c_lo, c_hi);
-            load_seg(1, n_lo, n_hi);
-            // swizzled destination of this row: atom (r/8), row-in-atom (r%8)
-            const uint32_t rrow = (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u;
-            const uint32_t xr = (uint32_t)(r & 7);
+            if (have < 1) load_seg(cur, 0, c_lo, c_hi);
+            if (have < 2) load_seg(cur, 1, n_lo, n_hi);
             bool ok = true;
-            for (int sg = 0; sg < nseg && ok; ++sg) {
+            for (int sg = 0; sg < cur.nseg && ok; ++sg, ++it) {
                 const uint32_t w[8] = {c_lo.x, c_lo.y, c_lo.z, c_lo.w, c_hi.x, c_hi.y, c_hi.z, c_hi.w};
                 c_lo = n_lo;
                 c_hi = n_hi;
-                load_seg(sg + 2, n_lo, n_hi);
+                // the segment two ahead: this tile's, else the next tile's first ones
+                const int k = sg + 2;
+                if (k < cur.nseg) load_seg(cur, k, n_lo, n_hi);
+                else load_seg(nxt, k - cur.nseg, n_lo, n_hi);
+                // segment sg: K byte 32 p + 4 c + i is plane p (0/1 bytes), i.e. TMEM column 8 p + c of
+                // the stage holds (w[c] >> p) & 0x01010101. Expanded before waiting for the stage, so
+                // that only the two 32-column stores follow the wait
+                uint32_t e[2][32];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int s = it % STAGES;
-                    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                    ++it;
-                    // one lane polls, the warp follows
-                    bool got = true;
-                    if ((threadIdx.x & 31) == 0) got = ptx::mbar_wait(&empty[s], ph ^ 1u);
-                    got = __shfl_sync(0xffffffffu, got, 0);
-                    __syncwarp();
-                    if (!got) { if ((threadIdx.x & 31) == 0) { set_err(a.err, DFSSM_DEVERR_TIMEOUT); *abort_flag = 1; } ok = false; break; }
-                    uint8_t* dst = sA + s * A_STAGE + rrow;
-                    // k-block 2 sg + h: bytes 32 p' + 4 c + i of plane p = 4 h + p' (0/1 bytes);
-                    // 16-byte chunk 2 p' holds words c = 0..3, chunk 2 p' + 1 words 4..7
+                for (int p = 0; p < 8; ++p)
 #pragma unroll
-                    for (int pp = 0; pp < 4; ++pp) {
-                        const int p = 4 * h + pp;
-                        const uint4 e0 = make_uint4((w[0] >> p) & 0x01010101u, (w[1] >> p) & 0x01010101u,
-                                                    (w[2] >> p) & 0x01010101u, (w[3] >> p) & 0x01010101u);
-                        const uint4 e1 = make_uint4((w[4] >> p) & 0x01010101u, (w[5] >> p) & 0x01010101u,
-                                                    (w[6] >> p) & 0x01010101u, (w[7] >> p) & 0x01010101u);
-                        *reinterpret_cast<uint4*>(dst + (((uint32_t)(2 * pp) ^ xr) << 4)) = e0;
-                        *reinterpret_cast<uint4*>(dst + (((uint32_t)(2 * pp + 1) ^ xr) << 4)) = e1;
-                    }
-                    ptx::fence_proxy_async_smem();
-                    ptx::mbar_arrive(&full_a[s]);
-                }
+                    for (int c = 0; c < 8; ++c) e[p >> 2][8 * (p & 3) + c] = (w[c] >> p) & 0x01010101u;
+                const int s = it % A_STAGES;
+                // one lane polls, the warp follows
+                bool got = true;
+                if ((threadIdx.x & 31) == 0) got = ptx::mbar_wait(&empty_a[s], ((uint32_t)(it / A_STAGES) & 1u) ^ 1u);
+                got = __shfl_sync(0xffffffffu, got, 0);
+                __syncwarp();
+                if (!got) { if ((threadIdx.x & 31) == 0) { set_err(a.err, DFSSM_DEVERR_TIMEOUT); *abort_flag = 1; } ok = false; break; }
+                ptx::tc_fence_after();                 // the MMAs that read this stage have completed
+                ptx::tmem_st_32x32b_x32(a_lane + (uint32_t)s * A_COLS, e[0]);
+                ptx::tmem_st_32x32b_x32(a_lane + (uint32_t)s * A_COLS + 32u, e[1]);
+                ptx::tmem_st_wait();
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(&full_a[s]);
             }
             if (!ok) break;
+            // the last two look-ahead loads of this tile fetched the next tile's segments 0 and 1
+            // (a one-segment tile reached only its segment 1: start over)
+            have = cur.nseg >= 2 ? min(2, nxt.nseg) : 0;
+            cur = nxt;
+            nxt = row_src(tile + 2 * gridDim.x);
         }
     } else if (warp >= 8) {
         // ------------------------------------------------ epilogue
@@ -277,9 +351,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
         uint8_t* stat_buf = sStat + (warp - 8) * 2 * STAT_CHUNK;
         int tcount = 0;
         for (int tile = blockIdx.x; tile < a.n_tiles && !*abort_flag; tile += gridDim.x, ++tcount) {
-            const TileCoord tc = tile_coord(a.desc, a.n, n_tt, tile);
-            const DevDesc d = a.desc[tc.lin];
-            const dfssm_stack_entry& e = entry_at(a.entries, a.single, tc.lin);
+            const TileCoord tc = tile_coord(a, lc, n_tt, tile);
+            const DevDesc d = lin_desc(a, lc, tc.lin);
+            const dfssm_stack_entry& e = lin_entry(a, lc, tc.lin);
             const bool lin_ok = entry_ptrs_ok(e);
             // entry fields in registers: the stores below must not force reloads
             void* const y_ptr = e.y;
