@@ -136,6 +136,27 @@ __device__ __forceinline__ TileCoord tile_coord(const PrefillArgs& a, const LinC
 
 __device__ __forceinline__ void set_err(uint32_t* err, uint32_t bit) { atomicOr(err, bit); }
 
+
+// Spin on a phase with the non-blocking probe (no suspend, so the waiter reacts as soon as the
+// phase completes); bounded by time like ptx::mbar_wait. Used where the hand-off latency is on
+// the critical path: the expansion warps refilling a TMEM stage the MMAs just released.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(ptx::smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_spin(uint64_t* bar, uint32_t parity) {
+    if (mbar_test(bar, parity)) return true;
+    const uint64_t t0 = ptx::globaltimer();
+    while (!mbar_test(bar, parity)) {
+        if (ptx::globaltimer() - t0 > 1000000000ull) return false;
+    }
+    return true;
+}
 __device__ __forceinline__ uint64_t globaltimer_elapsed(uint64_t t0) { return ptx::globaltimer() - t0; }
 
 // Wait for two mbarrier phases at once: the two probes go out back to back, so their latencies
@@ -321,7 +342,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) prefill_kernel(const __grid_co
                 const int s = it % A_STAGES;
                 // one lane polls, the warp follows
                 bool got = true;
-                if ((threadIdx.x & 31) == 0) got = ptx::mbar_wait(&empty_a[s], ((uint32_t)(it / A_STAGES) & 1u) ^ 1u);
+                if ((threadIdx.x & 31) == 0) got = mbar_spin(&empty_a[s], ((uint32_t)(it / A_STAGES) & 1u) ^ 1u);
                 got = __shfl_sync(0xffffffffu, got, 0);
                 __syncwarp();
                 if (!got) { if ((threadIdx.x & 31) == 0) { set_err(a.err, DFSSM_DEVERR_TIMEOUT); *abort_flag = 1; } ok = false; break; }
