@@ -63,6 +63,9 @@ DECODE_CASES = [  # (d_in, d_out, m, y_dtype)
 PREFILL_CASES = [
     (128, 1, 17, F32), (256, 129, 33, BF16), (384, 300, 300, F32), (2048, 200, 257, BF16),
     (4096, 256, 512, F32), (1024, 128, 100, BF16), (8192, 64, 40, F32),
+    # items of 10 and of 5 tokens in the quantiser (32768 / d_in not a power of two), a final
+    # half segment, a last row tile of 8 rows, ragged 192-token tiles
+    (3200, 520, 300, BF16), (6144, 136, 70, BF16),
 ]
 
 
