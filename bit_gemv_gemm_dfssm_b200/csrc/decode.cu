@@ -69,7 +69,8 @@ struct DecodeArgs {
     const DevDesc* desc;     // desc[0] is the first linear of this launch
     int n;
     int m;
-    const TokStats* st_ws;
+    const int* part;         // partial h of the quantisation kernel, per split
+    int splits;
     int64_t total_bytes;     // sign bytes of the n linears
     int slot_bytes;          // bytes of one ring slot
     int q_region;            // bytes of the staged-q region
@@ -79,14 +80,15 @@ struct DecodeArgs {
 struct Lin {
     int d_in, d_out, rb, nchunks, nblocks, y_dtype;
     int64_t byte_rel;        // first sign byte relative to desc[0]
-    int64_t st_off;
     const uint8_t* sign;
     const float* alpha;
     const float* sa;
     const int8_t* wa;
+    const float* sb;
     const uint16_t* x;
     void* y;
     int32_t* dbg_acc;
+    int32_t* dbg_h;
     bool ok;                 // entry pointers valid
 };
 
@@ -101,14 +103,15 @@ __device__ __forceinline__ void load_lin(const DecodeArgs& a, int l, Lin& L) {
     L.nblocks = (d.d_out + R - 1) / R;
     L.y_dtype = d.y_dtype;
     L.byte_rel = d.byte_begin - a.desc[0].byte_begin;
-    L.st_off = d.st_off;
     L.sign = e.w.sign;
     L.alpha = e.w.alpha;
     L.sa = e.w.sa;
     L.wa = e.w.wa;
+    L.sb = e.w.sb;
     L.x = reinterpret_cast<const uint16_t*>(e.x);
     L.y = e.y;
     L.dbg_acc = e.dbg.acc;
+    L.dbg_h = e.dbg.h;
     L.ok = entry_ptrs_ok(e);
 }
 
@@ -314,10 +317,16 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
         ptx::cp_async_wait<kStages - 1>();
         const bool last_chunk = cw.c.kc == L.nchunks - 1;
         if (last_chunk && u_lin != cw.c.l) {
-            // the LoRA vector u = s_B * h of this linear, from the quantisation kernel
+            // the LoRA vector u = s_B * h of this linear: h is the sum, in split order, of the
+            // quantisation kernel's partials (exact integers)
             ptx::pdl_wait();
-            for (int i = tid; i < m * kRank; i += kThreads)
-                ts.u[i >> 4][i & 15] = a.st_ws[L.st_off + (i >> 4)].u[i & 15];
+            for (int i = tid; i < m * kRank; i += kThreads) {
+                const int t = i >> 4, k = i & 15;
+                int h = 0;
+                for (int sp = 0; sp < a.splits; ++sp) h += __ldcg(a.part + part_index(cw.c.l, a.splits, sp, t, k));
+                ts.u[t][k] = __fmul_rn(L.sb[k], (float)h);
+                if (L.dbg_h) L.dbg_h[(int64_t)t * kRank + k] = h;
+            }
             u_lin = cw.c.l;
         }
         __syncthreads();
@@ -501,7 +510,8 @@ cudaError_t launch_cfg(const LaunchCtx& c) {
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     int grid = c.sm_count * per_sm;
     if (grid > blocks) grid = blocks;
-    DecodeArgs a{c.entries, c.single, c.desc, c.n, c.m, c.st_ws, total_bytes, geo.slot_bytes, geo.q_region};
+    DecodeArgs a{c.entries, c.single, c.desc, c.n, c.m, c.part, quant_splits(c), total_bytes, geo.slot_bytes,
+                 geo.q_region};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);

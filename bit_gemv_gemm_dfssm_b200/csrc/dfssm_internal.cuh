@@ -15,6 +15,13 @@ constexpr int kMaxDIn = 8192;
 constexpr int kMaxM = 65536;
 constexpr int kMaxSplits = 8;        // d_in splits of the quantisation kernel for m <= 16
 constexpr int kPartTok = 16;         // tokens covered by the split partials
+constexpr int kPartInts = 20;        // ints per token in the split partials (16 partial h, padded)
+
+// partial h of (linear lin, split sp of `splits`, token t, LoRA row k), written by the
+// quantisation kernel for m <= 16 and added up by the decode kernel
+__host__ __device__ inline int64_t part_index(int lin, int splits, int sp, int t, int k) {
+    return (((int64_t)lin * splits + sp) * kPartTok + t) * kPartInts + k;
+}
 
 // Per-linear shape and workspace offsets, resident in device memory.
 struct DevDesc {
@@ -79,6 +86,7 @@ struct LaunchCtx {
 cudaError_t launch_pack_sign(const void* src, int src_dtype, int d_out, int d_in, uint8_t* packed,
                              cudaStream_t s);
 cudaError_t launch_quant(const LaunchCtx& c);
+int quant_splits(const LaunchCtx& c);   // d_in splits of the m <= 16 quantisation kernel
 cudaError_t launch_decode(const LaunchCtx& c);
 cudaError_t launch_prefill(const LaunchCtx& c);
 

@@ -1,34 +1,26 @@
-// Per-token activation quantisation and the fused LoRA down-projection.
+// Per-token activation quantisation and the fused LoRA down-projection for the
+// decode path (1 <= m <= 16 tokens; many tokens go to quant_rows.cu).
 //
 // The scaffold matmul runs on int8 activations ("Density Field State Space
 // Models", gist.science technical summary, §2.C: packed bits expanded to int8
 // for an int8 x int8 -> int32 matmul), and the rank-16 int8 LoRA
 // (§2.B: W_B in R^{r x d_in}, r = 16, int8 with per-row scales) reads the
-// same int8 activations. For each token t of each linear this kernel computes
+// same int8 activations. For each token t of each linear:
 //   amax   = max_j |x[t,j]|                       (fp32, exact)
 //   q[t,j] = clamp(rint(x[t,j] * (127/amax)), +-127), s_x = amax/127 (IEEE fp32,
 //            round-to-nearest; amax == 0 gives q = 0, s_x = 0)
-//   sumq   = sum_j q[t,j]                          (int32)
 //   h[t,k] = sum_j W_B[k,j] q[t,j]                 (int32, warp MMA s8 x s8)
-//   u[t,k] = s_B[k] * h[t,k]                       (fp32)
-// and, for the prefill (m > 16), stores q in the plane-major int8 rows its
-// tensor-core kernel reads, plus s_x, sumq and u.
+// The decode kernel quantises x again into its own shared memory (same
+// arithmetic, same bytes) and computes s_x and sum q itself, so this kernel only
+// supplies h, as partial sums.
 //
-// A block owns one linear and up to kTokPerBlock = 16 tokens (one MMA tile;
-// many small blocks keep enough loads in flight). The 8 warps split the 32-column k-blocks of d_in
-// between them: pass 1 finds each token's amax, pass 2 quantises x straight
-// into MMA A fragments (16 tokens x 32 columns), runs h += q * W_B^T on the
-// warp MMA (m16n8k32, two n-tiles for the 16 LoRA rows) and writes q to a
-// shared tile. From there each thread takes 128 columns of a token and stores
-// them as eight 16-byte plane pieces (two 4x4 byte transposes with PRMT per
-// 32-column group).
-//
-// Few tokens (m <= 16, one round): the 128-column pieces of a linear are split
-// over S blocks so that W_B (the only large read) streams through many SMs. Every
-// split block finds the full-row amax itself, handles its own columns, and
-// writes partial h and sum q; the last split block to finish (atomic ticket)
-// adds the partials in split order, writes the per-token scalars and resets
-// the ticket for the next call.
+// The 128-column pieces of a linear are split over S blocks so that W_B (the
+// only large read) streams through many SMs. Every block finds the full-row amax
+// itself (x is a few KB per token), quantises its own columns straight into
+// warp-MMA A fragments and writes its partial h; the decode kernel adds the S
+// partials in split order (exact integer sums) and scales them by s_B. The W_B
+// fragments of each warp's first k-blocks are loaded before the amax pass, so
+// their latency hides behind the activation reads.
 #include "dfssm_internal.cuh"
 #include "epilogue.cuh"
 #include "ptx.cuh"
@@ -41,7 +33,6 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kTok = 16;              // tokens per round
 constexpr int kQsPad = 16;            // bytes of padding per shared q row
-constexpr int kTokPerBlock = 16;      // one round per block: more blocks in flight hide the loads
 
 struct QuantRed {
     unsigned int amax[kTok];     // fp32 bits of max |x| (order-preserving as unsigned; NaN above Inf)
@@ -83,36 +74,23 @@ __device__ __forceinline__ void mma_s8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) { return __byte_perm(a, b, sel); }
-
-// word r of the result = byte r of a, b, c, d (4x4 byte transpose)
-__device__ __forceinline__ uint4 transpose4x4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    const uint32_t t0 = prmt(a, b, 0x5140), t1 = prmt(a, b, 0x7362);
-    const uint32_t t2 = prmt(c, d, 0x5140), t3 = prmt(c, d, 0x7362);
-    return make_uint4(prmt(t0, t2, 0x5410), prmt(t0, t2, 0x7632), prmt(t1, t3, 0x5410), prmt(t1, t3, 0x7632));
-}
-
 struct QuantArgs {
     const dfssm_stack_entry* entries;
     dfssm_stack_entry single;
     const DevDesc* descs;
-    int m;
-    int splits;             // blocks per linear along d_in (1 when m > 16)
-    int8_t* q_ws;
-    TokStats* st_ws;
-    int* part;              // [linear][split][16 tokens][kPartInts] partial h and sum q (splits > 1)
-    unsigned int* tickets;  // one per linear, zero between calls
+    int m;                  // tokens, 1..16
+    int splits;             // blocks per linear along d_in
+    int* part;              // [linear][split][16 tokens][kPartInts] partial h (the decode kernel adds them)
     uint32_t* err;
 };
 
-constexpr int kPartInts = 20;   // 16 h + sum q, padded
+// W_B fragments of up to kWbAhead k-blocks per warp are loaded before the activation pass
+constexpr int kWbAhead = 4;
 
 __global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__ QuantArgs qa) {
     const dfssm_stack_entry* entries = qa.entries;
     const DevDesc* descs = qa.descs;
     const int m = qa.m;
-    int8_t* __restrict__ q_ws = qa.q_ws;
-    TokStats* __restrict__ st_ws = qa.st_ws;
     uint32_t* err = qa.err;
     extern __shared__ __align__(16) uint8_t smem_raw[];
     // let the dependent scaffold kernel start streaming weights right away;
@@ -135,183 +113,131 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__
     const int g = lane >> 2, c = lane & 3;
 
     QuantRed& red = *reinterpret_cast<QuantRed*>(smem_raw);
-    // [kTok][qs_row]: rows padded by 16 bytes so the 8 token rows of an MMA fragment hit 8 bank groups
+    // [m][qs_row]: rows padded by 16 bytes so the 8 token rows of an MMA fragment hit 8 bank groups
     const int qs_row = d_in + kQsPad;
     int8_t* q_s = reinterpret_cast<int8_t*>(smem_raw + ((sizeof(QuantRed) + 127) & ~(size_t)127));
 
     const uint16_t* xg = reinterpret_cast<const uint16_t*>(e.x);
     const uint8_t* wb = reinterpret_cast<const uint8_t*>(e.w.wb);
 
-    // split along d_in (few tokens) or along tokens (many tokens)
-    const int split = qa.splits > 1 ? (int)blockIdx.x : 0;
+    // this block's 128-column pieces of the linear
+    const int split = blockIdx.x;
     const int pc_lo = split * nquad / qa.splits, pc_hi = (split + 1) * nquad / qa.splits;
     const int kb_lo = 4 * pc_lo, kb_hi = 4 * pc_hi;
-    const int tb0 = qa.splits > 1 ? 0 : blockIdx.x * kTokPerBlock;
-    const int tb1 = min(m, tb0 + kTokPerBlock);
-    for (int t0 = tb0; t0 < tb1; t0 += kTok) {
-        const int nt = min(kTok, tb1 - t0);
+    const int nt = m;
 
-        // ---- pass 1: amax of each token's row, one warp per token, lanes across the row
-        for (int tk = warp; tk < nt; tk += kWarps) {
-            const uint4* p = reinterpret_cast<const uint4*>(xg + (int64_t)(t0 + tk) * d_in);
-            uint32_t am = 0u;
-#pragma unroll 8
-            for (int i = lane; i < (d_in >> 3); i += 32) am = absmax8_bits(p[i], am);
+    // B fragments (W_B rows g and g + 8) of this warp's first k-blocks: in flight during pass 1
+    uint32_t wbf[kWbAhead][4];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) am = max(am, __shfl_xor_sync(0xffffffffu, am, o));
-            if (lane == 0) red.amax[tk] = am;
+    for (int j = 0; j < kWbAhead; ++j) {
+        const int kb = kb_lo + warp + kWarps * j;
+        const int col = 32 * kb;
+        if (kb < kb_hi) {
+            wbf[j][0] = __ldg(reinterpret_cast<const uint32_t*>(wb + (int64_t)g * d_in + col + 4 * c));
+            wbf[j][1] = __ldg(reinterpret_cast<const uint32_t*>(wb + (int64_t)g * d_in + col + 16 + 4 * c));
+            wbf[j][2] = __ldg(reinterpret_cast<const uint32_t*>(wb + (int64_t)(g + 8) * d_in + col + 4 * c));
+            wbf[j][3] = __ldg(reinterpret_cast<const uint32_t*>(wb + (int64_t)(g + 8) * d_in + col + 16 + 4 * c));
+        } else {
+            wbf[j][0] = wbf[j][1] = wbf[j][2] = wbf[j][3] = 0u;
         }
-        if (tid >= nt && tid < kTok) red.amax[tid] = 0u;    // tokens past the round: q = 0
-        __syncthreads();
-        if (tid < kTok) {
-            const float am = __uint_as_float(red.amax[tid]);
-            if (tid < nt && !isfinite(am)) atomicOr(err, DFSSM_DEVERR_NONFINITE);
-            red.inv[tid] = quant_inv(am);
-            red.sx[tid] = quant_sx(am);
-        }
-        __syncthreads();
+    }
 
-        // ---- pass 2: quantise into A fragments, h += q * W_B^T, q -> shared tile
-        const float invA = red.inv[g], invB = red.inv[g + 8];
-        const bool zA = invA == 0.0f, zB = invB == 0.0f;
-        const bool hasA = g < nt, hasB = g + 8 < nt;
-        const uint16_t* xA = xg + (int64_t)(t0 + g) * d_in + 4 * c;
-        const uint16_t* xB = xg + (int64_t)(t0 + g + 8) * d_in + 4 * c;
-        int D0[4] = {0, 0, 0, 0}, D1[4] = {0, 0, 0, 0};
-        int sA = 0, sB = 0;
-#pragma unroll 4
-        for (int kb = kb_lo + warp; kb < kb_hi; kb += kWarps) {
-            const int col = 32 * kb;
-            const uint2 zero2 = make_uint2(0u, 0u);
-            const uint2 xa0 = hasA ? *reinterpret_cast<const uint2*>(xA + col) : zero2;
-            const uint2 xa1 = hasA ? *reinterpret_cast<const uint2*>(xA + col + 16) : zero2;
-            const uint2 xb0 = hasB ? *reinterpret_cast<const uint2*>(xB + col) : zero2;
-            const uint2 xb1 = hasB ? *reinterpret_cast<const uint2*>(xB + col + 16) : zero2;
-            const uint32_t a0 = quant4(xa0, invA, zA, sA);
-            const uint32_t a2 = quant4(xa1, invA, zA, sA);
-            const uint32_t a1 = quant4(xb0, invB, zB, sB);
-            const uint32_t a3 = quant4(xb1, invB, zB, sB);
-            // B fragments: W_B rows g (n-tile 0) and g + 8 (n-tile 1), k = 4c.. and 16 + 4c..
-            const uint32_t b00 = *reinterpret_cast<const uint32_t*>(wb + (int64_t)g * d_in + col + 4 * c);
-            const uint32_t b01 = *reinterpret_cast<const uint32_t*>(wb + (int64_t)g * d_in + col + 16 + 4 * c);
-            const uint32_t b10 = *reinterpret_cast<const uint32_t*>(wb + (int64_t)(g + 8) * d_in + col + 4 * c);
-            const uint32_t b11 = *reinterpret_cast<const uint32_t*>(wb + (int64_t)(g + 8) * d_in + col + 16 + 4 * c);
-            mma_s8s8(D0, a0, a1, a2, a3, b00, b01);
-            mma_s8s8(D1, a0, a1, a2, a3, b10, b11);
-            // the shared tile holds the round's nt tokens only
-            if (hasA) {
-                *reinterpret_cast<uint32_t*>(q_s + g * qs_row + col + 4 * c) = a0;
-                *reinterpret_cast<uint32_t*>(q_s + g * qs_row + col + 16 + 4 * c) = a2;
-            }
-            if (hasB) {
-                *reinterpret_cast<uint32_t*>(q_s + (g + 8) * qs_row + col + 4 * c) = a1;
-                *reinterpret_cast<uint32_t*>(q_s + (g + 8) * qs_row + col + 16 + 4 * c) = a3;
-            }
-        }
-        // quad reduction of the token sums
-        sA += __shfl_xor_sync(0xffffffffu, sA, 1);
-        sA += __shfl_xor_sync(0xffffffffu, sA, 2);
-        sB += __shfl_xor_sync(0xffffffffu, sB, 1);
-        sB += __shfl_xor_sync(0xffffffffu, sB, 2);
-        if (c == 0) {
-            red.sumq[warp][g] = sA;
-            red.sumq[warp][g + 8] = sB;
-        }
-        // D fragment: (token g, lora 2c), (g, 2c+1), (g+8, 2c), (g+8, 2c+1); D1 for lora + 8
-        red.h[warp][g][2 * c] = D0[0];
-        red.h[warp][g][2 * c + 1] = D0[1];
-        red.h[warp][g + 8][2 * c] = D0[2];
-        red.h[warp][g + 8][2 * c + 1] = D0[3];
-        red.h[warp][g][8 + 2 * c] = D1[0];
-        red.h[warp][g][8 + 2 * c + 1] = D1[1];
-        red.h[warp][g + 8][8 + 2 * c] = D1[2];
-        red.h[warp][g + 8][8 + 2 * c + 1] = D1[3];
-        __syncthreads();
+    // ---- pass 1: amax of each token's row, one warp per token, lanes across the row
+    for (int tk = warp; tk < nt; tk += kWarps) {
+        const uint4* p = reinterpret_cast<const uint4*>(xg + (int64_t)tk * d_in);
+        uint32_t am = 0u;
+#pragma unroll 8
+        for (int i = lane; i < (d_in >> 3); i += 32) am = absmax8_bits(p[i], am);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) am = max(am, __shfl_xor_sync(0xffffffffu, am, o));
+        if (lane == 0) red.amax[tk] = am;
+    }
+    if (tid >= nt && tid < kTok) red.amax[tid] = 0u;    // tokens past m: q = 0
+    __syncthreads();
+    if (tid < kTok) {
+        const float am = __uint_as_float(red.amax[tid]);
+        if (tid < nt && !isfinite(am)) atomicOr(err, DFSSM_DEVERR_NONFINITE);
+        red.inv[tid] = quant_inv(am);
+        red.sx[tid] = quant_sx(am);
+    }
+    __syncthreads();
 
-        // ---- per-token scalars: thread (token tid / 16, lora row tid % 16)
-        {
-            const int tk = tid >> 4, k = tid & 15;
-            int h = 0, sq = 0;
+    // ---- pass 2: quantise into A fragments, h += q * W_B^T, q -> shared tile (debug export)
+    const float invA = red.inv[g], invB = red.inv[g + 8];
+    const bool zA = invA == 0.0f, zB = invB == 0.0f;
+    const bool hasA = g < nt, hasB = g + 8 < nt;
+    const uint16_t* xA = xg + (int64_t)g * d_in + 4 * c;
+    const uint16_t* xB = xg + (int64_t)(g + 8) * d_in + 4 * c;
+    int D0[4] = {0, 0, 0, 0}, D1[4] = {0, 0, 0, 0};
+    auto kblock = [&](int kb, uint32_t b00, uint32_t b01, uint32_t b10, uint32_t b11) {
+        const int col = 32 * kb;
+        const uint2 zero2 = make_uint2(0u, 0u);
+        const uint2 xa0 = hasA ? *reinterpret_cast<const uint2*>(xA + col) : zero2;
+        const uint2 xa1 = hasA ? *reinterpret_cast<const uint2*>(xA + col + 16) : zero2;
+        const uint2 xb0 = hasB ? *reinterpret_cast<const uint2*>(xB + col) : zero2;
+        const uint2 xb1 = hasB ? *reinterpret_cast<const uint2*>(xB + col + 16) : zero2;
+        int unused = 0;
+        const uint32_t a0 = quant4(xa0, invA, zA, unused);
+        const uint32_t a2 = quant4(xa1, invA, zA, unused);
+        const uint32_t a1 = quant4(xb0, invB, zB, unused);
+        const uint32_t a3 = quant4(xb1, invB, zB, unused);
+        mma_s8s8(D0, a0, a1, a2, a3, b00, b01);
+        mma_s8s8(D1, a0, a1, a2, a3, b10, b11);
+        if (hasA) {
+            *reinterpret_cast<uint32_t*>(q_s + g * qs_row + col + 4 * c) = a0;
+            *reinterpret_cast<uint32_t*>(q_s + g * qs_row + col + 16 + 4 * c) = a2;
+        }
+        if (hasB) {
+            *reinterpret_cast<uint32_t*>(q_s + (g + 8) * qs_row + col + 4 * c) = a1;
+            *reinterpret_cast<uint32_t*>(q_s + (g + 8) * qs_row + col + 16 + 4 * c) = a3;
+        }
+    };
+#pragma unroll
+    for (int j = 0; j < kWbAhead; ++j) {
+        const int kb = kb_lo + warp + kWarps * j;
+        if (kb < kb_hi) kblock(kb, wbf[j][0], wbf[j][1], wbf[j][2], wbf[j][3]);
+    }
+    for (int kb = kb_lo + warp + kWarps * kWbAhead; kb < kb_hi; kb += kWarps) {
+        const int col = 32 * kb;
+        kblock(kb, __ldg(reinterpret_cast<const uint32_t*>(wb + (int64_t)g * d_in + col + 4 * c)),
+               __ldg(reinterpret_cast<const uint32_t*>(wb + (int64_t)g * d_in + col + 16 + 4 * c)),
+               __ldg(reinterpret_cast<const uint32_t*>(wb + (int64_t)(g + 8) * d_in + col + 4 * c)),
+               __ldg(reinterpret_cast<const uint32_t*>(wb + (int64_t)(g + 8) * d_in + col + 16 + 4 * c)));
+    }
+    // D fragment: (token g, lora 2c), (g, 2c+1), (g+8, 2c), (g+8, 2c+1); D1 for lora + 8
+    red.h[warp][g][2 * c] = D0[0];
+    red.h[warp][g][2 * c + 1] = D0[1];
+    red.h[warp][g + 8][2 * c] = D0[2];
+    red.h[warp][g + 8][2 * c + 1] = D0[3];
+    red.h[warp][g][8 + 2 * c] = D1[0];
+    red.h[warp][g][8 + 2 * c + 1] = D1[1];
+    red.h[warp][g + 8][8 + 2 * c] = D1[2];
+    red.h[warp][g + 8][8 + 2 * c + 1] = D1[3];
+    __syncthreads();
+
+    // ---- this split's partial h: thread (token tid / 16, lora row tid % 16). The decode kernel
+    // adds the splits' partials in split order and scales by s_B (exact integer sums).
+    {
+        const int tk = tid >> 4, k = tid & 15;
+        if (tk < nt) {
+            int h = 0;
 #pragma unroll
             for (int w = 0; w < kWarps; ++w) h += red.h[w][tk][k];
-            if (k == 0) {
-#pragma unroll
-                for (int w = 0; w < kWarps; ++w) sq += red.sumq[w][tk];
-            }
-            bool final_block = true;
-            if (qa.splits > 1) {
-                int* mine = qa.part + ((int64_t)lin * qa.splits + split) * kTok * kPartInts + tk * kPartInts;
-                mine[k] = h;
-                if (k == 0) mine[16] = sq;
-                // the block's partials are ordered before its ticket by the barrier and one
-                // device-scope fence (cumulative over what the barrier made visible to thread 0)
-                __syncthreads();
-                __shared__ unsigned int ticket;
-                if (tid == 0) {
-                    __threadfence();
-                    ticket = atomicAdd(qa.tickets + lin, 1u);
-                }
-                __syncthreads();
-                final_block = ticket == (unsigned int)(qa.splits - 1);
-                if (final_block) {
-                    __threadfence();
-                    h = 0;
-                    sq = 0;
-                    for (int sp = 0; sp < qa.splits; ++sp) {
-                        const int* pp = qa.part + ((int64_t)lin * qa.splits + sp) * kTok * kPartInts + tk * kPartInts;
-                        h += __ldcg(pp + k);
-                        if (k == 0) sq += __ldcg(pp + 16);
-                    }
-                    if (tid == 0) qa.tickets[lin] = 0u;
-                }
-            }
-            if (final_block && tk < nt) {
-                TokStats* st = st_ws + d.st_off + t0 + tk;
-                st->u[k] = __fmul_rn(e.w.sb[k], (float)h);
-                if (e.dbg.h) e.dbg.h[(int64_t)(t0 + tk) * kRank + k] = h;
-                if (k == 0) {
-                    st->sx = red.sx[tk];
-                    st->sumq = sq;
-                    if (e.dbg.sx) e.dbg.sx[t0 + tk] = red.sx[tk];
-                }
-            }
+            qa.part[part_index(lin, qa.splits, split, tk, k)] = h;
+            if (split == 0 && k == 0 && e.dbg.sx) e.dbg.sx[tk] = red.sx[tk];
         }
+    }
 
-        // ---- q out: token tk, 128-column piece pc = half hc of segment sg. For each 32-column
-        // group c4 of the piece, words W0..W7 of the natural bytes give plane p's four bytes
-        // (columns 32c + 8i + p, i = 0..3) as byte p % 4 of W[p / 4], W[2 + p / 4], W[4 + p / 4],
-        // W[6 + p / 4]; the four groups' words of plane p form one 16-byte piece.
+    // ---- debug export of q (natural order), this block's columns
+    if (e.dbg.q) {
         const int npc = pc_hi - pc_lo;
-        // the decode kernel (m <= 16) quantises into its own shared memory; only the prefill reads rows
-        const bool rows = m > kDecodeMaxTokens;
         for (int i = tid; i < nt * npc; i += kThreads) {
             const int tk = i / npc, pc = pc_lo + (i - tk * npc);
-            const int sg = pc >> 1, hc = pc & 1, t = t0 + tk;
-            const uint32_t* src = reinterpret_cast<const uint32_t*>(q_s + tk * qs_row + 128 * pc);
-            if (rows) {
-                uint32_t P[8][4];
+            const uint4* sq = reinterpret_cast<const uint4*>(q_s + tk * qs_row + 128 * pc);
+            uint4* dq = reinterpret_cast<uint4*>(e.dbg.q + (int64_t)tk * d_in + 128 * pc);
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    const uint32_t* W = src + 8 * c4;
-                    const uint4 lo = transpose4x4(W[0], W[2], W[4], W[6]);   // planes 0..3
-                    const uint4 hi = transpose4x4(W[1], W[3], W[5], W[7]);   // planes 4..7
-                    P[0][c4] = lo.x; P[1][c4] = lo.y; P[2][c4] = lo.z; P[3][c4] = lo.w;
-                    P[4][c4] = hi.x; P[5][c4] = hi.y; P[6][c4] = hi.z; P[7][c4] = hi.w;
-                }
-                // plane p of segment sg, K half hc: 16 bytes at 256 sg + 32 p + 16 hc of the token row
-                int8_t* base = q_ws + d.q_off + (int64_t)t * d.qrow + 256 * sg + 16 * hc;
-#pragma unroll
-                for (int p = 0; p < 8; ++p)
-                    *reinterpret_cast<uint4*>(base + 32 * p) = make_uint4(P[p][0], P[p][1], P[p][2], P[p][3]);
-            }
-            if (e.dbg.q) {
-                const uint4* sq = reinterpret_cast<const uint4*>(src);
-                uint4* dq = reinterpret_cast<uint4*>(e.dbg.q + (int64_t)t * d_in + 128 * pc);
-#pragma unroll
-                for (int u = 0; u < 8; ++u) dq[u] = sq[u];
-            }
+            for (int u = 0; u < 8; ++u) dq[u] = sq[u];
         }
-        __syncthreads();   // q_s and red are reused by the next round
     }
 }
 
@@ -319,20 +245,25 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__
 
 cudaError_t launch_quant_rows(const LaunchCtx& c);
 
+// d_in splits of the quantisation kernel for m <= 16 tokens: enough blocks to cover the SMs
+// twice, at least two 128-column pieces (8 k-blocks, one per warp) per split. The decode kernel
+// uses the same count to add the partials.
+int quant_splits(const LaunchCtx& c) {
+    int min_pc = 1 << 30;
+    for (int i = 0; i < c.n; ++i) min_pc = min(min_pc, c.host_desc[i].d_in / 128);
+    int splits = (2 * c.sm_count + c.n - 1) / c.n;
+    return max(1, min(splits, min(kMaxSplits, min_pc / 2)));
+}
+
+cudaError_t launch_quant_rows(const LaunchCtx& c);
+
 cudaError_t launch_quant(const LaunchCtx& c) {
     if (c.m > kDecodeMaxTokens) return launch_quant_rows(c);
-    int splits = 1;
-    if (c.m <= kTok) {
-        // enough blocks to cover the SMs twice, at least two 128-column pieces (8 k-blocks,
-        // one per warp) per split
-        int min_pc = 1 << 30;
-        for (int i = 0; i < c.n; ++i) min_pc = min(min_pc, c.host_desc[i].d_in / 128);
-        splits = (2 * c.sm_count + c.n - 1) / c.n;
-        splits = max(1, min(splits, min(kMaxSplits, min_pc / 2)));
-    }
-    dim3 grid(splits > 1 ? splits : (c.m + kTokPerBlock - 1) / kTokPerBlock, c.n);
-    const size_t smem = ((sizeof(QuantRed) + 127) & ~(size_t)127) + (size_t)kTok * (c.max_d_in + kQsPad);
-    QuantArgs qa{c.entries, c.single, c.desc, c.m, splits, c.q_ws, c.st_ws, c.part, c.tickets, c.err};
+    const int splits = quant_splits(c);
+    dim3 grid(splits, c.n);
+    // the shared q tile holds the call's m <= 16 tokens
+    const size_t smem = ((sizeof(QuantRed) + 127) & ~(size_t)127) + (size_t)c.m * (c.max_d_in + kQsPad);
+    QuantArgs qa{c.entries, c.single, c.desc, c.m, splits, c.part, c.err};
     quant_kernel<<<grid, kThreads, smem, c.stream>>>(qa);
     return cudaGetLastError();
 }
