@@ -47,7 +47,6 @@ struct dfssm_plan_s {
     TokStats* st_ws = nullptr;
     uint32_t* err = nullptr;
     int* part = nullptr;
-    unsigned int* tickets = nullptr;
     CUtensorMap* tmaps = nullptr;       // prefill: activation rows of each linear
     size_t ws_bytes = 0;
 };
@@ -103,7 +102,6 @@ void free_plan(dfssm_plan_s* p) {
     if (p->st_ws) cudaFree(p->st_ws);
     if (p->err) cudaFree(p->err);
     if (p->part) cudaFree(p->part);
-    if (p->tickets) cudaFree(p->tickets);
     if (p->tmaps) cudaFree(p->tmaps);
     delete p;
 }
@@ -180,7 +178,6 @@ dfssm_status dfssm_linear_plan(const dfssm_linear_desc* descs, int n_descs, dfss
     if (e == cudaSuccess) e = cudaMalloc(&p->tmaps, sizeof(CUtensorMap) * n_descs);
     const size_t part_bytes = sizeof(int) * (size_t)n_descs * kMaxSplits * kPartTok * 20;
     if (e == cudaSuccess) e = cudaMalloc(&p->part, part_bytes);
-    if (e == cudaSuccess) e = cudaMalloc(&p->tickets, sizeof(unsigned int) * n_descs);
     if (e != cudaSuccess) {
         cudaGetLastError();
         free_plan(p);
@@ -210,7 +207,6 @@ dfssm_status dfssm_linear_plan(const dfssm_linear_desc* descs, int n_descs, dfss
     e = cudaMemcpy(p->tmaps, tm.data(), sizeof(CUtensorMap) * n_descs, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(p->ddesc, p->hdesc.data(), sizeof(DevDesc) * n_descs, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemset(p->err, 0, 16);
-    if (e == cudaSuccess) e = cudaMemset(p->tickets, 0, sizeof(unsigned int) * n_descs);
     if (e == cudaSuccess) e = set_kernel_attributes(optin);
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) { free_plan(p); return DFSSM_ERR_CUDA; }
@@ -267,7 +263,6 @@ dfssm_status dfssm_linear_fwd(dfssm_plan plan, int32_t desc_index, const dfssm_l
     c.st_ws = plan->st_ws;
     c.err = plan->err;
     c.part = plan->part + (size_t)desc_index * kMaxSplits * kPartTok * 20;
-    c.tickets = plan->tickets + desc_index;
     c.tmaps = plan->tmaps + desc_index;
     c.max_d_in = hd.d_in;
     c.total_rows = hd.d_out;
@@ -300,7 +295,6 @@ dfssm_status dfssm_linear_stack_fwd(dfssm_plan plan, const dfssm_stack_entry* en
     c.st_ws = plan->st_ws;
     c.err = plan->err;
     c.part = plan->part;
-    c.tickets = plan->tickets;
     c.tmaps = plan->tmaps;
     c.max_d_in = max_d_in;
     c.total_rows = rows;

@@ -75,7 +75,6 @@ struct LaunchCtx {
     TokStats* st_ws;
     uint32_t* err;
     int* part;                         // split partials: n x kMaxSplits x 16 tokens x 20 ints
-    unsigned int* tickets;             // n split tickets, zero between calls
     const void* tmaps;                 // device array of CUtensorMap (prefill activation rows), one per desc
     int max_d_in;                      // largest d_in among the n linears
     int64_t total_rows;                // sum of d_out over the n linears

@@ -5,8 +5,8 @@
 // captured, allocators that must not be re-entered, or embedders whose memory
 // budget is fixed up front. This entry point needs no plan: the quantisation
 // and decode kernels run exactly as for dfssm_linear_fwd, with their scratch
-// (per-token scalars, split partials and their ticket, the linear's
-// descriptor and the error word) in the file-scope device array
+// (the quantisation kernel's split partials, the linear's descriptor and the
+// error word) in the file-scope device array
 // below, which every GPU that loads this library keeps until the process exits.
 //
 // Limits: 1 <= m <= DFSSM_NOALLOC_MAX_M (16) tokens, 128 <= d_in <= 8192.
@@ -32,11 +32,9 @@ constexpr int kMaxDevices = 64;
 // scratch layout (byte offsets, 256-byte aligned pieces)
 constexpr size_t kOffDesc = 0;                                                      // DevDesc
 constexpr size_t kOffErr = 256;                                                     // uint32 error word
-constexpr size_t kOffTicket = 512;                                                  // split ticket
-constexpr size_t kOffStats = 768;                                                   // TokStats[16]
-constexpr size_t kOffPart = kOffStats + ((sizeof(TokStats) * kNoAllocMaxM + 255) & ~(size_t)255);
-constexpr size_t kPartBytes = sizeof(int) * kMaxSplits * kPartTok * 20;
-constexpr size_t kScratchBytes = kOffPart + ((kPartBytes + 255) & ~(size_t)255);  // about 8 KB
+constexpr size_t kOffPart = 512;                                                    // split partials of h
+constexpr size_t kPartBytes = sizeof(int) * kMaxSplits * kPartTok * kPartInts;
+constexpr size_t kScratchBytes = kOffPart + ((kPartBytes + 255) & ~(size_t)255);  // about 11 KB
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kScratchBytes];
 
@@ -118,10 +116,9 @@ extern "C" dfssm_status dfssm_linear_fwd_noalloc(const dfssm_linear_desc* desc, 
     c.desc = ddesc;
     c.host_desc = &hd;
     c.q_ws = nullptr;     // the decode kernel quantises into shared memory; no activation rows are stored
-    c.st_ws = reinterpret_cast<TokStats*>(s->scratch + kOffStats);
+    c.st_ws = nullptr;     // the decode path reads only the split partials
     c.err = reinterpret_cast<uint32_t*>(s->scratch + kOffErr);
     c.part = reinterpret_cast<int*>(s->scratch + kOffPart);
-    c.tickets = reinterpret_cast<unsigned int*>(s->scratch + kOffTicket);   // zero at load, reset by each call
     c.tmaps = nullptr;
     c.max_d_in = desc->d_in;
     c.total_rows = desc->d_out;
