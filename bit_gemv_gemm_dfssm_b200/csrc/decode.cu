@@ -9,7 +9,10 @@
 //
 //  * Work: blocks of R = 64 * RT output rows (4 warps, RT 16-row tiles per
 //    warp), flattened over all linears of the call. Each CTA is persistent and
-//    owns a contiguous range of blocks holding an equal share of the sign bytes.
+//    owns a contiguous range of blocks holding an equal share of the work units
+//    (one per k-chunk, plus a charge for entering a linear; dfssm_internal.cuh):
+//    CTA durations follow these units, not bytes (a partial last block costs
+//    as many iterations as a full one, and entering a linear costs a quantisation).
 //  * Streaming: a block is consumed in k-chunks of 1024 columns (128 bytes per
 //    row). A ring of kStages shared-memory slots is filled with 16-byte
 //    cp.async; in slot row r, 16-byte chunk j sits at (j + r) mod 8, so the
@@ -71,7 +74,8 @@ struct DecodeArgs {
     int m;
     const int* part;         // partial h of the quantisation kernel, per split
     int splits;
-    int64_t total_bytes;     // sign bytes of the n linears
+    int64_t total_units;     // decode work units of the n linears (dfssm_internal.cuh)
+    int ri;                  // which work_begin: 0 for 128-row blocks, 1 for 64-row blocks
     int slot_bytes;          // bytes of one ring slot
     int q_region;            // bytes of the staged-q region
 };
@@ -79,7 +83,7 @@ struct DecodeArgs {
 // Fields of one linear, cached in registers while a cursor is on it.
 struct Lin {
     int d_in, d_out, rb, nchunks, nblocks, y_dtype;
-    int64_t byte_rel;        // first sign byte relative to desc[0]
+    int64_t work_rel;        // first work unit relative to desc[0]
     const uint8_t* sign;
     const float* alpha;
     const float* sa;
@@ -102,7 +106,7 @@ __device__ __forceinline__ void load_lin(const DecodeArgs& a, int l, Lin& L) {
     L.nchunks = (d.d_in / 8 + kChunkBytes - 1) / kChunkBytes;
     L.nblocks = (d.d_out + R - 1) / R;
     L.y_dtype = d.y_dtype;
-    L.byte_rel = d.byte_begin - a.desc[0].byte_begin;
+    L.work_rel = d.work_begin[a.ri] - a.desc[0].work_begin[a.ri];
     L.sign = e.w.sign;
     L.alpha = e.w.alpha;
     L.sa = e.w.sa;
@@ -124,7 +128,7 @@ struct Walk {
     Cursor c;
     Lin L;
     __device__ __forceinline__ bool valid(const DecodeArgs& a, int64_t hi) const {
-        return c.l < a.n && L.byte_rel + (int64_t)c.b * R * L.rb < hi;
+        return c.l < a.n && L.work_rel + kDecodeLinStart + (int64_t)c.b * L.nchunks < hi;
     }
     __device__ __forceinline__ void advance(const DecodeArgs& a) {
         if (++c.kc >= L.nchunks) {
@@ -135,18 +139,19 @@ struct Walk {
             }
         }
     }
-    // first block whose first sign byte is at or after `lo`
+    // first block whose first work unit is at or after `lo` (a linear's blocks follow its
+    // kDecodeLinStart entry units)
     __device__ void start(const DecodeArgs& a, int64_t lo) {
-        const int64_t base = a.desc[0].byte_begin;
+        const int64_t base = a.desc[0].work_begin[a.ri];
         int lo_l = 0, hi_l = a.n - 1;
         while (lo_l < hi_l) {
             const int mid = (lo_l + hi_l + 1) >> 1;
-            if (a.desc[mid].byte_begin - base <= lo) lo_l = mid; else hi_l = mid - 1;
+            if (a.desc[mid].work_begin[a.ri] - base <= lo) lo_l = mid; else hi_l = mid - 1;
         }
         c = Cursor{lo_l, 0, 0};
         load_lin<R>(a, c.l, L);
-        const int64_t bb = (int64_t)R * L.rb;
-        c.b = (int)((lo - L.byte_rel + bb - 1) / bb);
+        const int64_t rel = lo - L.work_rel - kDecodeLinStart;
+        c.b = rel <= 0 ? 0 : (int)((rel + L.nchunks - 1) / L.nchunks);
         if (c.b >= L.nblocks) {
             c.b = 0;
             if (++c.l < a.n) load_lin<R>(a, c.l, L);
@@ -278,8 +283,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
     const int g = lane >> 2, c = lane & 3;
     const int m = a.m;
 
-    const int64_t lo = a.total_bytes * blockIdx.x / gridDim.x;
-    const int64_t hi = a.total_bytes * (blockIdx.x + 1) / gridDim.x;
+    const int64_t lo = a.total_units * blockIdx.x / gridDim.x;
+    const int64_t hi = a.total_units * (blockIdx.x + 1) / gridDim.x;
     Walk<R> cw, lw;
     cw.start(a, lo);
     lw = cw;
@@ -497,10 +502,12 @@ template <int RT, int NT>
 cudaError_t launch_cfg(const LaunchCtx& c) {
     constexpr int R = 16 * RT * kWarps;
     const Geometry geo = geometry<RT>(c.m, c.max_d_in);
-    int64_t total_bytes = 0;
+    static_assert(R == 128 || R == 64, "work units exist for 128- and 64-row blocks");
+    static_assert(kChunkBytes * 8 == kDecodeChunkCols, "work unit = one k-chunk");
+    int64_t total_units = 0;
     int blocks = 0;
     for (int i = 0; i < c.n; ++i) {
-        total_bytes += (int64_t)c.host_desc[i].d_out * (c.host_desc[i].d_in / 8);
+        total_units += decode_units(c.host_desc[i].d_in, c.host_desc[i].d_out, R);
         blocks += (c.host_desc[i].d_out + R - 1) / R;
     }
     int per_sm = 0;
@@ -510,8 +517,8 @@ cudaError_t launch_cfg(const LaunchCtx& c) {
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     int grid = c.sm_count * per_sm;
     if (grid > blocks) grid = blocks;
-    DecodeArgs a{c.entries, c.single, c.desc, c.n, c.m, c.part, quant_splits(c), total_bytes, geo.slot_bytes,
-                 geo.q_region};
+    DecodeArgs a{c.entries, c.single, c.desc, c.n, c.m, c.part, quant_splits(c), total_units, R == 128 ? 0 : 1,
+                 geo.slot_bytes, geo.q_region};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);

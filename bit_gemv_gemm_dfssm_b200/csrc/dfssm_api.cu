@@ -150,7 +150,7 @@ dfssm_status dfssm_linear_plan(const dfssm_linear_desc* descs, int n_descs, dfss
     }
     p->n = n_descs;
     p->hdesc.resize(n_descs);
-    int64_t q_bytes = 0, st_count = 0, sign_bytes = 0;
+    int64_t q_bytes = 0, st_count = 0, units128 = 0, units64 = 0;
     int32_t rt = 0;
     for (int i = 0; i < n_descs; ++i) {
         DevDesc& d = p->hdesc[i];
@@ -165,8 +165,10 @@ dfssm_status dfssm_linear_plan(const dfssm_linear_desc* descs, int n_descs, dfss
         if (d.max_m > kDecodeMaxM) q_bytes += (int64_t)d.max_m * d.qrow;
         d.st_off = st_count;
         d.rt_begin = rt;
-        d.byte_begin = sign_bytes;
-        sign_bytes += (int64_t)d.d_out * (d.d_in / 8);
+        d.work_begin[0] = units128;
+        d.work_begin[1] = units64;
+        units128 += decode_units(d.d_in, d.d_out, 128);
+        units64 += decode_units(d.d_in, d.d_out, 64);
         st_count += d.max_m;
         rt += (d.d_out + 127) / 128;
     }

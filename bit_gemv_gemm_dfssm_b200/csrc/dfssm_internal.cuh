@@ -33,7 +33,7 @@ struct DevDesc {
     int64_t st_off;     // index of its first TokStats record
     int32_t qrow;       // activation bytes per token: d_in rounded up to a whole 256-column segment
     int32_t rt_begin;   // first 128-row tile of this linear in the flattened stack order
-    int64_t byte_begin; // sign bytes of all preceding linears (decode work balance)
+    int64_t work_begin[2]; // decode work units of all preceding linears, for 128- and 64-row blocks
 };
 
 // Per-token values the main kernels need after quantisation.
@@ -58,6 +58,17 @@ static_assert(sizeof(dfssm_stack_entry) == 104, "dfssm_stack_entry layout");
 // bit plane p of sign word c meet four consecutive activation bytes, and the 32
 // bytes of plane p form one K = 32 step of an int8 MMA. Token t, segment s is at
 // q_off + t * qrow + 256 s (K-major rows, loaded by TMA with 128-byte swizzle).
+// Decode work balance. The decode kernel splits the rows of all linears of a call over its CTAs
+// in work units: one per k-chunk of a row block (kDecodeChunkCols columns of R rows, a partial
+// last block counting in full), plus kDecodeLinStart for entering a linear (the CTA quantises
+// that linear's x first). A CTA's cost is close to linear in these units.
+constexpr int kDecodeChunkCols = 1024;
+constexpr int kDecodeLinStart = 2;
+__host__ __device__ inline int64_t decode_units(int d_in, int d_out, int rows) {
+    const int nch = (d_in + kDecodeChunkCols - 1) / kDecodeChunkCols;
+    return (int64_t)((d_out + rows - 1) / rows) * nch + kDecodeLinStart;
+}
+
 constexpr int kSegCols = 256;
 constexpr int kDecodeMaxTokens = 16;   // m up to this runs the decode kernel
 __host__ __device__ inline int seg_qrow(int d_in) { return (d_in + kSegCols - 1) / kSegCols * kSegCols; }
