@@ -66,6 +66,8 @@ __host__ __device__ __forceinline__ int q_stride(int d_in) { return ((d_in + 255
 constexpr int kStages = DFSSM_DECODE_STAGES;
 constexpr int kMaxTok = 16;
 
+constexpr int kStartTable = 900;   // CTAs whose start the host supplies (keeps the arguments under 4 KB)
+
 struct DecodeArgs {
     const dfssm_stack_entry* entries;
     dfssm_stack_entry single;
@@ -78,9 +80,15 @@ struct DecodeArgs {
     int ri;                  // which work_begin: 0 for 128-row blocks, 1 for 64-row blocks
     int slot_bytes;          // bytes of one ring slot
     int q_region;            // bytes of the staged-q region
+    // first (linear, block) of each CTA, found on the host (linear << 16 | block), so a CTA
+    // needs no search through the descriptors before its first loads; has_start = 0 when the
+    // grid is larger than the table (the CTAs then search themselves)
+    int has_start;
+    uint32_t start[kStartTable];
 };
 
 // Fields of one linear, cached in registers while a cursor is on it.
+// (kStartTable is defined before DecodeArgs.)
 struct Lin {
     int d_in, d_out, rb, nchunks, nblocks, y_dtype;
     int64_t work_rel;        // first work unit relative to desc[0]
@@ -138,6 +146,11 @@ struct Walk {
                 if (++c.l < a.n) load_lin<R>(a, c.l, L);
             }
         }
+    }
+    // start at (linear l, block b), as found by the host
+    __device__ void start_at(const DecodeArgs& a, int l, int b) {
+        c = Cursor{l, b, 0};
+        if (c.l < a.n) load_lin<R>(a, c.l, L);
     }
     // first block whose first work unit is at or after `lo` (a linear's blocks follow its
     // kDecodeLinStart entry units)
@@ -286,8 +299,16 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
     const int64_t lo = a.total_units * blockIdx.x / gridDim.x;
     const int64_t hi = a.total_units * (blockIdx.x + 1) / gridDim.x;
     Walk<R> cw, lw;
-    cw.start(a, lo);
+    if (a.has_start) cw.start_at(a, (int)(a.start[blockIdx.x] >> 16), (int)(a.start[blockIdx.x] & 0xFFFFu));
+    else cw.start(a, lo);
     lw = cw;
+    // the first linear's activations into L2 ahead of the weight stream (quantised below)
+    if (cw.valid(a, hi) && cw.L.ok) {
+        const char* xp = reinterpret_cast<const char*>(cw.L.x);
+        const int xbytes = m * cw.L.d_in * 2;
+        for (int off = 16 * tid; off < xbytes; off += 16 * kThreads)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(xp + off));
+    }
 
     // ---- prologue: kStages - 1 slots in flight
 #pragma unroll
@@ -518,7 +539,28 @@ cudaError_t launch_cfg(const LaunchCtx& c) {
     int grid = c.sm_count * per_sm;
     if (grid > blocks) grid = blocks;
     DecodeArgs a{c.entries, c.single, c.desc, c.n, c.m, c.part, quant_splits(c), total_units, R == 128 ? 0 : 1,
-                 geo.slot_bytes, geo.q_region};
+                 geo.slot_bytes, geo.q_region, 0, {}};
+    // each CTA's first block, as Walk::start finds it on the device
+    if (grid <= kStartTable && c.n < 65536) {
+        bool fits = true;
+        const int ri = R == 128 ? 0 : 1;
+        const int64_t base = c.host_desc[0].work_begin[ri];
+        int l = 0;
+        for (int i = 0; i < grid && fits; ++i) {
+            const int64_t lo = total_units * i / grid;
+            while (l + 1 < c.n && c.host_desc[l + 1].work_begin[ri] - base <= lo) ++l;
+            const DevDesc& d = c.host_desc[l];
+            const int nch = (d.d_in + kDecodeChunkCols - 1) / kDecodeChunkCols;
+            const int nblocks = (d.d_out + R - 1) / R;
+            const int64_t rel = lo - (d.work_begin[ri] - base) - kDecodeLinStart;
+            int b = rel <= 0 ? 0 : (int)((rel + nch - 1) / nch);
+            int sl = l;
+            if (b >= nblocks) { b = 0; ++sl; }
+            if (b > 0xFFFF) fits = false;
+            a.start[i] = ((uint32_t)sl << 16) | (uint32_t)b;
+        }
+        a.has_start = fits ? 1 : 0;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);
