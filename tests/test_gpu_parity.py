@@ -167,6 +167,27 @@ def test_stack_entry_desc_mismatch_sets_error_word():
         dfssm.dfssm_plan_destroy(plan)
 
 
+@pytest.mark.parametrize("m", [3, 40])
+def test_nonfinite_activation_row_sets_error_word(m):
+    # an Inf in token 1: the error word reports it (that token's outputs are undefined), while
+    # the other tokens, quantised independently, still match the oracle (decode and prefill)
+    d_in, d_out = 512, 96
+    x = synth.activations(SEED, 9, 11, m, d_in).copy()
+    x[1, 5] = 0x7F80                                  # +Inf
+    lin = Linear(SEED, 9, 11, d_in, d_out, m, F32, x=x, dbg=False)
+    plan = dfssm.dfssm_linear_plan([lin.desc()])
+    try:
+        stream = torch.cuda.current_stream().cuda_stream
+        dfssm.dfssm_linear_fwd(plan, 0, lin.weights(), lin.dx.data_ptr(), m, lin.dy.data_ptr(), None, stream)
+        st, bits = dfssm.dfssm_plan_check(plan)
+        assert st == dfssm.DFSSM_ERR_DEVICE_CHECK and bits & dfssm.DFSSM_DEVERR_NONFINITE
+    finally:
+        dfssm.dfssm_plan_destroy(plan)
+    keep = [t for t in range(m) if t != 1]
+    ref = oracle.linear(np.ascontiguousarray(x[keep]), lin.w, len(keep), d_in, d_out)
+    check_y(lin.y_host()[keep], ref["y"], term_bound(ref, lin.w), F32)
+
+
 def test_argument_errors_launch_nothing():
     lin = Linear(SEED, 9, 1, 256, 64, 4, F32)
     plan = dfssm.dfssm_linear_plan([lin.desc()])
