@@ -21,9 +21,10 @@
 //  * Activations: when a CTA reaches a new linear it quantises that linear's
 //    x itself (same fp32 arithmetic as the quantisation kernel, so the same
 //    bits) into shared memory, while its weight chunks are already in flight.
-//    Only the LoRA vector u = s_B * h comes from the quantisation kernel, and
-//    the CTA waits for that kernel (programmatic dependent launch) just before
-//    its first epilogue.
+//    Only the LoRA vector u = s_B * h comes from the quantisation kernel (for
+//    one token the slice kernel, which shares the SMs with this one), and the
+//    CTA waits for that kernel (programmatic dependent launch) just before its
+//    first epilogue.
 //  * Expansion: for a 32-bit word of sign bits w and bit position p,
 //    w & (0x01010101 << p) is four bytes, each 0 or 2^p: the bits of columns
 //    8i + p (i = 0..3) scaled by 2^p. One LOP3 expands four weights.
@@ -76,6 +77,7 @@ struct DecodeArgs {
     int m;
     const int* part;         // partial h of the quantisation kernel, per split
     int splits;
+    int slices;              // 1: one token, partial h per kLoraSliceCols-column slice (lora_slice_kernel)
     int64_t total_units;     // decode work units of the n linears (dfssm_internal.cuh)
     int ri;                  // which work_begin: 0 for 128-row blocks, 1 for 64-row blocks
     int slot_bytes;          // bytes of one ring slot
@@ -348,8 +350,10 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
             ptx::pdl_wait();
             for (int i = tid; i < m * kRank; i += kThreads) {
                 const int t = i >> 4, k = i & 15;
+                const int nsp = a.slices ? lora_slices(L.d_in) : a.splits;
+                const int stride = a.slices ? kLoraMaxSlices : a.splits;
                 int h = 0;
-                for (int sp = 0; sp < a.splits; ++sp) h += __ldcg(a.part + part_index(cw.c.l, a.splits, sp, t, k));
+                for (int sp = 0; sp < nsp; ++sp) h += __ldcg(a.part + part_index(cw.c.l, stride, sp, t, k));
                 ts.u[t][k] = __fmul_rn(L.sb[k], (float)h);
                 if (L.dbg_h) L.dbg_h[(int64_t)t * kRank + k] = h;
             }
@@ -538,7 +542,8 @@ cudaError_t launch_cfg(const LaunchCtx& c) {
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     int grid = c.sm_count * per_sm;
     if (grid > blocks) grid = blocks;
-    DecodeArgs a{c.entries, c.single, c.desc, c.n, c.m, c.part, quant_splits(c), total_units, R == 128 ? 0 : 1,
+    DecodeArgs a{c.entries, c.single, c.desc, c.n, c.m, c.part, quant_splits(c), use_lora_slices(c) ? 1 : 0,
+                 total_units, R == 128 ? 0 : 1,
                  geo.slot_bytes, geo.q_region, 0, {}};
     // each CTA's first block, as Walk::start finds it on the device
     if (grid <= kStartTable && c.n < 65536) {

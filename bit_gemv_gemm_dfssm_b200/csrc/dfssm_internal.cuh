@@ -93,6 +93,21 @@ struct LaunchCtx {
     cudaStream_t stream;
 };
 
+// One token: the LoRA down-projection h = W_B q runs as (linear, slice) items of
+// kLoraSliceCols columns in a kernel small enough to share the SMs with the decode kernel;
+// the decode kernel adds the slices' partial h (part_index with kLoraMaxSlices).
+constexpr int kLoraSliceCols = 2048;
+constexpr int kLoraMaxSlices = kMaxDIn / kLoraSliceCols;
+constexpr int kMaxSliceItems = 768;
+static_assert(kLoraMaxSlices <= kMaxSplits, "slice partials fit the split partial buffer");
+__host__ __device__ inline int lora_slices(int d_in) { return (d_in + kLoraSliceCols - 1) / kLoraSliceCols; }
+inline bool use_lora_slices(const LaunchCtx& c) {
+    if (c.m != 1) return false;
+    int items = 0;
+    for (int i = 0; i < c.n; ++i) items += lora_slices(c.host_desc[i].d_in);
+    return items <= kMaxSliceItems;
+}
+
 cudaError_t launch_pack_sign(const void* src, int src_dtype, int d_out, int d_in, uint8_t* packed,
                              cudaStream_t s);
 cudaError_t launch_quant(const LaunchCtx& c);

@@ -1,5 +1,6 @@
 // Per-token activation quantisation and the fused LoRA down-projection for the
-// decode path (1 <= m <= 16 tokens; many tokens go to quant_rows.cu).
+// decode path (1 <= m <= 16 tokens; many tokens go to quant_rows.cu). One token
+// takes the slice kernel at the end of this file.
 //
 // The scaffold matmul runs on int8 activations ("Density Field State Space
 // Models", gist.science technical summary, §2.C: packed bits expanded to int8
@@ -241,6 +242,117 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__
     }
 }
 
+// ---- one token: LoRA down-projection slices beside the decode kernel ------------------
+// Item (linear, slice) covers columns [2048 s, 2048 (s + 1)) of that linear. A CTA of two
+// warps brings the slice of W_B (16 rows) into shared memory with bulk copies while it finds
+// the token's amax over the whole row, then quantises its columns (the same fp32 arithmetic
+// as above) and takes h over the slice with dp4a, summed across the CTA with warp
+// reductions. 64 threads of at most 64 registers and ~33 KB of shared memory leave room
+// for three decode CTAs on the same SM, so the decode kernel's weight stream starts at once.
+constexpr int kSliceThreads = 64;
+constexpr int kSliceHead = 256;      // shared bytes before the W_B slice
+
+struct SliceArgs {
+    const dfssm_stack_entry* entries;
+    dfssm_stack_entry single;
+    const DevDesc* descs;
+    int n_items;
+    int* part;
+    uint32_t* err;
+    uint32_t item[kMaxSliceItems];   // linear << 8 | slice
+};
+
+struct SliceShared {
+    uint64_t bar;
+    unsigned int amax[kSliceThreads / 32];
+    int h[kSliceThreads / 32][kRank];
+};
+static_assert(sizeof(SliceShared) <= kSliceHead, "slice kernel shared header");
+
+__global__ void __launch_bounds__(kSliceThreads, 16) lora_slice_kernel(const __grid_constant__ SliceArgs sa) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    SliceShared& sh = *reinterpret_cast<SliceShared*>(smem_raw);
+    int8_t* wb_s = reinterpret_cast<int8_t*>(smem_raw + kSliceHead);     // [16][kLoraSliceCols]
+    // the decode kernel may start streaming weights now; it waits for this grid before its epilogues
+    ptx::pdl_launch_dependents();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) {
+        ptx::mbar_init(&sh.bar, 1);
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    uint32_t phase = 0;
+    for (int it = blockIdx.x; it < sa.n_items; it += gridDim.x) {
+        const int lin = (int)(sa.item[it] >> 8), sl = (int)(sa.item[it] & 0xFFu);
+        const dfssm_stack_entry& e = entry_at(sa.entries, sa.single, lin);
+        const bool desc_ok = !(sa.entries && e.desc_index != lin), ptrs_ok = entry_ptrs_ok(e);
+        if (!desc_ok || !ptrs_ok) {
+            if (tid == 0 && sl == 0) atomicOr(sa.err, desc_ok ? DFSSM_DEVERR_ENTRY_PTR : DFSSM_DEVERR_ENTRY_DESC);
+            continue;
+        }
+        const int d_in = sa.descs[lin].d_in;
+        const int c0 = sl * kLoraSliceCols, ncols = min(kLoraSliceCols, d_in - c0);
+        __syncthreads();                           // the previous item is done with wb_s and sh
+        if (tid == 0) {
+            ptx::mbar_arrive_expect_tx(&sh.bar, (uint32_t)(kRank * ncols));
+            for (int k = 0; k < kRank; ++k)
+                ptx::bulk_g2s(wb_s + k * kLoraSliceCols, e.w.wb + (int64_t)k * d_in + c0, (uint32_t)ncols, &sh.bar);
+        }
+        // amax of the whole row, as fp32 bit patterns (a NaN wins)
+        const uint16_t* x = reinterpret_cast<const uint16_t*>(e.x);
+        uint32_t am = 0u;
+        for (int ch = tid; ch < (d_in >> 3); ch += kSliceThreads)
+            am = absmax8_bits(__ldg(reinterpret_cast<const uint4*>(x) + ch), am);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) am = max(am, __shfl_xor_sync(0xffffffffu, am, o));
+        if (lane == 0) sh.amax[warp] = am;
+        __syncthreads();
+        am = sh.amax[0];
+#pragma unroll
+        for (int w = 1; w < kSliceThreads / 32; ++w) am = max(am, sh.amax[w]);
+        const float amax = __uint_as_float(am);
+        const float inv = quant_inv(amax);
+        const bool zero = inv == 0.0f;
+        if (tid == 0 && sl == 0) {
+            if (!isfinite(amax)) atomicOr(sa.err, DFSSM_DEVERR_NONFINITE);
+            if (e.dbg.sx) e.dbg.sx[0] = quant_sx(amax);
+        }
+        if (!ptx::mbar_wait(&sh.bar, phase)) {
+            if (tid == 0) atomicOr(sa.err, DFSSM_DEVERR_TIMEOUT);
+        }
+        phase ^= 1u;
+        // this thread's 8-column chunks of the slice: quantise, export, h += q . W_B
+        int h[kRank];
+#pragma unroll
+        for (int k = 0; k < kRank; ++k) h[k] = 0;
+        for (int j = tid; j < (ncols >> 3); j += kSliceThreads) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + c0) + j);
+            int unused = 0;
+            const uint32_t q0 = quant4(make_uint2(v.x, v.y), inv, zero, unused);
+            const uint32_t q1 = quant4(make_uint2(v.z, v.w), inv, zero, unused);
+            if (e.dbg.q) *reinterpret_cast<uint2*>(e.dbg.q + c0 + 8 * j) = make_uint2(q0, q1);
+#pragma unroll
+            for (int k = 0; k < kRank; ++k) {
+                const uint2 w = *reinterpret_cast<const uint2*>(wb_s + k * kLoraSliceCols + 8 * j);
+                h[k] = __dp4a((int)q0, (int)w.x, h[k]);
+                h[k] = __dp4a((int)q1, (int)w.y, h[k]);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < kRank; ++k) {
+            const int v = __reduce_add_sync(0xffffffffu, h[k]);
+            if (lane == k) sh.h[warp][k] = v;
+        }
+        __syncthreads();
+        if (tid < kRank) {
+            int hs = 0;
+#pragma unroll
+            for (int w = 0; w < kSliceThreads / 32; ++w) hs += sh.h[w][tid];
+            sa.part[part_index(lin, kLoraMaxSlices, sl, 0, tid)] = hs;
+        }
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_quant_rows(const LaunchCtx& c);
@@ -259,6 +371,15 @@ cudaError_t launch_quant_rows(const LaunchCtx& c);
 
 cudaError_t launch_quant(const LaunchCtx& c) {
     if (c.m > kDecodeMaxTokens) return launch_quant_rows(c);
+    if (use_lora_slices(c)) {
+        SliceArgs sa{c.entries, c.single, c.desc, 0, c.part, c.err, {}};
+        for (int i = 0; i < c.n; ++i)
+            for (int s = 0; s < lora_slices(c.host_desc[i].d_in); ++s) sa.item[sa.n_items++] = ((uint32_t)i << 8) | (uint32_t)s;
+        const int grid = sa.n_items < c.sm_count ? sa.n_items : c.sm_count;
+        const size_t smem = kSliceHead + (size_t)kRank * kLoraSliceCols;
+        lora_slice_kernel<<<grid, kSliceThreads, smem, c.stream>>>(sa);
+        return cudaGetLastError();
+    }
     const int splits = quant_splits(c);
     dim3 grid(splits, c.n);
     // the shared q tile holds the call's m <= 16 tokens
@@ -268,6 +389,14 @@ cudaError_t launch_quant(const LaunchCtx& c) {
     return cudaGetLastError();
 }
 
-cudaError_t set_quant_attr(int optin) { return allow_dyn_smem(quant_kernel, optin); }
+cudaError_t set_quant_attr(int optin) {
+    cudaError_t e = allow_dyn_smem(quant_kernel, optin);
+    if (e == cudaSuccess) e = allow_dyn_smem(lora_slice_kernel, optin);
+    // shared memory carved out like the decode kernel's, so both can share an SM
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(lora_slice_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+    return e;
+}
 
 }  // namespace dfssm
