@@ -436,7 +436,8 @@ def run_gpu(args, wl_name):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm"], "traffic": recorded_traffic(wl_name),
                      "peak_source": f"{peaks['src']} copy bandwidth",
-                     "timed": ("quant_kernel + decode_kernel" if m <= 16 else "quant_rows_kernel + prefill_kernel")
+                     "timed": ("lora_slice_kernel + decode_kernel" if m == 1 else
+                               "quant_kernel + decode_kernel" if m <= 16 else "quant_rows_kernel + prefill_kernel")
                      + " per call (PDL-overlapped)"},
         "e2e": e2e,
         "gpu_launches": 2 * args.steps,

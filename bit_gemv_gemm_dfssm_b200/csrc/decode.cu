@@ -10,7 +10,7 @@
 //  * Work: blocks of R = 64 * RT output rows (4 warps, RT 16-row tiles per
 //    warp), flattened over all linears of the call. Each CTA is persistent and
 //    owns a contiguous range of blocks holding an equal share of the work units
-//    (one per k-chunk, plus a charge for entering a linear; dfssm_internal.cuh):
+//    (per k-chunk, per block epilogue and for entering a linear; dfssm_internal.cuh):
 //    CTA durations follow these units, not bytes (a partial last block costs
 //    as many iterations as a full one, and entering a linear costs a quantisation).
 //  * Streaming: a block is consumed in k-chunks of 1024 columns (128 bytes per
@@ -93,6 +93,7 @@ struct DecodeArgs {
 // (kStartTable is defined before DecodeArgs.)
 struct Lin {
     int d_in, d_out, rb, nchunks, nblocks, y_dtype;
+    int bunits;              // work units of one block
     int64_t work_rel;        // first work unit relative to desc[0]
     const uint8_t* sign;
     const float* alpha;
@@ -114,6 +115,7 @@ __device__ __forceinline__ void load_lin(const DecodeArgs& a, int l, Lin& L) {
     L.d_out = d.d_out;
     L.rb = d.d_in >> 3;
     L.nchunks = (d.d_in / 8 + kChunkBytes - 1) / kChunkBytes;
+    L.bunits = decode_block_units(d.d_in);
     L.nblocks = (d.d_out + R - 1) / R;
     L.y_dtype = d.y_dtype;
     L.work_rel = d.work_begin[a.ri] - a.desc[0].work_begin[a.ri];
@@ -138,7 +140,7 @@ struct Walk {
     Cursor c;
     Lin L;
     __device__ __forceinline__ bool valid(const DecodeArgs& a, int64_t hi) const {
-        return c.l < a.n && L.work_rel + kDecodeLinStart + (int64_t)c.b * L.nchunks < hi;
+        return c.l < a.n && L.work_rel + kDecodeLinStart + (int64_t)c.b * L.bunits < hi;
     }
     __device__ __forceinline__ void advance(const DecodeArgs& a) {
         if (++c.kc >= L.nchunks) {
@@ -166,7 +168,7 @@ struct Walk {
         c = Cursor{lo_l, 0, 0};
         load_lin<R>(a, c.l, L);
         const int64_t rel = lo - L.work_rel - kDecodeLinStart;
-        c.b = rel <= 0 ? 0 : (int)((rel + L.nchunks - 1) / L.nchunks);
+        c.b = rel <= 0 ? 0 : (int)((rel + L.bunits - 1) / L.bunits);
         if (c.b >= L.nblocks) {
             c.b = 0;
             if (++c.l < a.n) load_lin<R>(a, c.l, L);
@@ -528,7 +530,7 @@ cudaError_t launch_cfg(const LaunchCtx& c) {
     constexpr int R = 16 * RT * kWarps;
     const Geometry geo = geometry<RT>(c.m, c.max_d_in);
     static_assert(R == 128 || R == 64, "work units exist for 128- and 64-row blocks");
-    static_assert(kChunkBytes * 8 == kDecodeChunkCols, "work unit = one k-chunk");
+    static_assert(kChunkBytes * 8 == kDecodeChunkCols, "kUnitChunk work units per k-chunk");
     int64_t total_units = 0;
     int blocks = 0;
     for (int i = 0; i < c.n; ++i) {
@@ -555,10 +557,10 @@ cudaError_t launch_cfg(const LaunchCtx& c) {
             const int64_t lo = total_units * i / grid;
             while (l + 1 < c.n && c.host_desc[l + 1].work_begin[ri] - base <= lo) ++l;
             const DevDesc& d = c.host_desc[l];
-            const int nch = (d.d_in + kDecodeChunkCols - 1) / kDecodeChunkCols;
+            const int bu = decode_block_units(d.d_in);
             const int nblocks = (d.d_out + R - 1) / R;
             const int64_t rel = lo - (d.work_begin[ri] - base) - kDecodeLinStart;
-            int b = rel <= 0 ? 0 : (int)((rel + nch - 1) / nch);
+            int b = rel <= 0 ? 0 : (int)((rel + bu - 1) / bu);
             int sl = l;
             if (b >= nblocks) { b = 0; ++sl; }
             if (b > 0xFFFF) fits = false;

@@ -59,14 +59,25 @@ static_assert(sizeof(dfssm_stack_entry) == 104, "dfssm_stack_entry layout");
 // bytes of plane p form one K = 32 step of an int8 MMA. Token t, segment s is at
 // q_off + t * qrow + 256 s (K-major rows, loaded by TMA with 128-byte swizzle).
 // Decode work balance. The decode kernel splits the rows of all linears of a call over its CTAs
-// in work units: one per k-chunk of a row block (kDecodeChunkCols columns of R rows, a partial
-// last block counting in full), plus kDecodeLinStart for entering a linear (the CTA quantises
-// that linear's x first). A CTA's cost is close to linear in these units.
+// in work units: kUnitChunk per k-chunk of a row block (kDecodeChunkCols columns of R rows, a
+// partial last block counting in full), kUnitBlock for the block's epilogue, and
+// kDecodeLinStart for entering a linear (the CTA quantises that linear's x first). A CTA's
+// cost is close to linear in these units.
+#ifndef DFSSM_UNIT_CHUNK
+#define DFSSM_UNIT_CHUNK 5
+#endif
+#ifndef DFSSM_UNIT_BLOCK
+#define DFSSM_UNIT_BLOCK 1
+#endif
 constexpr int kDecodeChunkCols = 1024;
-constexpr int kDecodeLinStart = 2;
+constexpr int kUnitChunk = DFSSM_UNIT_CHUNK;       // one k-chunk of a block
+constexpr int kUnitBlock = DFSSM_UNIT_BLOCK;       // the epilogue of a block
+constexpr int kDecodeLinStart = 2 * kUnitChunk;    // entering a linear (its quantisation pass)
+__host__ __device__ inline int decode_block_units(int d_in) {
+    return (d_in + kDecodeChunkCols - 1) / kDecodeChunkCols * kUnitChunk + kUnitBlock;
+}
 __host__ __device__ inline int64_t decode_units(int d_in, int d_out, int rows) {
-    const int nch = (d_in + kDecodeChunkCols - 1) / kDecodeChunkCols;
-    return (int64_t)((d_out + rows - 1) / rows) * nch + kDecodeLinStart;
+    return (int64_t)((d_out + rows - 1) / rows) * decode_block_units(d_in) + kDecodeLinStart;
 }
 
 constexpr int kSegCols = 256;
@@ -96,7 +107,10 @@ struct LaunchCtx {
 // One token: the LoRA down-projection h = W_B q runs as (linear, slice) items of
 // kLoraSliceCols columns in a kernel small enough to share the SMs with the decode kernel;
 // the decode kernel adds the slices' partial h (part_index with kLoraMaxSlices).
-constexpr int kLoraSliceCols = 2048;
+#ifndef DFSSM_LORA_SLICE_COLS
+#define DFSSM_LORA_SLICE_COLS 2048
+#endif
+constexpr int kLoraSliceCols = DFSSM_LORA_SLICE_COLS;
 constexpr int kLoraMaxSlices = kMaxDIn / kLoraSliceCols;
 constexpr int kMaxSliceItems = 768;
 static_assert(kLoraMaxSlices <= kMaxSplits, "slice partials fit the split partial buffer");

@@ -244,13 +244,28 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__
 
 // ---- one token: LoRA down-projection slices beside the decode kernel ------------------
 // Item (linear, slice) covers columns [2048 s, 2048 (s + 1)) of that linear. A CTA of two
-// warps brings the slice of W_B (16 rows) into shared memory with bulk copies while it finds
-// the token's amax over the whole row, then quantises its columns (the same fp32 arithmetic
-// as above) and takes h over the slice with dp4a, summed across the CTA with warp
-// reductions. 64 threads of at most 64 registers and ~33 KB of shared memory leave room
-// for three decode CTAs on the same SM, so the decode kernel's weight stream starts at once.
-constexpr int kSliceThreads = 64;
+// warps brings the slice of W_B into shared memory with bulk copies (kWbRows rows per pass)
+// while it finds the token's amax over the whole row, then quantises its columns (the same
+// fp32 arithmetic as above) and takes h over the slice with dp4a, summed across the CTA with
+// warp reductions. The CTA is kept small (64 threads, 32 registers, ~33 KB of shared memory)
+// so that it fits beside three decode CTAs on an SM: the decode kernel starts streaming
+// weights at once and waits for h only before its first epilogue.
+#ifndef DFSSM_SLICE_THREADS
+#define DFSSM_SLICE_THREADS 64
+#endif
+constexpr int kSliceThreads = DFSSM_SLICE_THREADS;
 constexpr int kSliceHead = 256;      // shared bytes before the W_B slice
+#ifndef DFSSM_SLICE_WB_ROWS
+#define DFSSM_SLICE_WB_ROWS 16
+#endif
+constexpr int kWbRows = DFSSM_SLICE_WB_ROWS;                    // W_B rows per shared-memory pass
+constexpr int kSliceChunks = kLoraSliceCols / 8 / kSliceThreads;  // 8-column chunks per thread
+#ifndef DFSSM_SLICE_REGS
+#define DFSSM_SLICE_REGS 32
+#endif
+constexpr int kSliceRegs = DFSSM_SLICE_REGS;     // register cap per thread
+static_assert(kSliceThreads % 32 == 0 && kLoraSliceCols % (8 * kSliceThreads) == 0, "slice chunks per thread");
+static_assert(kRank % kWbRows == 0, "W_B passes");
 
 struct SliceArgs {
     const dfssm_stack_entry* entries;
@@ -269,7 +284,7 @@ struct SliceShared {
 };
 static_assert(sizeof(SliceShared) <= kSliceHead, "slice kernel shared header");
 
-__global__ void __launch_bounds__(kSliceThreads, 16) lora_slice_kernel(const __grid_constant__ SliceArgs sa) {
+__global__ void __launch_bounds__(kSliceThreads, 65536 / (kSliceThreads * kSliceRegs)) lora_slice_kernel(const __grid_constant__ SliceArgs sa) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     SliceShared& sh = *reinterpret_cast<SliceShared*>(smem_raw);
     int8_t* wb_s = reinterpret_cast<int8_t*>(smem_raw + kSliceHead);     // [16][kLoraSliceCols]
@@ -292,11 +307,12 @@ __global__ void __launch_bounds__(kSliceThreads, 16) lora_slice_kernel(const __g
         }
         const int d_in = sa.descs[lin].d_in;
         const int c0 = sl * kLoraSliceCols, ncols = min(kLoraSliceCols, d_in - c0);
+        const int8_t* wb = e.w.wb + c0;
         __syncthreads();                           // the previous item is done with wb_s and sh
         if (tid == 0) {
-            ptx::mbar_arrive_expect_tx(&sh.bar, (uint32_t)(kRank * ncols));
-            for (int k = 0; k < kRank; ++k)
-                ptx::bulk_g2s(wb_s + k * kLoraSliceCols, e.w.wb + (int64_t)k * d_in + c0, (uint32_t)ncols, &sh.bar);
+            ptx::mbar_arrive_expect_tx(&sh.bar, (uint32_t)(kWbRows * ncols));
+            for (int k = 0; k < kWbRows; ++k)
+                ptx::bulk_g2s(wb_s + k * kLoraSliceCols, wb + (int64_t)k * d_in, (uint32_t)ncols, &sh.bar);
         }
         // amax of the whole row, as fp32 bit patterns (a NaN wins)
         const uint16_t* x = reinterpret_cast<const uint16_t*>(e.x);
@@ -317,31 +333,55 @@ __global__ void __launch_bounds__(kSliceThreads, 16) lora_slice_kernel(const __g
             if (!isfinite(amax)) atomicOr(sa.err, DFSSM_DEVERR_NONFINITE);
             if (e.dbg.sx) e.dbg.sx[0] = quant_sx(amax);
         }
-        if (!ptx::mbar_wait(&sh.bar, phase)) {
-            if (tid == 0) atomicOr(sa.err, DFSSM_DEVERR_TIMEOUT);
-        }
-        phase ^= 1u;
-        // this thread's 8-column chunks of the slice: quantise, export, h += q . W_B
-        int h[kRank];
+        // this thread's 8-column chunks j = tid + kSliceThreads i of the slice, quantised
+        uint32_t qv[kSliceChunks][2];
 #pragma unroll
-        for (int k = 0; k < kRank; ++k) h[k] = 0;
-        for (int j = tid; j < (ncols >> 3); j += kSliceThreads) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + c0) + j);
-            int unused = 0;
-            const uint32_t q0 = quant4(make_uint2(v.x, v.y), inv, zero, unused);
-            const uint32_t q1 = quant4(make_uint2(v.z, v.w), inv, zero, unused);
-            if (e.dbg.q) *reinterpret_cast<uint2*>(e.dbg.q + c0 + 8 * j) = make_uint2(q0, q1);
-#pragma unroll
-            for (int k = 0; k < kRank; ++k) {
-                const uint2 w = *reinterpret_cast<const uint2*>(wb_s + k * kLoraSliceCols + 8 * j);
-                h[k] = __dp4a((int)q0, (int)w.x, h[k]);
-                h[k] = __dp4a((int)q1, (int)w.y, h[k]);
+        for (int i = 0; i < kSliceChunks; ++i) {
+            const int j = tid + kSliceThreads * i;
+            qv[i][0] = qv[i][1] = 0u;
+            if (j < (ncols >> 3)) {
+                const uint4 v = __ldg(reinterpret_cast<const uint4*>(x + c0) + j);
+                int unused = 0;
+                qv[i][0] = quant4(make_uint2(v.x, v.y), inv, zero, unused);
+                qv[i][1] = quant4(make_uint2(v.z, v.w), inv, zero, unused);
+                if (e.dbg.q) *reinterpret_cast<uint2*>(e.dbg.q + c0 + 8 * j) = make_uint2(qv[i][0], qv[i][1]);
             }
         }
+        // h += q . W_B, kWbRows LoRA rows per pass through the shared buffer, each pass summed
+        // across the warp (redux.sync) into sh.h
 #pragma unroll
-        for (int k = 0; k < kRank; ++k) {
-            const int v = __reduce_add_sync(0xffffffffu, h[k]);
-            if (lane == k) sh.h[warp][k] = v;
+        for (int k0 = 0; k0 < kRank; k0 += kWbRows) {
+            if (k0 > 0) {
+                __syncthreads();                   // every thread is done with the previous rows
+                if (tid == 0) {
+                    ptx::mbar_arrive_expect_tx(&sh.bar, (uint32_t)(kWbRows * ncols));
+                    for (int k = 0; k < kWbRows; ++k)
+                        ptx::bulk_g2s(wb_s + k * kLoraSliceCols, wb + (int64_t)(k0 + k) * d_in, (uint32_t)ncols,
+                                      &sh.bar);
+                }
+            }
+            if (!ptx::mbar_wait(&sh.bar, phase)) {
+                if (tid == 0) atomicOr(sa.err, DFSSM_DEVERR_TIMEOUT);
+            }
+            phase ^= 1u;
+            int h[kWbRows];
+#pragma unroll
+            for (int k = 0; k < kWbRows; ++k) h[k] = 0;
+#pragma unroll
+            for (int i = 0; i < kSliceChunks; ++i) {
+                const int j = tid + kSliceThreads * i;
+#pragma unroll
+                for (int k = 0; k < kWbRows; ++k) {
+                    const uint2 w = *reinterpret_cast<const uint2*>(wb_s + k * kLoraSliceCols + 8 * j);
+                    h[k] = __dp4a((int)qv[i][0], (int)w.x, h[k]);
+                    h[k] = __dp4a((int)qv[i][1], (int)w.y, h[k]);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < kWbRows; ++k) {
+                const int v = __reduce_add_sync(0xffffffffu, h[k]);
+                if (lane == k) sh.h[warp][k0 + k] = v;
+            }
         }
         __syncthreads();
         if (tid < kRank) {
@@ -376,7 +416,7 @@ cudaError_t launch_quant(const LaunchCtx& c) {
         for (int i = 0; i < c.n; ++i)
             for (int s = 0; s < lora_slices(c.host_desc[i].d_in); ++s) sa.item[sa.n_items++] = ((uint32_t)i << 8) | (uint32_t)s;
         const int grid = sa.n_items < c.sm_count ? sa.n_items : c.sm_count;
-        const size_t smem = kSliceHead + (size_t)kRank * kLoraSliceCols;
+        const size_t smem = kSliceHead + (size_t)kWbRows * kLoraSliceCols;
         lora_slice_kernel<<<grid, kSliceThreads, smem, c.stream>>>(sa);
         return cudaGetLastError();
     }
