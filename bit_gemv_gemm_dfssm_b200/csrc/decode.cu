@@ -139,7 +139,10 @@ template <int R>
 struct Walk {
     Cursor c;
     Lin L;
-    __device__ __forceinline__ bool valid(const DecodeArgs& a, int64_t hi) const {
+    // with the host's start table a CTA runs up to the next CTA's first block (`end`, packed as
+    // linear << 16 | block); otherwise up to its last work unit `hi`
+    __device__ __forceinline__ bool valid(const DecodeArgs& a, int64_t hi, uint32_t end) const {
+        if (a.has_start) return (((uint32_t)c.l << 16) | (uint32_t)c.b) < end;
         return c.l < a.n && L.work_rel + kDecodeLinStart + (int64_t)c.b * L.bunits < hi;
     }
     __device__ __forceinline__ void advance(const DecodeArgs& a) {
@@ -302,12 +305,13 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
 
     const int64_t lo = a.total_units * blockIdx.x / gridDim.x;
     const int64_t hi = a.total_units * (blockIdx.x + 1) / gridDim.x;
+    const uint32_t end = blockIdx.x + 1 < gridDim.x ? a.start[blockIdx.x + 1] : ((uint32_t)a.n << 16);
     Walk<R> cw, lw;
     if (a.has_start) cw.start_at(a, (int)(a.start[blockIdx.x] >> 16), (int)(a.start[blockIdx.x] & 0xFFFFu));
     else cw.start(a, lo);
     lw = cw;
     // the first linear's activations into L2 ahead of the weight stream (quantised below)
-    if (cw.valid(a, hi) && cw.L.ok) {
+    if (cw.valid(a, hi, end) && cw.L.ok) {
         const char* xp = reinterpret_cast<const char*>(cw.L.x);
         const int xbytes = m * cw.L.d_in * 2;
         for (int off = 16 * tid; off < xbytes; off += 16 * kThreads)
@@ -317,7 +321,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
     // ---- prologue: kStages - 1 slots in flight
 #pragma unroll
     for (int s = 0; s < kStages - 1; ++s) {
-        if (lw.valid(a, hi)) {
+        if (lw.valid(a, hi, end)) {
             issue_step<R>(lw.c, lw.L, ring + s * a.slot_bytes);
             lw.advance(a);
         }
@@ -332,14 +336,14 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
     const int wrow0 = warp * 16 * RT;             // first row of this warp in a block
     const int q_off = (int)(q_s - smem);          // staged q, as an offset into the shared array
 
-    for (int it = 0; cw.valid(a, hi); ++it) {
+    for (int it = 0; cw.valid(a, hi, end); ++it) {
         const Lin& L = cw.L;
         if (cw.c.l != q_lin) {
             // a new linear: quantise its activations (its weights are already streaming)
             if (L.ok) quantise_into_smem(L, m, q_s, ts);
             q_lin = cw.c.l;
         }
-        if (lw.valid(a, hi)) {
+        if (lw.valid(a, hi, end)) {
             issue_step<R>(lw.c, lw.L, ring + ((it + kStages - 1) % kStages) * a.slot_bytes);
             lw.advance(a);
         }
@@ -547,7 +551,8 @@ cudaError_t launch_cfg(const LaunchCtx& c) {
     DecodeArgs a{c.entries, c.single, c.desc, c.n, c.m, c.part, quant_splits(c), use_lora_slices(c) ? 1 : 0,
                  total_units, R == 128 ? 0 : 1,
                  geo.slot_bytes, geo.q_region, 0, {}};
-    // each CTA's first block, as Walk::start finds it on the device
+    // each CTA's first block, as Walk::start finds it on the device; a CTA runs up to the next
+    // CTA's first block
     if (grid <= kStartTable && c.n < 65536) {
         bool fits = true;
         const int ri = R == 128 ? 0 : 1;

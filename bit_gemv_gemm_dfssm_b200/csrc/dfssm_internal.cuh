@@ -115,11 +115,16 @@ constexpr int kLoraMaxSlices = kMaxDIn / kLoraSliceCols;
 constexpr int kMaxSliceItems = 768;
 static_assert(kLoraMaxSlices <= kMaxSplits, "slice partials fit the split partial buffer");
 __host__ __device__ inline int lora_slices(int d_in) { return (d_in + kLoraSliceCols - 1) / kLoraSliceCols; }
-inline bool use_lora_slices(const LaunchCtx& c) {
-    if (c.m != 1) return false;
+inline int lora_slice_items(const LaunchCtx& c) {
     int items = 0;
     for (int i = 0; i < c.n; ++i) items += lora_slices(c.host_desc[i].d_in);
-    return items <= kMaxSliceItems;
+    return items;
+}
+inline bool use_lora_slices(const LaunchCtx& c) { return c.m == 1 && lora_slice_items(c) <= kMaxSliceItems; }
+// CTAs of the slice kernel (one item each while they last, at most one per SM)
+inline int lora_slice_grid(const LaunchCtx& c) {
+    const int items = lora_slice_items(c);
+    return items < c.sm_count ? items : c.sm_count;
 }
 
 cudaError_t launch_pack_sign(const void* src, int src_dtype, int d_out, int d_in, uint8_t* packed,

@@ -415,7 +415,7 @@ cudaError_t launch_quant(const LaunchCtx& c) {
         SliceArgs sa{c.entries, c.single, c.desc, 0, c.part, c.err, {}};
         for (int i = 0; i < c.n; ++i)
             for (int s = 0; s < lora_slices(c.host_desc[i].d_in); ++s) sa.item[sa.n_items++] = ((uint32_t)i << 8) | (uint32_t)s;
-        const int grid = sa.n_items < c.sm_count ? sa.n_items : c.sm_count;
+        const int grid = lora_slice_grid(c);
         const size_t smem = kSliceHead + (size_t)kWbRows * kLoraSliceCols;
         lora_slice_kernel<<<grid, kSliceThreads, smem, c.stream>>>(sa);
         return cudaGetLastError();
