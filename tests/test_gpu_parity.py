@@ -59,6 +59,8 @@ DECODE_CASES = [  # (d_in, d_out, m, y_dtype)
     (128, 1, 1, F32), (128, 17, 3, BF16), (384, 200, 1, F32), (384, 64, 8, BF16),
     (256, 130, 9, F32), (2048, 8512, 1, BF16), (4096, 2048, 1, F32), (4096, 100, 16, BF16),
     (8192, 70, 2, F32), (2048, 333, 16, F32),
+    # one token: four 2048-column LoRA slices; a ragged second slice of 1152 columns
+    (8192, 70, 1, BF16), (3200, 96, 1, F32),
 ]
 PREFILL_CASES = [
     (128, 1, 17, F32), (256, 129, 33, BF16), (384, 300, 300, F32), (2048, 200, 257, BF16),
