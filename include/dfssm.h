@@ -163,8 +163,8 @@ dfssm_status dfssm_linear_stack_fwd(dfssm_plan plan, const dfssm_stack_entry* en
  * No counterpart in the paper: this is for callers that cannot call cudaMalloc
  * (code running while a CUDA graph is being captured, allocators that must not
  * be re-entered, hosts with a fixed memory budget). It needs no plan: its
- * scratch (the quantisation kernel's split partials, descriptor,
- * error word) is a file-scope device array of about 11 KB that every GPU using
+ * scratch (partial LoRA sums h, descriptor, error word) is a file-scope
+ * device array of about 11 KB that every GPU using
  * this library keeps until the process exits.
  * desc: HOST pointer to the linear's shape (rank 16, 128 <= d_in <= 8192,
  * d_in % 128 == 0; max_m is ignored); w: HOST struct of device pointers;
