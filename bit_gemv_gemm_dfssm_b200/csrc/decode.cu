@@ -593,9 +593,18 @@ cudaError_t launch_decode(const LaunchCtx& c) {
     return launch_cfg<1, 2>(c);
 }
 
+// The largest shared-memory carveout: three decode CTAs take 196 KB, and the one-token slice
+// kernel's CTA (34 KB) fits beside them only if the SM is configured for 228 KB.
 cudaError_t set_decode_attr(int optin) {
     cudaError_t e = allow_dyn_smem(decode_kernel<2, 1>, optin);
-    return e != cudaSuccess ? e : allow_dyn_smem(decode_kernel<1, 2>, optin);
+    if (e == cudaSuccess) e = allow_dyn_smem(decode_kernel<1, 2>, optin);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(decode_kernel<2, 1>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(decode_kernel<1, 2>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+    return e;
 }
 
 }  // namespace dfssm
