@@ -243,19 +243,38 @@ def test_single_projection_full(workload):
 @pytest.mark.parametrize("workload,samples", [("stack48_m1", 0), ("stack48_m4", 400), ("stack48_m16", 400),
                                               ("stack48_m64", 300), ("stack48_m2048", 200)])
 def test_stack_full_size(workload, samples):
+    # First the call exactly as bench.py makes it (bf16 y, no debug exports: for M = 2048 this
+    # is the 16-byte row-piece store path of the tcgen05 epilogue), y checked against the
+    # oracle; then the same call with the debug exports, integers checked bit for bit.
     wl = synth.WORKLOADS[workload]
     m = wl["m"]
-    lins, plan, ent = build_stack(wl["shapes"], m, BF16, cfg=wl["cfg"])
-    # weights as the bench draws them
+    lins, plan, ent_dbg = build_stack(wl["shapes"], m, BF16, cfg=wl["cfg"])
+    ent_bench = entries_device([l.entry(i, with_dbg=False) for i, l in enumerate(lins)])
+    stream = torch.cuda.current_stream().cuda_stream
     try:
-        dfssm.dfssm_linear_stack_fwd(plan, ent.data_ptr(), len(lins), m, torch.cuda.current_stream().cuda_stream)
-        st, bits = dfssm.dfssm_plan_check(plan)
-        assert st == dfssm.DFSSM_OK, hex(bits)
-        rng = np.random.default_rng(m)
-        for i, lin in enumerate(lins):
-            if samples == 0:
-                check_linear_full(lin)
-            else:
-                check_linear_sampled(lin, samples, rng)
+        for ent, ints in ((ent_bench, False), (ent_dbg, True)):
+            for lin in lins:
+                lin.dy.fill_(float("nan"))
+            dfssm.dfssm_linear_stack_fwd(plan, ent.data_ptr(), len(lins), m, stream)
+            st, bits = dfssm.dfssm_plan_check(plan)
+            assert st == dfssm.DFSSM_OK, hex(bits)
+            rng = np.random.default_rng(m)
+            for i, lin in enumerate(lins):
+                if samples == 0:
+                    check_linear_full(lin, ints=ints)
+                else:
+                    check_linear_sampled(lin, samples, rng, ints=ints)
     finally:
         dfssm.dfssm_plan_destroy(plan)
+
+
+# bf16 output without debug exports and d_out % 8 == 0: the tcgen05 epilogue stores 16-byte row
+# pieces for whole 32-row groups and single elements for a last partial group; ragged token tiles
+BENCH_STORE_CASES = [(2048, 136, 200), (4096, 520, 400), (1024, 256, 385), (384, 40, 17), (8192, 64, 193)]
+
+
+@pytest.mark.parametrize("d_in,d_out,m", BENCH_STORE_CASES)
+def test_prefill_bf16_store_path(d_in, d_out, m):
+    lin = Linear(SEED, 9, d_in + 7 * d_out + m, d_in, d_out, m, BF16, dbg=False)
+    run_one(lin)
+    check_linear_full(lin)
