@@ -14,10 +14,19 @@
 //    CTA durations follow these units, not bytes (a partial last block costs
 //    as many iterations as a full one, and entering a linear costs a quantisation).
 //  * Streaming: a block is consumed in k-chunks of 1024 columns (128 bytes per
-//    row). A ring of kStages shared-memory slots is filled with 16-byte
-//    cp.async; in slot row r, 16-byte chunk j sits at (j + r) mod 8, so the
-//    ldmatrix reads of 8 rows hit 8 different bank groups. The last k-chunk of
-//    a block also brings its alpha, s_A and W_A.
+//    row), each one TMA load (cp.async.bulk.tensor, no multicast) of an
+//    R x 128-byte box into a ring of kStages shared-memory slots, issued by one
+//    thread; the 128-byte swizzle puts 16-byte piece j of slot row r at
+//    j ^ (r & 7), so the ldmatrix reads of 8 rows hit 8 different bank groups,
+//    and rows past d_out or bytes past the row end arrive as zeros. The last
+//    k-chunk of a block also brings its alpha, s_A and W_A (16-byte cp.async).
+//    A slot's mbarrier completes when the TMA bytes and every thread's
+//    cp.async have landed (cp.async.mbarrier.arrive), so a chunk costs the
+//    computing threads no copy instructions and one CTA barrier. The tensor
+//    map of a single linear is encoded on the host and passed with the launch;
+//    for a stack (pointers in device memory) warp 0 copies the linear's
+//    template map into shared memory, sets its global address
+//    (tensormap.replace) and publishes it to one of the CTA's map slots.
 //  * Activations: when a CTA reaches a new linear it quantises that linear's
 //    x itself (same fp32 arithmetic as the quantisation kernel, so the same
 //    bits) into shared memory, while its weight chunks are already in flight.
@@ -41,6 +50,8 @@
 //  * Epilogue (epilogue.cuh): lane i of a warp takes output row i, gathers its
 //    sums with warp shuffles, and applies the LoRA up-projection and the
 //    dequantisation in the same fp32 order as the prefill path.
+#include <cstring>
+
 #include "dfssm_internal.cuh"
 #include "epilogue.cuh"
 #include "ptx.cuh"
@@ -67,9 +78,17 @@ __host__ __device__ __forceinline__ int q_stride(int d_in) { return ((d_in + 255
 constexpr int kStages = DFSSM_DECODE_STAGES;
 constexpr int kMaxTok = 16;
 
-constexpr int kStartTable = 900;   // CTAs whose start the host supplies (keeps the arguments under 4 KB)
+constexpr int kStartTable = 700;   // CTAs whose start the host supplies (keeps the arguments under 4 KB)
+constexpr int kMapSlots = 4;       // device-edited maps per CTA; >= kStages, so a slot's old loads are done
+constexpr int kMaxCtasPerSm = 8;   // map slots are allocated for this many CTAs per SM
+static_assert(kMapSlots >= kStages, "map slot reuse");
 
 struct DecodeArgs {
+    CUtensorMap single_map;  // sign map of `single` (one linear), encoded on the host
+    const CUtensorMap* tmpl; // stack: per linear, its sign map with a placeholder address
+    CUtensorMap* map_slots;  // stack: kMapSlots per CTA
+    uint64_t wait_limit_ns;
+    int stall_test;          // test hook: CTA 0 waits on a barrier nothing arrives on
     const dfssm_stack_entry* entries;
     dfssm_stack_entry single;
     const DevDesc* desc;     // desc[0] is the first linear of this launch
@@ -86,6 +105,7 @@ struct DecodeArgs {
     // needs no search through the descriptors before its first loads; has_start = 0 when the
     // grid is larger than the table (the CTAs then search themselves)
     int has_start;
+    uint32_t* err;           // the plan's device error word
     uint32_t start[kStartTable];
 };
 
@@ -179,41 +199,58 @@ struct Walk {
     }
 };
 
-// Fill a ring slot with k-chunk kc of block b: R rows x (up to) 128 sign bytes,
-// plus alpha, s_A and W_A of the block when kc is its last chunk.
+// Control block in shared memory.
+struct DecCtl {
+    alignas(128) uint8_t map_s[128];   // tensor map being edited (stack calls)
+    uint64_t full[kStages];            // slot filled: TMA bytes + every thread's cp.async
+    uint64_t never;                    // test hook: nothing arrives on it
+};
+
+// Fill a ring slot with k-chunk kc of block b: R rows x 128 sign bytes by one TMA load (thread 0),
+// plus alpha, s_A and W_A of the block (cp.async, all threads) when kc is its last chunk. Every
+// thread then arrives on the slot's barrier once its own copies have landed.
 template <int R>
-__device__ __forceinline__ void issue_step(const Cursor& c, const Lin& L, uint8_t* slot) {
-    if (!L.ok) return;                    // flagged by the quantisation kernel
+__device__ __forceinline__ void issue_step(const Cursor& c, const Lin& L, uint32_t slot_s, const CUtensorMap* map,
+                                           uint64_t* full) {
     const int row0 = c.b * R;
-    const int nrows = min(R, L.d_out - row0);
-    const int nch = min(kChunkBytes, L.rb - kChunkBytes * c.kc) >> 4;   // 16-byte pieces in this chunk
-    // thread t copies 16-byte piece j = t % kChunkJ of rows r0 + k * kRowStep (r0 = t / kChunkJ),
-    // each to its rotated position (j + r) mod kChunkJ
-    constexpr int kRowStep = kThreads / kChunkJ;
-    static_assert(R % kRowStep == 0, "copy pattern");
-    const int j = threadIdx.x % kChunkJ;
-    const int r0 = threadIdx.x / kChunkJ;
-    if (j < nch) {
-        const uint8_t* s0 = L.sign + (int64_t)(row0 + r0) * L.rb + kChunkBytes * c.kc + 16 * j;
-        const int64_t sstep = (int64_t)kRowStep * L.rb;
-        const uint32_t d0 = ptx::smem_u32(slot) + r0 * kChunkBytes;
-#pragma unroll
-        for (int k = 0; k < R / kRowStep; ++k)
-            if (r0 + k * kRowStep < nrows)
-                ptx::cp_async16_s(d0 + k * kRowStep * kChunkBytes + 16 * ((j + r0 + k * kRowStep) & (kChunkJ - 1)),
-                                  s0 + k * sstep);
-    }
-    if (c.kc == L.nchunks - 1) {
-        uint8_t* par = slot + R * kChunkBytes;
-        const int n4 = (nrows + 3) >> 2;
-        for (int i = threadIdx.x; i < n4; i += kThreads) {
-            const uint32_t bytes = (uint32_t)min(16, 4 * (nrows - 4 * i));
-            ptx::cp_async16_zfill(par + 16 * i, L.alpha + row0 + 4 * i, bytes);
-            ptx::cp_async16_zfill(par + 4 * R + 16 * i, L.sa + row0 + 4 * i, bytes);
+    if (L.ok) {
+        if (threadIdx.x == 0) {
+            ptx::mbar_arrive_expect_tx(full, (uint32_t)(R * kChunkBytes));
+            ptx::tma_load_2d_s(slot_s, map, kChunkBytes * c.kc, row0, full);
         }
-        for (int r = threadIdx.x; r < nrows; r += kThreads)
-            ptx::cp_async16(par + 8 * R + 16 * r, L.wa + (int64_t)(row0 + r) * kRank);
+        if (c.kc == L.nchunks - 1) {
+            const int nrows = min(R, L.d_out - row0);
+            const uint32_t par = slot_s + R * kChunkBytes;
+            const int n4 = (nrows + 3) >> 2;
+            for (int i = threadIdx.x; i < n4; i += kThreads) {
+                const uint32_t bytes = (uint32_t)min(16, 4 * (nrows - 4 * i));
+                ptx::cp_async16_zfill_s(par + 16 * i, L.alpha + row0 + 4 * i, bytes);
+                ptx::cp_async16_zfill_s(par + 4 * R + 16 * i, L.sa + row0 + 4 * i, bytes);
+            }
+            for (int r = threadIdx.x; r < nrows; r += kThreads)
+                ptx::cp_async16_s(par + 8 * R + 16 * r, L.wa + (int64_t)(row0 + r) * kRank);
+        }
+    } else if (threadIdx.x == 0) {
+        ptx::mbar_arrive(full);        // bad entry (flagged by the quantisation kernel): nothing is read
     }
+    ptx::cp_async_mbar_arrive_noinc(full);
+}
+
+// The sign map for linear l: the launch's own map (one linear), or this CTA's next map slot
+// with the linear's template and its sign address (all 32 lanes of warp 0 call this).
+__device__ __forceinline__ const CUtensorMap* linear_map(const DecodeArgs& a, const Lin& L, int l, int& nmap,
+                                                        DecCtl& dc) {
+    if (a.entries == nullptr || !L.ok) return &a.single_map;
+    const int lane = threadIdx.x & 31;
+    CUtensorMap* ms = a.map_slots + (size_t)blockIdx.x * kMapSlots + (nmap++ % kMapSlots);
+    if (lane < 8) reinterpret_cast<uint4*>(dc.map_s)[lane] = reinterpret_cast<const uint4*>(a.tmpl + l)[lane];
+    __syncwarp();
+    if (lane == 0) ptx::tensormap_replace_addr(dc.map_s, L.sign);
+    __syncwarp();
+    ptx::tensormap_copy_release(ms, dc.map_s);
+    if (lane == 0) ptx::tensormap_acquire(ms);
+    __syncwarp();
+    return ms;
 }
 
 // Shared-memory position of q for column 32 gg + 8 i + p of a token row (gg: 32-column
@@ -294,18 +331,37 @@ __device__ void quantise_into_smem(const Lin& L, int m, uint8_t* q_s, TokShared&
 template <int RT, int NT>
 __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant__ DecodeArgs a) {
     constexpr int R = 16 * RT * kWarps;
-    extern __shared__ __align__(128) uint8_t smem[];
-    TokShared& ts = *reinterpret_cast<TokShared*>(smem);
-    uint8_t* q_s = smem + ((sizeof(TokShared) + 127) & ~(size_t)127);
-    uint8_t* ring = q_s + a.q_region;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    // 1024-byte aligned ring first (the 128-byte swizzle of the TMA boxes repeats every 1 KB)
+    uint8_t* ring = smem + ((1024u - (ptx::smem_u32(smem) & 1023u)) & 1023u);
+    uint8_t* q_s = ring + kStages * a.slot_bytes;
+    TokShared& ts = *reinterpret_cast<TokShared*>(q_s + a.q_region);
+    DecCtl& dc = *reinterpret_cast<DecCtl*>(q_s + a.q_region + ((sizeof(TokShared) + 127) & ~(size_t)127));
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, c = lane & 3;
     const int m = a.m;
+    const uint64_t lim = a.wait_limit_ns;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) ptx::mbar_init(&dc.full[s], 1 + kThreads);
+        ptx::mbar_init(&dc.never, 1);
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    if (a.stall_test && blockIdx.x == 0) {
+        // test hook: a wait that nothing ends; every thread gives up after the limit, the CTA
+        // reports DFSSM_DEVERR_TIMEOUT and stops before issuing anything
+        const bool ok = ptx::mbar_wait(&dc.never, 0u, lim);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) atomicOr(a.err, DFSSM_DEVERR_TIMEOUT);
+            return;
+        }
+    }
 
     const int64_t lo = a.total_units * blockIdx.x / gridDim.x;
     const int64_t hi = a.total_units * (blockIdx.x + 1) / gridDim.x;
-    const uint32_t end = blockIdx.x + 1 < gridDim.x ? a.start[blockIdx.x + 1] : ((uint32_t)a.n << 16);
+    const uint32_t end = a.has_start && blockIdx.x + 1 < gridDim.x ? a.start[blockIdx.x + 1] : ((uint32_t)a.n << 16);
     Walk<R> cw, lw;
     if (a.has_start) cw.start_at(a, (int)(a.start[blockIdx.x] >> 16), (int)(a.start[blockIdx.x] & 0xFFFFu));
     else cw.start(a, lo);
@@ -318,15 +374,27 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
             asm volatile("prefetch.global.L2 [%0];" ::"l"(xp + off));
     }
 
-    // ---- prologue: kStages - 1 slots in flight
+    // ---- prologue: kStages - 1 slots in flight (warp 0 keeps the sign map of the look-ahead
+    // cursor's linear; thread 0 issues the TMA loads)
+    const CUtensorMap* map = &a.single_map;
+    int map_lin = -1, nmap = 0;
+    auto issue = [&](int slot) {
+        if (warp == 0 && lw.c.l != map_lin) {
+            map = linear_map(a, lw.L, lw.c.l, nmap, dc);
+            map_lin = lw.c.l;
+        }
+        issue_step<R>(lw.c, lw.L, ptx::smem_u32(ring + slot * a.slot_bytes), map, &dc.full[slot]);
+        lw.advance(a);
+    };
+    int issued = 0;
 #pragma unroll
     for (int s = 0; s < kStages - 1; ++s) {
         if (lw.valid(a, hi, end)) {
-            issue_step<R>(lw.c, lw.L, ring + s * a.slot_bytes);
-            lw.advance(a);
+            issue(s);
+            ++issued;
         }
-        ptx::cp_async_commit();
     }
+    bool failed = false;
 
     int D[RT][NT][8][4];
     int q_lin = -1, u_lin = -1;
@@ -342,13 +410,14 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
             // a new linear: quantise its activations (its weights are already streaming)
             if (L.ok) quantise_into_smem(L, m, q_s, ts);
             q_lin = cw.c.l;
+            __syncthreads();
         }
         if (lw.valid(a, hi, end)) {
-            issue_step<R>(lw.c, lw.L, ring + ((it + kStages - 1) % kStages) * a.slot_bytes);
-            lw.advance(a);
+            issue((it + kStages - 1) % kStages);
+            ++issued;
         }
-        ptx::cp_async_commit();
-        ptx::cp_async_wait<kStages - 1>();
+        // this chunk's slot: TMA bytes and every thread's cp.async landed
+        if (!ptx::mbar_wait(&dc.full[it % kStages], (uint32_t)((it / kStages) & 1), lim)) failed = true;
         const bool last_chunk = cw.c.kc == L.nchunks - 1;
         if (last_chunk && u_lin != cw.c.l) {
             // the LoRA vector u = s_B * h of this linear: h is the sum, in split order, of the
@@ -364,8 +433,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
                 if (L.dbg_h) L.dbg_h[(int64_t)t * kRank + k] = h;
             }
             u_lin = cw.c.l;
+            __syncthreads();
         }
-        __syncthreads();
 
         const uint8_t* slot = ring + (it % kStages) * a.slot_bytes;
         const int row0 = cw.c.b * R;
@@ -385,15 +454,15 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
             const int qstride = q_stride(L.d_in);
             const int cb = min(kChunkBytes, L.rb - kChunkBytes * cw.c.kc);
             const uint32_t slot_s = ptx::smem_u32(slot);
-            // ldmatrix row addresses: row r's 16-byte piece j sits at (j + r) mod kChunkJ; rows
-            // of a tile start at multiples of 16, so the rotation depends on the lane only
-            const int rot = (lm_row & (kChunkJ - 1)) + lm_hi;
+            // ldmatrix row addresses: the TMA's 128-byte swizzle puts row r's 16-byte piece j at
+            // j ^ (r & 7); rows of a tile start at multiples of 16, so the XOR depends on the lane only
+            const int sw = lm_row & 7;
             uint32_t a_addr[RT][kGroups];
 #pragma unroll
             for (int rt = 0; rt < RT; ++rt)
 #pragma unroll
                 for (int G = 0; G < kGroups; ++G)
-                    a_addr[rt][G] = slot_s + (wrow0 + 16 * rt + lm_row) * kChunkBytes + 16 * ((2 * G + rot) % kChunkJ);
+                    a_addr[rt][G] = slot_s + (wrow0 + 16 * rt + lm_row) * kChunkBytes + 16 * ((2 * G + lm_hi) ^ sw);
             // B rows: tokens nt * 8 + g; lanes past m read token 0 (their MMA columns are never stored)
             // (32-bit offsets into the shared array, so the loads need no 64-bit address math)
             int qk[NT][4];
@@ -508,7 +577,15 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
                 }
             }
         }
-        __syncthreads();     // slot it % kStages is refilled by the next iteration
+        // slot it % kStages is refilled by the next iteration; a wait that gave up ends the CTA
+        if (__syncthreads_or(failed)) {
+            if (tid == 0) {
+                atomicOr(a.err, DFSSM_DEVERR_TIMEOUT);
+                // let the loads still in flight into this CTA's shared memory land (bounded)
+                for (int j = it; j < issued; ++j) ptx::mbar_wait(&dc.full[j % kStages], (uint32_t)((j / kStages) & 1), lim);
+            }
+            break;
+        }
         cw.advance(a);
     }
     ptx::cp_async_wait<0>();
@@ -519,13 +596,17 @@ struct Geometry {
     size_t smem;
 };
 
+// Ring slots of R x 128 sign bytes + the block's alpha, s_A, W_A, each a multiple of 1 KB (the
+// TMA swizzle pattern repeats every 1 KB); then the staged q, the per-token values and the
+// control block; 1 KB for aligning the base.
 template <int RT>
 Geometry geometry(int m, int max_d_in) {
     constexpr int R = 16 * RT * kWarps;
     Geometry g;
-    g.slot_bytes = (R * kChunkBytes + R * (4 + 4 + kRank) + 127) & ~127;
+    g.slot_bytes = (R * kChunkBytes + R * (4 + 4 + kRank) + 1023) & ~1023;
     g.q_region = (m * q_stride(max_d_in) + 127) & ~127;
-    g.smem = ((sizeof(TokShared) + 127) & ~(size_t)127) + g.q_region + (size_t)kStages * g.slot_bytes;
+    g.smem = 1024 + (size_t)kStages * g.slot_bytes + g.q_region + ((sizeof(TokShared) + 127) & ~(size_t)127) +
+             sizeof(DecCtl);
     return g;
 }
 
@@ -546,11 +627,35 @@ cudaError_t launch_cfg(const LaunchCtx& c) {
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<RT, NT>, kThreads, geo.smem);
     if (err != cudaSuccess) return err;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    if (per_sm > kMaxCtasPerSm) per_sm = kMaxCtasPerSm;     // the plan's map slots
     int grid = c.sm_count * per_sm;
     if (grid > blocks) grid = blocks;
-    DecodeArgs a{c.entries, c.single, c.desc, c.n, c.m, c.part, quant_splits(c), use_lora_slices(c) ? 1 : 0,
-                 total_units, R == 128 ? 0 : 1,
-                 geo.slot_bytes, geo.q_region, 0, {}};
+    DecodeArgs a;
+    std::memset(&a.single_map, 0, sizeof(a.single_map));
+    if (c.entries == nullptr) {
+        if (!encode_sign_map(&a.single_map, c.single.w.sign, c.host_desc[0].d_in, c.host_desc[0].d_out, R))
+            return cudaErrorInvalidValue;
+    } else if (c.sign_tmpl == nullptr || c.map_slots == nullptr) {
+        return cudaErrorInvalidValue;
+    }
+    a.tmpl = reinterpret_cast<const CUtensorMap*>(c.sign_tmpl) + (R == 128 ? 0 : c.tmpl_stride);
+    a.map_slots = reinterpret_cast<CUtensorMap*>(c.map_slots);
+    a.wait_limit_ns = c.wait_limit_ns;
+    a.stall_test = c.stall_test;
+    a.entries = c.entries;
+    a.single = c.single;
+    a.desc = c.desc;
+    a.n = c.n;
+    a.m = c.m;
+    a.part = c.part;
+    a.splits = quant_splits(c);
+    a.slices = use_lora_slices(c) ? 1 : 0;
+    a.total_units = total_units;
+    a.ri = R == 128 ? 0 : 1;
+    a.slot_bytes = geo.slot_bytes;
+    a.q_region = geo.q_region;
+    a.has_start = 0;
+    a.err = c.err;
     // each CTA's first block, as Walk::start finds it on the device; a CTA runs up to the next
     // CTA's first block
     if (grid <= kStartTable && c.n < 65536) {
@@ -593,7 +698,25 @@ cudaError_t launch_decode(const LaunchCtx& c) {
     return launch_cfg<1, 2>(c);
 }
 
-// The largest shared-memory carveout: three decode CTAs take 196 KB, and the one-token slice
+// The decode kernel's tensor map over a linear's sign rows: d_out rows of d_in / 8 bytes, boxes of
+// 128 bytes x `rows` (the block rows), 128-byte swizzle, zeros outside the matrix.
+bool encode_sign_map(CUtensorMap* map, const void* sign, int d_in, int d_out, int rows) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return false;
+    const int rb = d_in / 8;
+    cuuint64_t dims[2] = {(cuuint64_t)rb, (cuuint64_t)d_out};
+    cuuint64_t strides[1] = {(cuuint64_t)rb};
+    cuuint32_t box[2] = {(cuuint32_t)kChunkBytes, (cuuint32_t)rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(sign), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int decode_map_slots_per_sm() { return kMapSlots * kMaxCtasPerSm; }
+int decode_block_rows(int m) { return m <= 8 ? 128 : 64; }
+
+// The largest shared-memory carveout: three decode CTAs take about 196 KB, and the one-token slice
 // kernel's CTA (34 KB) fits beside them only if the SM is configured for 228 KB.
 cudaError_t set_decode_attr(int optin) {
     cudaError_t e = allow_dyn_smem(decode_kernel<2, 1>, optin);

@@ -48,6 +48,10 @@ struct dfssm_plan_s {
     uint32_t* err = nullptr;
     int* part = nullptr;
     CUtensorMap* tmaps = nullptr;       // prefill: activation rows of each linear
+    CUtensorMap* sign_tmpl = nullptr;   // decode: sign rows of each linear (placeholder address), 128- then 64-row boxes
+    CUtensorMap* map_slots = nullptr;   // decode: per-CTA slots for the device-edited sign maps
+    uint64_t wait_limit_ns = kWaitLimitNs;
+    int stall_test = 0;
     size_t ws_bytes = 0;
 };
 
@@ -103,6 +107,8 @@ void free_plan(dfssm_plan_s* p) {
     if (p->err) cudaFree(p->err);
     if (p->part) cudaFree(p->part);
     if (p->tmaps) cudaFree(p->tmaps);
+    if (p->sign_tmpl) cudaFree(p->sign_tmpl);
+    if (p->map_slots) cudaFree(p->map_slots);
     delete p;
 }
 
@@ -178,6 +184,9 @@ dfssm_status dfssm_linear_plan(const dfssm_linear_desc* descs, int n_descs, dfss
     if (e == cudaSuccess) e = cudaMalloc(&p->st_ws, sizeof(TokStats) * (size_t)st_count);
     if (e == cudaSuccess) e = cudaMalloc(&p->err, 16);
     if (e == cudaSuccess) e = cudaMalloc(&p->tmaps, sizeof(CUtensorMap) * n_descs);
+    const size_t n_slots = (size_t)p->sm_count * decode_map_slots_per_sm();
+    if (e == cudaSuccess) e = cudaMalloc(&p->sign_tmpl, sizeof(CUtensorMap) * 2 * n_descs);
+    if (e == cudaSuccess) e = cudaMalloc(&p->map_slots, sizeof(CUtensorMap) * n_slots);
     const size_t part_bytes = sizeof(int) * (size_t)n_descs * kMaxSplits * kPartTok * 20;
     if (e == cudaSuccess) e = cudaMalloc(&p->part, part_bytes);
     if (e != cudaSuccess) {
@@ -186,7 +195,7 @@ dfssm_status dfssm_linear_plan(const dfssm_linear_desc* descs, int n_descs, dfss
         return e == cudaErrorMemoryAllocation ? DFSSM_ERR_NO_MEMORY : DFSSM_ERR_CUDA;
     }
     p->ws_bytes = sizeof(DevDesc) * n_descs + (size_t)q_bytes + sizeof(TokStats) * st_count + 16 +
-                  sizeof(CUtensorMap) * n_descs + part_bytes + sizeof(unsigned int) * n_descs;
+                  sizeof(CUtensorMap) * (3 * (size_t)n_descs + n_slots) + part_bytes;
 
     // prefill: tensor maps over each linear's activation rows (B operand, 128-byte swizzle)
     std::vector<CUtensorMap> tm(n_descs);
@@ -206,7 +215,18 @@ dfssm_status dfssm_linear_plan(const dfssm_linear_desc* descs, int n_descs, dfss
             if (r != CUDA_SUCCESS) { free_plan(p); return DFSSM_ERR_CUDA; }
         }
     }
+    // decode: each linear's sign map with a placeholder address (set per call on the device), for
+    // the block rows of up to 8 tokens (first n) and of more (next n)
+    std::vector<CUtensorMap> st(2 * (size_t)n_descs);
+    for (int h = 0; h < 2; ++h)
+        for (int i = 0; i < n_descs; ++i)
+            if (!encode_sign_map(&st[(size_t)h * n_descs + i], p->ddesc, p->hdesc[i].d_in, p->hdesc[i].d_out,
+                                 decode_block_rows(h == 0 ? 1 : kDecodeMaxM))) {
+                free_plan(p);
+                return DFSSM_ERR_CUDA;
+            }
     e = cudaMemcpy(p->tmaps, tm.data(), sizeof(CUtensorMap) * n_descs, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(p->sign_tmpl, st.data(), sizeof(CUtensorMap) * 2 * n_descs, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(p->ddesc, p->hdesc.data(), sizeof(DevDesc) * n_descs, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemset(p->err, 0, 16);
     if (e == cudaSuccess) e = set_kernel_attributes(optin);
@@ -266,6 +286,8 @@ dfssm_status dfssm_linear_fwd(dfssm_plan plan, int32_t desc_index, const dfssm_l
     c.err = plan->err;
     c.part = plan->part + (size_t)desc_index * kMaxSplits * kPartTok * 20;
     c.tmaps = plan->tmaps + desc_index;
+    c.wait_limit_ns = plan->wait_limit_ns;
+    c.stall_test = plan->stall_test;
     c.max_d_in = hd.d_in;
     c.total_rows = hd.d_out;
     c.sm_count = plan->sm_count;
@@ -298,6 +320,11 @@ dfssm_status dfssm_linear_stack_fwd(dfssm_plan plan, const dfssm_stack_entry* en
     c.err = plan->err;
     c.part = plan->part;
     c.tmaps = plan->tmaps;
+    c.sign_tmpl = plan->sign_tmpl;
+    c.tmpl_stride = plan->n;
+    c.map_slots = plan->map_slots;
+    c.wait_limit_ns = plan->wait_limit_ns;
+    c.stall_test = plan->stall_test;
     c.max_d_in = max_d_in;
     c.total_rows = rows;
     c.sm_count = plan->sm_count;

@@ -98,11 +98,19 @@ struct LaunchCtx {
     uint32_t* err;
     int* part;                         // split partials: n x kMaxSplits x 16 tokens x 20 ints
     const void* tmaps;                 // device array of CUtensorMap (prefill activation rows), one per desc
+    const void* sign_tmpl;             // device CUtensorMap templates of the decode sign rows (stack calls):
+                                       // [0, tmpl_stride) for 128-row blocks, [tmpl_stride, 2 tmpl_stride) for 64
+    int tmpl_stride;
+    void* map_slots;                   // device CUtensorMap slots edited by the decode CTAs (stack calls)
     int max_d_in;                      // largest d_in among the n linears
     int64_t total_rows;                // sum of d_out over the n linears
     int sm_count;
+    uint64_t wait_limit_ns;            // bound of every in-kernel wait of the decode kernel
+    int stall_test;                    // test hook of the decode kernel (0 in normal use)
     cudaStream_t stream;
 };
+
+constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s
 
 // One token: the LoRA down-projection h = W_B q runs as (linear, slice) items of
 // kLoraSliceCols columns in a kernel small enough to share the SMs with the decode kernel;
@@ -132,6 +140,9 @@ cudaError_t launch_pack_sign(const void* src, int src_dtype, int d_out, int d_in
 cudaError_t launch_quant(const LaunchCtx& c);
 int quant_splits(const LaunchCtx& c);   // d_in splits of the m <= 16 quantisation kernel
 cudaError_t launch_decode(const LaunchCtx& c);
+bool encode_sign_map(CUtensorMap* map, const void* sign, int d_in, int d_out, int rows);   // decode sign rows
+int decode_map_slots_per_sm();                                                             // map slots the plan keeps per SM
+int decode_block_rows(int m);                                                              // decode block rows for m tokens
 cudaError_t launch_prefill(const LaunchCtx& c);
 
 // ---- tensor maps (host side) ----------------------------------------------------------

@@ -120,6 +120,7 @@ extern "C" dfssm_status dfssm_linear_fwd_noalloc(const dfssm_linear_desc* desc, 
     c.err = reinterpret_cast<uint32_t*>(s->scratch + kOffErr);
     c.part = reinterpret_cast<int*>(s->scratch + kOffPart);
     c.tmaps = nullptr;
+    c.wait_limit_ns = kWaitLimitNs;
     c.max_d_in = desc->d_in;
     c.total_rows = desc->d_out;
     c.sm_count = s->sm_count;
