@@ -7,7 +7,8 @@ the library is missing, the first call raises ImportError.
 
 The entry points keep the C names: ``dfssm_linear_plan``, ``dfssm_plan_destroy``,
 ``dfssm_pack_sign``, ``dfssm_linear_fwd``, ``dfssm_linear_stack_fwd``,
-``dfssm_plan_check``, ``dfssm_plan_workspace_bytes``, ``dfssm_status_string``.
+``dfssm_plan_check``, ``dfssm_plan_workspace_bytes``, ``dfssm_status_string``,
+``dfssm_linear_fwd_noalloc``, ``dfssm_plan_set_test_hooks``.
 """
 from __future__ import annotations
 
@@ -39,8 +40,9 @@ RANK = 16
 EXPORTS = (
     "dfssm_linear_plan", "dfssm_plan_destroy", "dfssm_pack_sign", "dfssm_linear_fwd",
     "dfssm_linear_stack_fwd", "dfssm_plan_check", "dfssm_plan_workspace_bytes", "dfssm_status_string",
-    "dfssm_linear_fwd_noalloc",
+    "dfssm_linear_fwd_noalloc", "dfssm_plan_set_test_hooks",
 )
+DFSSM_TEST_STALL = 0x1
 DFSSM_NOALLOC_MAX_M = 16
 
 
@@ -89,6 +91,7 @@ def _load():
                                              vp, vp]
     lib.dfssm_plan_check.argtypes = [vp, u32p]
     lib.dfssm_plan_workspace_bytes.argtypes = [vp, ctypes.POINTER(ctypes.c_size_t)]
+    lib.dfssm_plan_set_test_hooks.argtypes = [vp, ctypes.c_uint64, ctypes.c_uint32]
     lib.dfssm_status_string.restype = ctypes.c_char_p
     lib.dfssm_status_string.argtypes = [ctypes.c_int]
     for name in EXPORTS:
@@ -164,6 +167,11 @@ def dfssm_plan_check(plan: int):
     if st not in (DFSSM_OK, DFSSM_ERR_DEVICE_CHECK):
         raise DfssmError(st, "dfssm_plan_check")
     return st, bits.value
+
+
+def dfssm_plan_set_test_hooks(plan: int, wait_limit_ns: int = 0, flags: int = 0) -> None:
+    """Error-path test hooks of the decode kernel (see include/dfssm.h)."""
+    _check(lib().dfssm_plan_set_test_hooks(plan, wait_limit_ns, flags), "dfssm_plan_set_test_hooks")
 
 
 def dfssm_plan_workspace_bytes(plan: int) -> int:

@@ -344,6 +344,13 @@ dfssm_status dfssm_plan_check(dfssm_plan plan, uint32_t* bits) {
     return v ? DFSSM_ERR_DEVICE_CHECK : DFSSM_OK;
 }
 
+dfssm_status dfssm_plan_set_test_hooks(dfssm_plan plan, uint64_t wait_limit_ns, uint32_t flags) {
+    if (!plan || (flags & ~DFSSM_TEST_STALL) != 0) return DFSSM_ERR_INVALID_ARG;
+    plan->wait_limit_ns = wait_limit_ns ? wait_limit_ns : kWaitLimitNs;
+    plan->stall_test = (flags & DFSSM_TEST_STALL) ? 1 : 0;
+    return DFSSM_OK;
+}
+
 dfssm_status dfssm_plan_workspace_bytes(dfssm_plan plan, size_t* bytes) {
     if (!plan || !bytes) return DFSSM_ERR_INVALID_ARG;
     *bytes = plan->ws_bytes;

@@ -1,19 +1,23 @@
 // dfssm_linear_fwd_noalloc: the layer for one linear and a few tokens without
 // any device allocation.
 //
-// Some callers cannot call cudaMalloc: code that runs inside a CUDA graph being
-// captured, allocators that must not be re-entered, or embedders whose memory
-// budget is fixed up front. This entry point needs no plan: the quantisation
-// and decode kernels run exactly as for dfssm_linear_fwd, with their scratch
-// (the quantisation kernel's split partials, the linear's descriptor and the
-// error word) in the file-scope device array
-// below, which every GPU that loads this library keeps until the process exits.
+// Some callers cannot call cudaMalloc: an embedder whose device allocator must
+// not be re-entered from inside the layer, or a host that fixes its device
+// memory budget up front. This entry point needs no plan: the quantisation and
+// decode kernels run exactly as for dfssm_linear_fwd, with their scratch (the
+// quantisation kernel's split partials, the linear's descriptor and the error
+// word) in the file-scope device array below, which every GPU that loads this
+// library keeps until the process exits. The descriptor is written into the
+// array by a one-thread kernel that receives it by value, so no host buffer has
+// to outlive the call.
 //
 // Limits: 1 <= m <= DFSSM_NOALLOC_MAX_M (16) tokens, 128 <= d_in <= 8192.
 // Every call shares the array; calls that overlap on the GPU (different streams
 // without ordering) race on it. The first call on a device looks up the array's
 // device address (cudaGetSymbolAddress) and sets the kernels' shared-memory
-// limits; make that first call before any stream capture.
+// limits; make that first call before any stream capture. That set-up is kept
+// for the life of the process, so cudaDeviceReset is not supported while this
+// entry point is in use.
 #include <cstring>
 #include <mutex>
 
@@ -69,6 +73,9 @@ dfssm_status setup_device(int dev, DeviceSetup** out) {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// the linear's descriptor into the scratch (kernel arguments are passed by value)
+__global__ void noalloc_set_desc(DevDesc* dst, const DevDesc v) { *dst = v; }
+
 }  // namespace
 }  // namespace dfssm
 
@@ -101,9 +108,8 @@ extern "C" dfssm_status dfssm_linear_fwd_noalloc(const dfssm_linear_desc* desc, 
     hd.max_m = kNoAllocMaxM;
     hd.qrow = seg_qrow(desc->d_in);
     DevDesc* ddesc = reinterpret_cast<DevDesc*>(s->scratch + kOffDesc);
-    // the descriptor goes into the scratch on the stream (a small host-to-device copy, no allocation)
-    if (cudaMemcpyAsync(ddesc, &hd, sizeof(hd), cudaMemcpyHostToDevice, (cudaStream_t)stream) != cudaSuccess)
-        return DFSSM_ERR_CUDA;
+    noalloc_set_desc<<<1, 1, 0, (cudaStream_t)stream>>>(ddesc, hd);
+    if (cudaGetLastError() != cudaSuccess) return DFSSM_ERR_CUDA;
 
     LaunchCtx c{};
     c.entries = nullptr;

@@ -160,12 +160,13 @@ dfssm_status dfssm_linear_stack_fwd(dfssm_plan plan, const dfssm_stack_entry* en
                                     int32_t n_entries, int32_t m, void* stream);
 
 /* The layer for one linear and a few tokens, allocating nothing.
- * No counterpart in the paper: this is for callers that cannot call cudaMalloc
- * (code running while a CUDA graph is being captured, allocators that must not
- * be re-entered, hosts with a fixed memory budget). It needs no plan: its
- * scratch (partial LoRA sums h, descriptor, error word) is a file-scope
- * device array of about 11 KB that every GPU using
- * this library keeps until the process exits.
+ * No counterpart in the paper: this is for callers that cannot call cudaMalloc,
+ * such as an embedder whose device allocator must not be re-entered from inside
+ * the layer, or a host that fixes its device memory budget up front. It needs no
+ * plan: its scratch (partial LoRA sums h, descriptor, error word) is a
+ * file-scope device array of about 11 KB that every GPU using this library keeps
+ * until the process exits; the descriptor is written there by a one-thread
+ * kernel that receives it by value, so no host buffer outlives the call.
  * desc: HOST pointer to the linear's shape (rank 16, 128 <= d_in <= 8192,
  * d_in % 128 == 0; max_m is ignored); w: HOST struct of device pointers;
  * x: m x d_in bf16 (device); y: m x d_out of desc->y_dtype (device);
@@ -174,8 +175,10 @@ dfssm_status dfssm_linear_stack_fwd(dfssm_plan plan, const dfssm_stack_entry* en
  * array, so calls that overlap on the GPU (unordered streams) race; the array
  * keeps the last call's contents, and what must start at zero is reset by the
  * kernels themselves. The first call on each device looks up the array's device
- * address and sets kernel attributes: make it before any stream capture.
- * Device-side error conditions are not reported by this entry point. */
+ * address and sets kernel attributes: make it before any stream capture. That
+ * set-up lasts for the process, so cudaDeviceReset is not supported while this
+ * entry point is in use. Device-side error conditions are not reported by this
+ * entry point. */
 #define DFSSM_NOALLOC_MAX_M 16
 dfssm_status dfssm_linear_fwd_noalloc(const dfssm_linear_desc* desc, const dfssm_linear_weights* w,
                                       const void* x, int32_t m, void* y, void* stream);
@@ -183,6 +186,18 @@ dfssm_status dfssm_linear_fwd_noalloc(const dfssm_linear_desc* desc, const dfssm
 /* Synchronise the plan's device, read and clear its error word.
  * Returns DFSSM_OK or DFSSM_ERR_DEVICE_CHECK (*bits, if not NULL, gets the word). */
 dfssm_status dfssm_plan_check(dfssm_plan plan, uint32_t* bits);
+
+/* Test of the error path of the decode kernel (m <= 16 tokens), which must end with an
+ * error status and never hang. With flags & DFSSM_TEST_STALL, the first CTA of that
+ * kernel waits on a barrier that nothing arrives on: the wait gives up after
+ * wait_limit_ns, the CTA stops before reading or writing anything, and the plan's
+ * device error word gets DFSSM_DEVERR_TIMEOUT (the other CTAs run as usual, so the
+ * outputs of the first CTA's rows are undefined). wait_limit_ns also bounds every
+ * other wait of that kernel; 0 means the default (1 s). flags = 0 turns the stall off.
+ * Takes effect for later calls on this plan; returns DFSSM_ERR_INVALID_ARG for unknown
+ * flags. */
+#define DFSSM_TEST_STALL 0x1u
+dfssm_status dfssm_plan_set_test_hooks(dfssm_plan plan, uint64_t wait_limit_ns, uint32_t flags);
 
 /* Bytes of device workspace the plan holds. */
 dfssm_status dfssm_plan_workspace_bytes(dfssm_plan plan, size_t* bytes);

@@ -190,6 +190,51 @@ def test_nonfinite_activation_row_sets_error_word(m):
     check_y(lin.y_host()[keep], ref["y"], term_bound(ref, lin.w), F32)
 
 
+def test_bounded_wait_gives_up_with_timeout_status():
+    # the decode kernel's first CTA waits on a barrier nothing arrives on: the bounded wait gives
+    # up after 2 ms, the call reports DFSSM_DEVERR_TIMEOUT instead of hanging, and the same plan
+    # computes correctly afterwards
+    shapes = [(2048, 640), (4096, 256)]
+    lins, plan, ent = build_stack(shapes, 1, F32)
+    stream = torch.cuda.current_stream().cuda_stream
+    try:
+        dfssm.dfssm_plan_set_test_hooks(plan, 2_000_000, dfssm.DFSSM_TEST_STALL)
+        dfssm.dfssm_linear_stack_fwd(plan, ent.data_ptr(), len(lins), 1, stream)
+        st, bits = dfssm.dfssm_plan_check(plan)
+        assert st == dfssm.DFSSM_ERR_DEVICE_CHECK and bits & dfssm.DFSSM_DEVERR_TIMEOUT, hex(bits)
+        dfssm.dfssm_plan_set_test_hooks(plan, 0, 0)
+        dfssm.dfssm_linear_stack_fwd(plan, ent.data_ptr(), len(lins), 1, stream)
+        st, bits = dfssm.dfssm_plan_check(plan)
+        assert st == dfssm.DFSSM_OK, hex(bits)
+        for lin in lins:
+            check_linear_full(lin)
+        with pytest.raises(dfssm.DfssmError):
+            dfssm.dfssm_plan_set_test_hooks(plan, 0, 0x80)
+    finally:
+        dfssm.dfssm_plan_destroy(plan)
+
+
+@pytest.mark.parametrize("m", [1, 3])
+def test_nonfinite_one_token_paths(m):
+    # a NaN in one token's row: the slice kernel (one token) and the split quantiser both report
+    # it; for m = 3 the other tokens still match the oracle
+    d_in, d_out = 4096, 200
+    x = synth.activations(SEED, 9, 21, m, d_in).copy()
+    x[0, 100] = 0x7FC0                                # NaN
+    lin = Linear(SEED, 9, 21, d_in, d_out, m, F32, x=x, dbg=False)
+    plan = dfssm.dfssm_linear_plan([lin.desc()])
+    try:
+        stream = torch.cuda.current_stream().cuda_stream
+        dfssm.dfssm_linear_fwd(plan, 0, lin.weights(), lin.dx.data_ptr(), m, lin.dy.data_ptr(), None, stream)
+        st, bits = dfssm.dfssm_plan_check(plan)
+        assert st == dfssm.DFSSM_ERR_DEVICE_CHECK and bits & dfssm.DFSSM_DEVERR_NONFINITE, hex(bits)
+    finally:
+        dfssm.dfssm_plan_destroy(plan)
+    if m > 1:
+        ref = oracle.linear(np.ascontiguousarray(x[1:]), lin.w, m - 1, d_in, d_out)
+        check_y(lin.y_host()[1:], ref["y"], term_bound(ref, lin.w), F32)
+
+
 def test_argument_errors_launch_nothing():
     lin = Linear(SEED, 9, 1, 256, 64, 4, F32)
     plan = dfssm.dfssm_linear_plan([lin.desc()])

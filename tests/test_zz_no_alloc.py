@@ -1,30 +1,33 @@
 """dfssm_linear_fwd_noalloc: the entry point that allocates nothing.
 
-It exists for callers that cannot call cudaMalloc (for instance code running
-while a CUDA graph is captured, or a host with a fixed memory budget): its
-scratch is a fixed device array inside the library. This test calls it through
-the C ABI and checks its output against dfssm_linear_fwd on the same inputs,
-on two calls in a row with different shapes and tokens, so the second call
-also shows that what the first left in the shared scratch does not leak into
-its result. The file is named to be collected last.
+It is there for callers that cannot call cudaMalloc, for instance an embedder
+whose device allocator must not be re-entered from inside the layer, or a host
+with a fixed device memory budget: the kernel's only scratch (its error word)
+is a fixed device array inside the library. This test calls it through the C
+ABI and checks its output bit for bit against dfssm_linear_fwd (the same
+kernel on the same inputs) and against the oracle, on two calls in a row with
+different shapes and tokens, so the second call also shows that what the first
+left in the shared scratch does not leak into its result. The file is named to
+be collected last.
 """
 import numpy as np
 import pytest
 import torch
 
 import bit_gemv_gemm_dfssm_b200 as dfssm
-from gpu_util import TOL_NORMWISE, Linear
+from gpu_util import Linear, check_linear_full
 
 pytestmark = pytest.mark.gpu
 
 
 def run_plan(lin):
+    lin.dy.fill_(float("nan"))
     plan = dfssm.dfssm_linear_plan([lin.desc()])
     try:
         dfssm.dfssm_linear_fwd(plan, 0, lin.weights(), lin.dx.data_ptr(), lin.m, lin.dy.data_ptr(), None,
                                torch.cuda.current_stream().cuda_stream)
         torch.cuda.synchronize()
-        return lin.dy.float().cpu().numpy().copy()
+        return lin.y_host().copy()
     finally:
         dfssm.dfssm_plan_destroy(plan)
 
@@ -36,7 +39,7 @@ def run_noalloc(lin):
                                               torch.cuda.current_stream().cuda_stream)
     assert st == dfssm.DFSSM_OK, dfssm.dfssm_status_string(st)
     torch.cuda.synchronize()
-    return lin.dy.float().cpu().numpy().copy()
+    return lin.y_host().copy()
 
 
 def test_noalloc_matches_plan_entry_point_twice():
@@ -45,12 +48,11 @@ def test_noalloc_matches_plan_entry_point_twice():
         lin = Linear(0x5EED + i, 9, 500 + i, d_in, d_out, m, y_dtype, dbg=False)
         ref = run_plan(lin)
         got = run_noalloc(lin)
-        assert np.all(np.isfinite(got))
-        err = np.abs(got - ref).max() / np.abs(ref).max()
-        assert err <= TOL_NORMWISE, err
+        assert np.array_equal(got.view(np.uint8), ref.view(np.uint8)), "outputs differ from dfssm_linear_fwd"
+        check_linear_full(lin)          # lin.dy holds the no-allocation call's output
 
 
-def test_noalloc_refuses_sizes_beyond_its_scratch():
+def test_noalloc_refuses_sizes_beyond_its_limits():
     lin = Linear(7, 9, 1, 256, 64, 1, dfssm.DFSSM_F32, dbg=False)
     too_many = dfssm.LinearDesc(256, 64, dfssm.RANK, 32, dfssm.DFSSM_F32, 0)
     st = dfssm.lib().dfssm_linear_fwd_noalloc(too_many, lin.weights(), lin.dx.data_ptr(),
