@@ -53,6 +53,10 @@ def _L():
         lib.dfssm_oracle_linear_sampled.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp,
                                                     vp, vp, i64, vp, vp]
         lib.dfssm_oracle_weight_bytes.argtypes = [i32, i32, i32, vp, vp, vp]
+        lib.dfssm_oracle_embed.restype = i32
+        lib.dfssm_oracle_embed.argtypes = [vp, vp, i32, i32, vp, i32, vp]
+        lib.dfssm_oracle_lm_head.argtypes = [vp, vp, i32, i32, vp, i32, vp, vp, i32]
+        lib.dfssm_oracle_lm_head_sampled.argtypes = [vp, vp, i32, i32, vp, i32, vp, vp, i64, vp, vp]
         _lib = lib
     return _lib
 
@@ -144,3 +148,41 @@ def weight_bytes(d_in: int, d_out: int, rank: int = 16):
     a, b, c = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
     _L().dfssm_oracle_weight_bytes(d_in, d_out, rank, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c))
     return a.value, b.value, c.value
+
+
+def embed(table, scale, ids):
+    """Rows of the int8 table times their scales (fp32). Returns (out m x d float32, #bad ids)."""
+    tb, ptb = _c(table, np.int8)
+    sc, psc = _c(scale, np.float32)
+    i, pi = _c(ids, np.int32)
+    vocab, d = tb.shape
+    out = np.empty((i.size, d), np.float32)
+    bad = _L().dfssm_oracle_embed(ptb, psc, vocab, d, pi, i.size, out.ctypes.data)
+    return out, bad
+
+
+def lm_head(table, scale, h_bf16_bits, m: int, threads: int = 0):
+    """Logits (float64, m x vocab) and int32 sums of the int8 head over the quantised h."""
+    tb, ptb = _c(table, np.int8)
+    sc, psc = _c(scale, np.float32)
+    h, ph = _c(h_bf16_bits, np.uint16)
+    vocab, d = tb.shape
+    acc = np.empty((m, vocab), np.int32)
+    logits = np.empty((m, vocab), np.float64)
+    _L().dfssm_oracle_lm_head(ptb, psc, vocab, d, ph, m, acc.ctypes.data, logits.ctypes.data, threads)
+    return dict(acc=acc, logits=logits)
+
+
+def lm_head_sampled(table, scale, h_bf16_bits, m: int, t_idx, v_idx):
+    """Logits and int32 sums at the pairs (t_idx[i], v_idx[i]) only."""
+    tb, ptb = _c(table, np.int8)
+    sc, psc = _c(scale, np.float32)
+    h, ph = _c(h_bf16_bits, np.uint16)
+    t, pt = _c(t_idx, np.int32)
+    v, pv = _c(v_idx, np.int32)
+    vocab, d = tb.shape
+    acc = np.empty(t.size, np.int32)
+    logits = np.empty(t.size, np.float64)
+    _L().dfssm_oracle_lm_head_sampled(ptb, psc, vocab, d, ph, m, pt, pv, t.size, acc.ctypes.data,
+                                      logits.ctypes.data)
+    return dict(acc=acc, logits=logits)

@@ -1,4 +1,5 @@
-// CPU oracle for the DF-SSM 1-bit scaffold + int8 LoRA linear.
+// CPU oracle for the DF-SSM 1-bit scaffold + int8 LoRA linear, and for the int8
+// embedding table / LM head (at the end of this file).
 //
 // TEST INFRASTRUCTURE ONLY. This file is the plain, slow, obviously correct
 // statement of what the layer computes. Only the tests, the smoke check and the
@@ -253,6 +254,78 @@ void dfssm_oracle_weight_bytes(int d_in, int d_out, int rank, int64_t* sign_byte
     *sign_bytes = (int64_t)d_out * d_in / 8;
     *lora_bytes = (int64_t)d_out * rank + (int64_t)rank * d_in;
     *scale_bytes = 4 * ((int64_t)d_out * 2 + rank);
+}
+
+// ---- int8 embedding table and LM head ------------------------------------------------
+// "Density Field State Space Models" (gist.science technical summary), §2.B: the embedding
+// and the LM head are quantised to int8 with per-channel/row scales; §3: they are 37 % of
+// the 278 MB model. One table E (vocab x d int8, row-major) with one fp32 scale per row
+// serves both (Mamba ties the two). Readings taken here:
+//   - a looked-up row is the fp32 product s_E[id] * E[id, j], rounded once (the exact
+//     product in float64, then to fp32);
+//   - the head reads the activations through the layer's own quantiser (q, s_x of the
+//     final hidden state, as for every linear) and sums E[v, j] * q[t, j] in int32;
+//     logits[t, v] = s_x[t] * s_E[v] * sum, in float64.
+
+// Returns the number of ids outside [0, vocab); their rows are zeros.
+int dfssm_oracle_embed(const int8_t* table, const float* scale, int vocab, int d, const int32_t* ids, int m,
+                       float* out) {
+    int bad = 0;
+    for (int t = 0; t < m; ++t) {
+        const int32_t id = ids[t];
+        float* o = out + (int64_t)t * d;
+        if (id < 0 || id >= vocab) {
+            ++bad;
+            for (int j = 0; j < d; ++j) o[j] = 0.0f;
+            continue;
+        }
+        for (int j = 0; j < d; ++j)
+            o[j] = (float)((double)scale[id] * (double)table[(int64_t)id * d + j]);   // exact, then one rounding
+    }
+    return bad;
+}
+
+// logits (float64, m x vocab) and, if acc_out is not NULL, the int32 sums.
+void dfssm_oracle_lm_head(const int8_t* table, const float* scale, int vocab, int d, const uint16_t* h, int m,
+                          int32_t* acc_out, double* logits, int threads) {
+    std::vector<int8_t> q((size_t)m * d);
+    std::vector<float> sx((size_t)m);
+    dfssm_oracle_quantize(h, m, d, q.data(), sx.data());
+#ifdef _OPENMP
+    int nt = threads > 0 ? threads : omp_get_max_threads();
+#pragma omp parallel for collapse(2) schedule(static) num_threads(nt)
+#endif
+    for (int t = 0; t < m; ++t) {
+        for (int v = 0; v < vocab; ++v) {
+            int32_t acc = 0;
+            const int8_t* er = table + (int64_t)v * d;
+            const int8_t* qt = q.data() + (int64_t)t * d;
+            for (int j = 0; j < d; ++j) acc += (int32_t)er[j] * (int32_t)qt[j];
+            if (acc_out) acc_out[(int64_t)t * vocab + v] = acc;
+            logits[(int64_t)t * vocab + v] = (double)sx[t] * (double)scale[v] * (double)acc;
+        }
+    }
+}
+
+// The same at the n pairs (t_idx[i], v_idx[i]) only (for full-size tables).
+void dfssm_oracle_lm_head_sampled(const int8_t* table, const float* scale, int vocab, int d, const uint16_t* h,
+                                  int m, const int32_t* t_idx, const int32_t* v_idx, int64_t n, int32_t* acc_out,
+                                  double* logits) {
+    (void)vocab; (void)m;
+    std::vector<int8_t> q((size_t)d);
+    float sx = 0.0f;
+    int cur_t = -1;
+    for (int64_t i = 0; i < n; ++i) {
+        const int t = t_idx[i], v = v_idx[i];
+        if (t != cur_t) {
+            quantize_token(h + (int64_t)t * d, d, q.data(), &sx);
+            cur_t = t;
+        }
+        int32_t acc = 0;
+        for (int j = 0; j < d; ++j) acc += (int32_t)table[(int64_t)v * d + j] * (int32_t)q[j];
+        if (acc_out) acc_out[i] = acc;
+        logits[i] = (double)sx * (double)scale[v] * (double)acc;
+    }
 }
 
 }  // extern "C"

@@ -338,3 +338,107 @@ def test_scaffold_share_matches_pages():
     assert round(100 * sign / total) == int(g["scaffold_percent"][0])
     # LoRA: 4.6 % of 278 MB against a printed "4 %"; consistent to the page's one digit
     assert abs(100 * lora / total - int(g["lora_percent"][0])) < 1.0
+
+
+# ---------------------------------------------------------------- int8 embedding table / LM head
+
+def tiny_table():
+    g = {ln.split()[0]: ln.split()[1:] for ln in golden_lines("int8_table_tiny.txt")}
+    table = np.array([[int(v) for v in g[f"E{i}"]] for i in range(3)], np.int8)
+    scale = np.array([float(v) for v in g["scale"]], np.float32)
+    return g, table, scale
+
+
+def test_embed_golden_hand_worked():
+    g, table, scale = tiny_table()
+    ids = np.array([int(v) for v in g["embed_ids"]], np.int32)
+    out, bad = oracle.embed(table, scale, ids)
+    assert bad == 0
+    np.testing.assert_array_equal(out[0], np.array([float(v) for v in g["embed_row0"]], np.float32))
+    np.testing.assert_array_equal(out[1], np.array([float(v) for v in g["embed_row1"]], np.float32))
+
+
+def test_embed_matches_float64_product_rounded_once_and_flags_bad_ids():
+    rng = np.random.default_rng(3)
+    table = rng.integers(-127, 128, size=(50, 96)).astype(np.int8)
+    scale = rng.uniform(1e-4, 1e-2, 50).astype(np.float32)
+    ids = np.array([0, 49, 7, -1, 50, 7], np.int32)
+    out, bad = oracle.embed(table, scale, ids)
+    assert bad == 2
+    ref = (table.astype(np.float64) * scale.astype(np.float64)[:, None]).astype(np.float32)
+    for t, i in enumerate(ids):
+        if 0 <= i < 50:
+            np.testing.assert_array_equal(out[t], ref[i])
+        else:
+            assert np.all(out[t] == 0)
+
+
+def test_lm_head_golden_hand_worked():
+    g, table, scale = tiny_table()
+    h0 = bf16_bits([float(v) for v in g["h_t0"]])
+    h = np.stack([h0, bf16_bits(2 * np.array([float(v) for v in g["h_t0"]], np.float32))])
+    q, sx = oracle.quantize(h, 2, 4)
+    np.testing.assert_array_equal(q[0], np.array([int(v) for v in g["q_t0"]], np.int8))
+    out = oracle.lm_head(table, scale, h, 2)
+    acc0 = np.array([int(v) for v in g["acc_t0"]], np.int32)
+    np.testing.assert_array_equal(out["acc"][0], acc0)
+    np.testing.assert_array_equal(out["acc"][1], acc0)
+    sx0 = np.float32(2.0) / np.float32(127.0)
+    expect = float(sx0) * scale.astype(np.float64) * acc0
+    np.testing.assert_array_equal(out["logits"][0], expect)
+    np.testing.assert_array_equal(out["logits"][1], 2 * expect)
+
+
+@pytest.mark.parametrize("m,vocab,d", [(1, 37, 128), (3, 64, 256), (5, 11, 2048)])
+def test_lm_head_brute_force(m, vocab, d):
+    rng = np.random.default_rng(vocab * d + m)
+    table = rng.integers(-127, 128, size=(vocab, d)).astype(np.int8)
+    scale = rng.uniform(1e-4, 1e-2, vocab).astype(np.float32)
+    h = synth.activations(11, 7, vocab, m, d)
+    out = oracle.lm_head(table, scale, h, m)
+    q, sx = oracle.quantize(h, m, d)
+    acc = q.astype(np.float64) @ table.astype(np.float64).T          # exact below 2^53
+    np.testing.assert_array_equal(out["acc"], acc.astype(np.int64))
+    ref = sx.astype(np.float64)[:, None] * scale.astype(np.float64)[None, :] * acc
+    np.testing.assert_allclose(out["logits"], ref, rtol=1e-15, atol=0)
+    # sampled pairs agree with the full head
+    t = np.array([0, m - 1, m - 1], np.int32)
+    v = np.array([vocab - 1, 0, vocab // 2], np.int32)
+    s = oracle.lm_head_sampled(table, scale, h, m, t, v)
+    np.testing.assert_array_equal(s["acc"], out["acc"][t, v])
+    np.testing.assert_array_equal(s["logits"], out["logits"][t, v])
+
+
+def test_lm_head_invariants():
+    rng = np.random.default_rng(5)
+    vocab, d, m = 20, 256, 2
+    table = rng.integers(-127, 128, size=(vocab, d)).astype(np.int8)
+    scale = rng.uniform(1e-4, 1e-2, vocab).astype(np.float32)
+    h = synth.activations(5, 7, 3, m, d)
+    base = oracle.lm_head(table, scale, h, m)
+    # a row scale times 4 gives that row's logits times 4 (exact), the others unchanged
+    s2 = scale.copy()
+    s2[3] *= 4
+    out = oracle.lm_head(table, s2, h, m)
+    np.testing.assert_array_equal(out["logits"][:, 3], 4 * base["logits"][:, 3])
+    np.testing.assert_array_equal(np.delete(out["logits"], 3, 1), np.delete(base["logits"], 3, 1))
+    # permuting the rows of the table permutes the logits
+    perm = rng.permutation(vocab)
+    out = oracle.lm_head(table[perm], scale[perm], h, m)
+    np.testing.assert_array_equal(out["logits"], base["logits"][:, perm])
+    # negating a row negates its sums
+    t2 = table.copy()
+    t2[5] = -t2[5]
+    out = oracle.lm_head(t2, scale, h, m)
+    np.testing.assert_array_equal(out["acc"][:, 5], -base["acc"][:, 5])
+    # h = 0: every logit is 0
+    out = oracle.lm_head(table, scale, np.zeros((m, d), np.uint16), m)
+    assert np.all(out["logits"] == 0) and np.all(out["acc"] == 0)
+
+
+def test_embedding_share_matches_pages():
+    g = {ln.split()[0]: ln.split()[1:] for ln in golden_lines("model_composition.txt")}
+    total = int(g["total_bytes"][0])
+    table_bytes = int(g["vocab"][0]) * int(g["d_model"][0])
+    assert table_bytes == 102_989_824
+    assert round(100 * table_bytes / total) == int(g["emb_percent"][0])
