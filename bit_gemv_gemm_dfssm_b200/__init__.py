@@ -8,7 +8,8 @@ the library is missing, the first call raises ImportError.
 The entry points keep the C names: ``dfssm_linear_plan``, ``dfssm_plan_destroy``,
 ``dfssm_pack_sign``, ``dfssm_linear_fwd``, ``dfssm_linear_stack_fwd``,
 ``dfssm_plan_check``, ``dfssm_plan_workspace_bytes``, ``dfssm_status_string``,
-``dfssm_linear_fwd_noalloc``, ``dfssm_plan_set_test_hooks``.
+``dfssm_linear_fwd_noalloc``, ``dfssm_plan_set_test_hooks``, ``dfssm_embed_fwd``,
+``dfssm_lm_head_fwd``.
 """
 from __future__ import annotations
 
@@ -40,8 +41,9 @@ RANK = 16
 EXPORTS = (
     "dfssm_linear_plan", "dfssm_plan_destroy", "dfssm_pack_sign", "dfssm_linear_fwd",
     "dfssm_linear_stack_fwd", "dfssm_plan_check", "dfssm_plan_workspace_bytes", "dfssm_status_string",
-    "dfssm_linear_fwd_noalloc", "dfssm_plan_set_test_hooks",
+    "dfssm_linear_fwd_noalloc", "dfssm_plan_set_test_hooks", "dfssm_embed_fwd", "dfssm_lm_head_fwd",
 )
+DFSSM_DEVERR_TOKEN_ID = 0x10
 DFSSM_TEST_STALL = 0x1
 DFSSM_NOALLOC_MAX_M = 16
 
@@ -75,6 +77,11 @@ class StackEntry(ctypes.Structure):
 assert ctypes.sizeof(StackEntry) == 104
 
 
+class Int8Table(ctypes.Structure):
+    _fields_ = [("table", ctypes.c_void_p), ("scale", ctypes.c_void_p), ("vocab", ctypes.c_int32),
+                ("d", ctypes.c_int32)]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"libdfssm.so is not built ({LIB_PATH}); run "
@@ -92,6 +99,8 @@ def _load():
     lib.dfssm_plan_check.argtypes = [vp, u32p]
     lib.dfssm_plan_workspace_bytes.argtypes = [vp, ctypes.POINTER(ctypes.c_size_t)]
     lib.dfssm_plan_set_test_hooks.argtypes = [vp, ctypes.c_uint64, ctypes.c_uint32]
+    lib.dfssm_embed_fwd.argtypes = [ctypes.POINTER(Int8Table), vp, i32, vp, i32, vp, vp]
+    lib.dfssm_lm_head_fwd.argtypes = [ctypes.POINTER(Int8Table), vp, i32, vp, i32, vp, vp]
     lib.dfssm_status_string.restype = ctypes.c_char_p
     lib.dfssm_status_string.argtypes = [ctypes.c_int]
     for name in EXPORTS:
@@ -167,6 +176,20 @@ def dfssm_plan_check(plan: int):
     if st not in (DFSSM_OK, DFSSM_ERR_DEVICE_CHECK):
         raise DfssmError(st, "dfssm_plan_check")
     return st, bits.value
+
+
+def dfssm_embed_fwd(table: Int8Table, ids_ptr: int, m: int, out_ptr: int, out_dtype: int, err_ptr: int = 0,
+                    stream: int = 0) -> None:
+    """Embedding rows of the int8 table (see include/dfssm.h)."""
+    _check(lib().dfssm_embed_fwd(ctypes.byref(table), ids_ptr, m, out_ptr, out_dtype, err_ptr or None, stream),
+           "dfssm_embed_fwd")
+
+
+def dfssm_lm_head_fwd(table: Int8Table, h_ptr: int, m: int, logits_ptr: int, out_dtype: int, acc_ptr: int = 0,
+                      stream: int = 0) -> None:
+    """Logits of the int8 LM head over the quantised hidden state (see include/dfssm.h)."""
+    _check(lib().dfssm_lm_head_fwd(ctypes.byref(table), h_ptr, m, logits_ptr, out_dtype, acc_ptr or None, stream),
+           "dfssm_lm_head_fwd")
 
 
 def dfssm_plan_set_test_hooks(plan: int, wait_limit_ns: int = 0, flags: int = 0) -> None:

@@ -12,6 +12,7 @@
 
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -24,6 +25,7 @@ cudaError_t set_quant_attr(int optin);
 cudaError_t set_quant_rows_attr(int optin);
 cudaError_t set_decode_attr(int optin);
 cudaError_t set_prefill_attr(int optin);
+cudaError_t set_int8_table_attr(int optin);
 int prefill_box_tokens();
 int prefill_box_bytes();
 
@@ -342,6 +344,69 @@ dfssm_status dfssm_plan_check(dfssm_plan plan, uint32_t* bits) {
     if (cudaMemset(plan->err, 0, 4) != cudaSuccess) return DFSSM_ERR_CUDA;
     if (bits) *bits = v;
     return v ? DFSSM_ERR_DEVICE_CHECK : DFSSM_OK;
+}
+
+// Per-device set-up of the plan-free int8 table calls (SM count, shared-memory limits).
+namespace {
+struct TableSetup {
+    int sm_count = 0;
+    bool ready = false;
+};
+TableSetup g_table_setup[64];
+std::mutex g_table_mu;
+
+dfssm_status table_setup(int* sm_count) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DFSSM_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_table_mu);
+    TableSetup& t = g_table_setup[dev];
+    if (!t.ready) {
+        int optin = 0;
+        if (cudaDeviceGetAttribute(&t.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+            set_int8_table_attr(optin) != cudaSuccess)
+            return DFSSM_ERR_CUDA;
+        t.ready = true;
+    }
+    *sm_count = t.sm_count;
+    return DFSSM_OK;
+}
+
+dfssm_status check_table(const dfssm_int8_table* t) {
+    if (!t || !t->table || !t->scale || !aligned16(t->table) || !aligned16(t->scale)) return DFSSM_ERR_INVALID_ARG;
+    if (t->d < 16 || t->d > kMaxDIn || t->d % 16 != 0 || t->vocab < 1 || t->vocab > (1 << 24))
+        return DFSSM_ERR_UNSUPPORTED_SHAPE;
+    return DFSSM_OK;
+}
+}  // namespace
+
+dfssm_status dfssm_embed_fwd(const dfssm_int8_table* table, const int32_t* ids, int32_t m, void* out,
+                             int32_t out_dtype, uint32_t* err, void* stream) {
+    dfssm_status s = check_table(table);
+    if (s != DFSSM_OK) return s;
+    if (!ids || !out || !aligned16(out) || (reinterpret_cast<uintptr_t>(ids) & 3u) || m < 1 || m > kMaxM)
+        return DFSSM_ERR_INVALID_ARG;
+    if ((out_dtype != DFSSM_BF16 && out_dtype != DFSSM_F32) || (reinterpret_cast<uintptr_t>(err) & 3u))
+        return DFSSM_ERR_INVALID_ARG;
+    int sms = 0;
+    if ((s = table_setup(&sms)) != DFSSM_OK) return s;
+    Int8TableArgs a{table->table, table->scale, table->vocab, table->d, ids, nullptr, m, out, out_dtype,
+                    nullptr, err};
+    return launch_embed(a, (cudaStream_t)stream) == cudaSuccess ? DFSSM_OK : DFSSM_ERR_CUDA;
+}
+
+dfssm_status dfssm_lm_head_fwd(const dfssm_int8_table* table, const void* h, int32_t m, void* logits,
+                               int32_t out_dtype, int32_t* acc, void* stream) {
+    dfssm_status s = check_table(table);
+    if (s != DFSSM_OK) return s;
+    if (!h || !logits || !aligned16(h) || !aligned16(logits) || !aligned16(acc) || m < 1 || m > 16)
+        return DFSSM_ERR_INVALID_ARG;
+    if (out_dtype != DFSSM_BF16 && out_dtype != DFSSM_F32) return DFSSM_ERR_INVALID_ARG;
+    int sms = 0;
+    if ((s = table_setup(&sms)) != DFSSM_OK) return s;
+    Int8TableArgs a{table->table, table->scale, table->vocab, table->d, nullptr, h, m, logits, out_dtype, acc,
+                    nullptr};
+    return launch_lm_head(a, sms, (cudaStream_t)stream) == cudaSuccess ? DFSSM_OK : DFSSM_ERR_CUDA;
 }
 
 dfssm_status dfssm_plan_set_test_hooks(dfssm_plan plan, uint64_t wait_limit_ns, uint32_t flags) {

@@ -135,6 +135,22 @@ inline int lora_slice_grid(const LaunchCtx& c) {
     return items < c.sm_count ? items : c.sm_count;
 }
 
+// Arguments of the int8 table kernels (int8_table.cu).
+struct Int8TableArgs {
+    const int8_t* table;   // vocab x d int8
+    const float* scale;    // vocab fp32
+    int vocab, d;
+    const int32_t* ids;    // embedding: m token ids
+    const void* in;        // LM head: m x d bf16 hidden state
+    int m;
+    void* out;             // m x d (embedding) or m x vocab (LM head) of out_dtype
+    int out_dtype;
+    int32_t* acc;          // LM head: optional int32 sums
+    uint32_t* err;         // embedding: optional error word
+};
+cudaError_t launch_embed(const Int8TableArgs& a, cudaStream_t s);
+cudaError_t launch_lm_head(const Int8TableArgs& a, int sm_count, cudaStream_t s);
+
 cudaError_t launch_pack_sign(const void* src, int src_dtype, int d_out, int d_in, uint8_t* packed,
                              cudaStream_t s);
 cudaError_t launch_quant(const LaunchCtx& c);

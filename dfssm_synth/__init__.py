@@ -30,8 +30,11 @@ OUT_PROJ = (4096, 2048)
 N_LAYERS = 48
 
 # tensor ids inside a stream
-T_X, T_COLS, T_SIGN, T_ALPHA, T_WA, T_SA, T_WB, T_SB = range(8)
+T_X, T_COLS, T_SIGN, T_ALPHA, T_WA, T_SA, T_WB, T_SB, T_TABLE, T_TSCALE, T_IDS = range(11)
 KIND_WEIGHTS, KIND_ACT = 1, 2
+# the tied int8 embedding / LM-head table of Mamba-2 1.3B: its 50,277-token vocabulary padded to
+# a multiple of 16, d_model columns
+VOCAB = 50288
 
 
 def build(force: bool = False) -> str:
@@ -132,6 +135,23 @@ def linear_weights(seed: int, cfg: int, index: int, d_in: int, d_out: int, rank:
     L.dfssm_synth_int8_sym127(k_(T_WB), out["wb"].size, _ptr(out["wb"]))
     L.dfssm_synth_uniform_f32(k_(T_SB), rank, 1e-4, 1e-3, _ptr(out["sb"]))
     return out
+
+
+def int8_table(seed: int, cfg: int, vocab: int, d: int) -> dict:
+    """An int8 table (vocab x d, uniform on -127..127) with one fp32 scale per row (U(1e-4, 1e-3))."""
+    out = dict(table=np.empty((vocab, d), np.int8), scale=np.empty(vocab, np.float32))
+    L = _L()
+    L.dfssm_synth_int8_sym127(key(seed, stream_id(KIND_WEIGHTS, cfg, 0, 0, T_TABLE)), out["table"].size,
+                              _ptr(out["table"]))
+    L.dfssm_synth_uniform_f32(key(seed, stream_id(KIND_WEIGHTS, cfg, 0, 0, T_TSCALE)), vocab, 1e-4, 1e-3,
+                              _ptr(out["scale"]))
+    return out
+
+
+def token_ids(seed: int, cfg: int, m: int, vocab: int) -> np.ndarray:
+    """m token ids drawn uniformly from [0, vocab)."""
+    r = raw(seed, stream_id(KIND_ACT, cfg, m, 0, T_IDS), 0, m)
+    return (r % np.uint64(vocab)).astype(np.int32)
 
 
 def stack_shapes(n_layers: int = N_LAYERS):

@@ -69,6 +69,7 @@ typedef enum { DFSSM_BF16 = 0, DFSSM_F32 = 1, DFSSM_I8 = 2 } dfssm_dtype;
 #define DFSSM_DEVERR_NONFINITE  0x2u   /* a token's amax was Inf or NaN (output undefined) */
 #define DFSSM_DEVERR_TIMEOUT    0x4u   /* a bounded in-kernel wait gave up (output undefined) */
 #define DFSSM_DEVERR_ENTRY_PTR  0x8u   /* a stack entry holds a NULL or misaligned pointer (entry skipped) */
+#define DFSSM_DEVERR_TOKEN_ID   0x10u  /* an embedding id outside [0, vocab) (its row is zeros) */
 
 /* Shape of one linear. d_in % 128 == 0, 128 <= d_in <= 8192; 1 <= d_out <= 2^20;
  * rank == 16; 1 <= max_m <= 65536; y_dtype DFSSM_BF16 or DFSSM_F32; flags = 0. */
@@ -186,6 +187,38 @@ dfssm_status dfssm_linear_fwd_noalloc(const dfssm_linear_desc* desc, const dfssm
 /* Synchronise the plan's device, read and clear its error word.
  * Returns DFSSM_OK or DFSSM_ERR_DEVICE_CHECK (*bits, if not NULL, gets the word). */
 dfssm_status dfssm_plan_check(dfssm_plan plan, uint32_t* bits);
+
+/* An int8 table with one fp32 scale per row: the embedding and the LM head ("Density
+ * Field State Space Models", technical summary §2.B: embedding / LM head quantised to
+ * int8 with per-channel/row scales; §3: 37 % of the 278 MB model; Mamba ties the two, so
+ * one table serves both). Device pointers, caller-owned, 16-byte aligned:
+ *   table : vocab x d int8, row-major; d % 16 == 0, 16 <= d <= 8192; 1 <= vocab <= 2^24
+ *   scale : vocab fp32 */
+typedef struct {
+    const int8_t* table;
+    const float* scale;
+    int32_t vocab;
+    int32_t d;
+} dfssm_int8_table;
+
+/* Embedding rows: out[t, j] = scale[ids[t]] * table[ids[t], j], one fp32 product (exact
+ * operands, one rounding), rounded to bf16 (nearest even) when out_dtype is DFSSM_BF16.
+ * table: HOST struct of device pointers; ids: m int32 (device); out: m x d of out_dtype
+ * (device); 1 <= m <= 65536. An id outside [0, vocab) gives a row of zeros and, if err (a
+ * device uint32, may be NULL) is given, ORs DFSSM_DEVERR_TOKEN_ID into it. Allocates
+ * nothing; the first call on a device sets kernel attributes (make it before any stream
+ * capture). */
+dfssm_status dfssm_embed_fwd(const dfssm_int8_table* table, const int32_t* ids, int32_t m, void* out,
+                             int32_t out_dtype, uint32_t* err, void* stream);
+
+/* LM head: logits[t, v] = s_x[t] * (scale[v] * sum_j table[v, j] * q[t, j]), the sum in
+ * int32, where q, s_x are the layer's per-token int8 quantisation of h (as for every
+ * linear above). table: HOST struct of device pointers; h: m x d bf16 (device),
+ * 1 <= m <= 16; logits: m x vocab of out_dtype (device); acc: optional m x vocab int32
+ * sums (device, may be NULL). Allocates nothing; the first call on a device sets kernel
+ * attributes (make it before any stream capture). */
+dfssm_status dfssm_lm_head_fwd(const dfssm_int8_table* table, const void* h, int32_t m, void* logits,
+                               int32_t out_dtype, int32_t* acc, void* stream);
 
 /* Test of the error path of the decode kernel (m <= 16 tokens), which must end with an
  * error status and never hang. With flags & DFSSM_TEST_STALL, the first CTA of that
