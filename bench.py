@@ -190,6 +190,37 @@ def oracle_stack_pass(shapes, m, seed, cfg, linear_ids, threads=0):
     return dt, nbytes
 
 
+def cpu_baseline_leg(shapes, m, seed, cfg, n_single=8):
+    """The oracle as it stands on the host cores: the +-1 unpack timed apart, then the forward
+    pass from the unpacked weights on every linear with all cores and on the first n_single
+    linears single-threaded."""
+    import oracle
+    inputs = []
+    for i, (d_in, d_out) in enumerate(shapes):
+        inputs.append((synth.linear_weights(seed, synth.weight_cfg(cfg), i, d_in, d_out),
+                       synth.activations(seed, cfg, i, m, d_in), d_in, d_out))
+    t0 = time.perf_counter()
+    unpacked = [oracle.unpack_sign(w["sign"], d_out, d_in) for w, _, d_in, d_out in inputs]
+    t_unpack = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    for (w, x, d_in, d_out), wpm in zip(inputs, unpacked):
+        oracle.linear_unpacked(x, wpm, w, m, d_in, d_out, threads=0)
+    t_all = time.perf_counter() - t0
+    ns = min(n_single, len(shapes))
+    t0 = time.perf_counter()
+    for (w, x, d_in, d_out), wpm in list(zip(inputs, unpacked))[:ns]:
+        oracle.linear_unpacked(x, wpm, w, m, d_in, d_out, threads=1)
+    t_one = time.perf_counter() - t0
+    b_all = stack_bytes(shapes, m)
+    b_one = stack_bytes(shapes[:ns], m)
+    return {"kind": "oracle", "value": b_all / t_all / 1e9, "unit": "GB/s", "cores": oracle_threads(),
+            "sample": f"all {len(shapes)} linears at M={m}, forward from unpacked +-1 weights (OpenMP over "
+                      f"tokens x rows); the unpack of all linears took {t_unpack:.2f} s and is not in the value",
+            "single_thread": {"value": b_one / t_one / 1e9, "unit": "GB/s", "cores": 1,
+                              "sample": f"the first {ns} linears at M={m}, one thread"},
+            "unpack_s": t_unpack}
+
+
 def oracle_threads():
     try:
         return len(os.sched_getaffinity(0))
@@ -198,24 +229,36 @@ def oracle_threads():
 
 
 def run_reference(args, wl_name):
-    """The oracle as it stands, timed on the host cores: one bounded sample per step."""
+    """The oracle as it stands, timed on the host cores: each step one forward pass over the
+    workload's linears from the unpacked +-1 weights (the unpack is done once, untimed, as in
+    the GPU arm's cpu_baseline); for more than 64 tokens a bounded token sample."""
+    import oracle
     ws, rank, _ = dist_env()
     if rank != 0:
         return 0
     wl = synth.WORKLOADS[wl_name]
     shapes, m, cfg = wl["shapes"], wl["m"], wl["cfg"]
-    sample_ids = [0, 1, 2, 3] if m <= 64 else [0, 1]
     m_s = m if m <= 64 else 4
     cores = oracle_threads()
+    inputs = []
+    for i, (d_in, d_out) in enumerate(shapes):
+        w = synth.linear_weights(synth.MASTER_SEED, synth.weight_cfg(cfg), i, d_in, d_out)
+        inputs.append((w, oracle.unpack_sign(w["sign"], d_out, d_in), synth.activations(synth.MASTER_SEED, cfg, i, m_s, d_in),
+                       d_in, d_out))
+
+    def one_pass():
+        t0 = time.perf_counter()
+        for w, wpm, x, d_in, d_out in inputs:
+            oracle.linear_unpacked(x, wpm, w, m_s, d_in, d_out, threads=0)
+        return time.perf_counter() - t0
+
     for _ in range(args.warmup):
-        oracle_stack_pass(shapes, m_s, synth.MASTER_SEED, cfg, sample_ids)
-    tot_t, tot_b = 0.0, 0
-    for _ in range(args.steps):
-        dt, nb = oracle_stack_pass(shapes, m_s, synth.MASTER_SEED, cfg, sample_ids)
-        tot_t += dt
-        tot_b += nb
-    gbs = tot_b / tot_t / 1e9
-    sample = f"{len(sample_ids)} of {len(shapes)} linears (in_proj/out_proj pairs), M={m_s}, per step"
+        one_pass()
+    tot_t = sum(one_pass() for _ in range(args.steps))
+    nb = stack_bytes(shapes, m_s) * args.steps
+    gbs = nb / tot_t / 1e9
+    sample = (f"all {len(shapes)} linears at M={m_s} per step" + ("" if m_s == m else f" (of M={m})") +
+              ", forward from unpacked +-1 weights, OpenMP over tokens x rows")
     line = {
         "impl": "reference", "metric": metric_name(), "value": gbs, "unit": "GB/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / max(args.steps, 1),
@@ -234,10 +277,23 @@ def metric_name():
 
 # --------------------------------------------------------------------------- GPU arm
 
+def device_weight_sets(shapes, cfg, seed, n_sets=2):
+    """n_sets independent weight sets of the stack on the device (alternated so steps miss L2)."""
+    import torch
+    sets = []
+    for s in range(n_sets):
+        ws = []
+        for i, (d_in, d_out) in enumerate(shapes):
+            w = synth.linear_weights(seed + 7919 * s, synth.weight_cfg(cfg), i, d_in, d_out)
+            ws.append({k: torch.from_numpy(v).cuda() for k, v in w.items()})
+        sets.append(ws)
+    return sets
+
+
 class StackRunner:
     """Device buffers, plan and stack entries for one workload, two weight sets."""
 
-    def __init__(self, shapes, m, cfg, seed, n_sets=2):
+    def __init__(self, shapes, m, cfg, seed, n_sets=2, weight_sets=None):
         import torch
         import bit_gemv_gemm_dfssm_b200 as dfssm
         self.torch, self.dfssm = torch, dfssm
@@ -261,11 +317,10 @@ class StackRunner:
         self.y = torch.empty(yo, dtype=torch.bfloat16, device="cuda")
         self.y_host = torch.empty(yo, dtype=torch.int16).pin_memory()
         self.sets = []
+        if weight_sets is None:
+            weight_sets = device_weight_sets(shapes, cfg, seed, n_sets)
         for s in range(n_sets):
-            ws = []
-            for i, (d_in, d_out) in enumerate(shapes):
-                w = synth.linear_weights(seed + 7919 * s, synth.weight_cfg(cfg), i, d_in, d_out)
-                ws.append({k: torch.from_numpy(v).cuda() for k, v in w.items()})
+            ws = weight_sets[s]
             ents = []
             for i, w in enumerate(ws):
                 ents.append(dfssm.StackEntry(
@@ -305,6 +360,103 @@ class StackRunner:
 
     def close(self):
         self.dfssm.dfssm_plan_destroy(self.plan)
+
+
+def stack_block(torch, wl_name, seed, steps, peaks, dist, dev, weight_sets=None, layers=0):
+    """One stack workload: ms per step (CUDA graph per step, two weight sets alternated), GB/s,
+    tokens/s, TOPS and both roofline fractions."""
+    wl = synth.WORKLOADS[wl_name]
+    shapes, m, cfg = wl["shapes"], wl["m"], wl["cfg"]
+    if layers:
+        shapes = shapes[:2 * layers]
+    r = StackRunner(shapes, m, cfg, seed, weight_sets=weight_sets)
+    graphs = r.graphs()
+    with ClockSampler(dev.index or 0) as clk:
+        ms = timed_device(torch, lambda i: graphs[i % 2].replay(), steps, 3, dist, dev)
+    r.check()
+    r.close()
+    del graphs
+    ms_step = ms / steps
+    nb, nops = stack_bytes(shapes, m), stack_ops(shapes, m)
+    gbs = nb / (ms_step * 1e-3) / 1e9
+    tops = nops / (ms_step * 1e-3) / 1e12
+    peak_i8 = peaks["bf16"] * INT8_PER_BF16
+    return {"workload": wl_name, "m": m, "steps": steps, "ms_per_step": ms_step, "GB/s": gbs,
+            "tokens_per_s": m / (ms_step * 1e-3), "TOPS": tops,
+            "hbm_frac": gbs / peaks["hbm"], "int8_frac": tops / peak_i8,
+            "path": "decode (slice/quant + decode kernels)" if m <= 16 else "quant_rows + tcgen05 prefill",
+            "clocks": clk.summary()}
+
+
+def single_block(torch, wl_name, seed, peaks, dev, min_bytes=256 << 20, reps=4):
+    """One projection at M = 1 with cold L2: the call rotates over enough copies of the weights
+    (>= 256 MB) inside one CUDA graph; per-call latency and GB/s."""
+    import bit_gemv_gemm_dfssm_b200 as dfssm
+    wl = synth.WORKLOADS[wl_name]
+    (d_in, d_out), m = wl["shapes"][0], wl["m"]
+    w = synth.linear_weights(seed, synth.weight_cfg(wl["cfg"]), 0, d_in, d_out)
+    dw = {k: torch.from_numpy(v).cuda() for k, v in w.items()}
+    per = sum(v.numel() * v.element_size() for v in dw.values())
+    n = (min_bytes + per - 1) // per
+    copies = [{k: v.clone() for k, v in dw.items()} for _ in range(n)]
+    x = torch.from_numpy(synth.activations(seed, wl["cfg"], 0, m, d_in).view(np.int16).copy()).cuda()
+    y = torch.empty((m, d_out), dtype=torch.bfloat16, device="cuda")
+    plan = dfssm.dfssm_linear_plan([(d_in, d_out, m, dfssm.DFSSM_BF16)])
+    structs = [dfssm.weights_struct(c["sign"], c["alpha"], c["wa"], c["sa"], c["wb"], c["sb"]) for c in copies]
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        st = torch.cuda.current_stream().cuda_stream
+        for ws in structs:
+            dfssm.dfssm_linear_fwd(plan, 0, ws, x.data_ptr(), m, y.data_ptr(), None, st)
+    torch.cuda.synchronize()
+    ms = timed_device(torch, lambda i: g.replay(), reps, 3, None, dev)
+    st_, bits = dfssm.dfssm_plan_check(plan)
+    dfssm.dfssm_plan_destroy(plan)
+    del g
+    if st_ != dfssm.DFSSM_OK:
+        raise RuntimeError(f"device error word {bits:#x}")
+    us = ms * 1e3 / (reps * n)
+    nb = stack_bytes([(d_in, d_out)], m)
+    return {"workload": wl_name, "m": m, "us_per_call": us, "GB/s": nb / (us * 1e-6) / 1e9,
+            "hbm_frac": nb / (us * 1e-6) / 1e9 / peaks["hbm"], "tokens_per_s": m / (us * 1e-6),
+            "l2": f"cold: {n} weight copies ({n * per / 2**20:.0f} MB) rotated in one CUDA graph",
+            "calls_timed": reps * n}
+
+
+def lm_head_block(torch, seed, peaks, dev, m=1, steps=200):
+    """The int8 LM head over the tied 50,288 x 2048 table at m tokens: two tables alternated
+    (2 x 103 MB > L2), one CUDA graph per call."""
+    import bit_gemv_gemm_dfssm_b200 as dfssm
+    vocab, d = synth.VOCAB, synth.D_MODEL
+    tabs = []
+    for s in range(2):
+        t = synth.int8_table(seed + s, 5, vocab, d)
+        tabs.append({k: torch.from_numpy(v).cuda() for k, v in t.items()})
+    h = torch.from_numpy(synth.activations(seed, 5, 1, m, d).view(np.int16).copy()).cuda()
+    logits = torch.empty((m, vocab), dtype=torch.bfloat16, device="cuda")
+    cs = [dfssm.Int8Table(t["table"].data_ptr(), t["scale"].data_ptr(), vocab, d) for t in tabs]
+    dfssm.dfssm_lm_head_fwd(cs[0], h.data_ptr(), m, logits.data_ptr(), dfssm.DFSSM_BF16, 0,
+                            torch.cuda.current_stream().cuda_stream)     # the per-device set-up
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    gs = []
+    for c in cs:
+        side.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            dfssm.dfssm_lm_head_fwd(c, h.data_ptr(), m, logits.data_ptr(), dfssm.DFSSM_BF16, 0,
+                                    torch.cuda.current_stream().cuda_stream)
+        gs.append(g)
+    torch.cuda.synchronize()
+    ms = timed_device(torch, lambda i: gs[i % 2].replay(), steps, 3, None, dev)
+    del gs
+    us = ms * 1e3 / steps
+    nb = vocab * d + 4 * vocab + 2 * m * d + 2 * m * vocab
+    return {"workload": f"lm_head_m{m}", "vocab": vocab, "d": d, "m": m, "us_per_call": us,
+            "GB/s": nb / (us * 1e-6) / 1e9, "hbm_frac": nb / (us * 1e-6) / 1e9 / peaks["hbm"],
+            "bytes_per_call": nb, "l2": "two 103 MB tables alternated"}
 
 
 def timed_device(torch, run_step, steps, warmup, dist, dev):
@@ -409,6 +561,20 @@ def run_gpu(args, wl_name):
         pr.close()
         del pgraphs
 
+    # the other configurations: single projections (cold L2), the stack at M = 4 / 16 / 64 / 512,
+    # the int8 LM head (every rank runs the same blocks; rank 0 reports them)
+    extras = None
+    if not args.no_extras:
+        extras = {"single": [], "stacks": [], "lm_head": None}
+        for wn in ("out_proj_m1", "in_proj_m1"):
+            extras["single"].append(single_block(torch, wn, seed, peaks, dev))
+        sets = device_weight_sets(synth.stack_shapes(), 2, seed)
+        for wn, st in (("stack48_m4", 300), ("stack48_m16", 200), ("stack48_m64", 100), ("stack48_m512", 20)):
+            extras["stacks"].append(stack_block(torch, wn, seed, st, peaks, dist, dev, weight_sets=sets))
+        del sets
+        torch.cuda.empty_cache()
+        extras["lm_head"] = lm_head_block(torch, seed, peaks, dev)
+
     if rank != 0:
         if dist is not None:
             dist.destroy_process_group()
@@ -416,10 +582,7 @@ def run_gpu(args, wl_name):
 
     cpu = None
     if ws == 1 and not args.no_cpu_baseline:
-        ids = list(range(len(shapes))) if m == 1 else [0, 1, 2, 3]
-        dt, cb = oracle_stack_pass(shapes, m, seed, cfg, ids)
-        cpu = {"kind": "oracle", "value": cb / dt / 1e9, "unit": "GB/s", "cores": oracle_threads(),
-               "sample": f"{len(ids)} of {len(shapes)} linears at M={m}, one pass, OpenMP over rows"}
+        cpu = cpu_baseline_leg(shapes, m, seed, cfg)
 
     line = {
         "metric": metric_name(), "value": value_gbs, "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
@@ -444,6 +607,7 @@ def run_gpu(args, wl_name):
         "clocks": clk.summary(),
         "cpu_baseline": cpu,
         "prefill": prefill,
+        "workloads": extras,
     }
     print(json.dumps(line), flush=True)
     if dist is not None:
@@ -462,6 +626,8 @@ def main(argv=None):
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other configurations (single projections, M = 4/16/64/512, LM head)")
     ap.add_argument("--layers", type=int, default=0,
                     help="use only the first L layers of the stack (small cases for profiling)")
     args = ap.parse_args(argv)

@@ -167,6 +167,7 @@ WORKLOADS = {
     "stack48_m4": dict(cfg=3, shapes=stack_shapes(), m=4),
     "stack48_m16": dict(cfg=3, shapes=stack_shapes(), m=16),
     "stack48_m64": dict(cfg=3, shapes=stack_shapes(), m=64),
+    "stack48_m512": dict(cfg=4, shapes=stack_shapes(), m=512),
     "stack48_m2048": dict(cfg=4, shapes=stack_shapes(), m=2048),
 }
 

@@ -50,6 +50,8 @@ def _L():
         lib.dfssm_oracle_quantize.argtypes = [vp, i32, i32, vp, vp]
         lib.dfssm_oracle_linear.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp,
                                             vp, vp, vp, vp, vp, i32]
+        lib.dfssm_oracle_linear_unpacked.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp,
+                                                     vp, vp, vp, vp, vp, i32]
         lib.dfssm_oracle_linear_sampled.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp,
                                                     vp, vp, i64, vp, vp]
         lib.dfssm_oracle_weight_bytes.argtypes = [i32, i32, i32, vp, vp, vp]
@@ -126,6 +128,17 @@ def linear(x_bf16_bits, w: dict, m: int, d_in: int, d_out: int, rank: int = 16, 
                              out["q"].ctypes.data, out["sx"].ctypes.data, out["acc"].ctypes.data,
                              out["h"].ctypes.data, out["y"].ctypes.data, threads)
     return out
+
+
+def linear_unpacked(x_bf16_bits, w_pm1, w: dict, m: int, d_in: int, d_out: int, rank: int = 16, threads: int = 0):
+    """The layer from the unpacked +-1 matrix (d_out x d_in int8, see unpack_sign): y (float64) only."""
+    x, px = _c(x_bf16_bits, np.uint16)
+    keep = [_c(w_pm1, np.int8), _c(w["alpha"], np.float32), _c(w["wa"], np.int8),
+            _c(w["sa"], np.float32), _c(w["wb"], np.int8), _c(w["sb"], np.float32)]
+    y = np.empty((m, d_out), np.float64)
+    _L().dfssm_oracle_linear_unpacked(px, m, d_in, d_out, rank, *[p for _, p in keep], None, None, None, None,
+                                      y.ctypes.data, threads)
+    return y
 
 
 def linear_sampled(x_bf16_bits, w: dict, m: int, d_in: int, d_out: int, t_idx, o_idx, rank: int = 16):

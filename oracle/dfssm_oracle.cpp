@@ -176,6 +176,13 @@ static double dequant(float sx, float alpha, float sa, const int8_t* wa_row, con
 
 // Full layer for m tokens. Any of q_out, sx_out, acc_out, h_out may be NULL.
 // threads <= 0 uses the OpenMP default; 1 runs single-threaded.
+// The layer from the unpacked +-1 matrix w (d_out x d_in int8): everything after the unpack.
+void dfssm_oracle_linear_unpacked(const uint16_t* x, int m, int d_in, int d_out, int rank,
+                                  const int8_t* w, const float* alpha, const int8_t* wa,
+                                  const float* sa, const int8_t* wb, const float* sb,
+                                  int8_t* q_out, float* sx_out, int32_t* acc_out, int32_t* h_out,
+                                  double* y, int threads);
+
 void dfssm_oracle_linear(const uint16_t* x, int m, int d_in, int d_out, int rank,
                          const uint8_t* sign, const float* alpha, const int8_t* wa,
                          const float* sa, const int8_t* wb, const float* sb,
@@ -183,7 +190,16 @@ void dfssm_oracle_linear(const uint16_t* x, int m, int d_in, int d_out, int rank
                          double* y, int threads) {
     std::vector<int8_t> w((size_t)d_out * d_in);
     dfssm_oracle_unpack_sign(sign, d_out, d_in, w.data());
+    dfssm_oracle_linear_unpacked(x, m, d_in, d_out, rank, w.data(), alpha, wa, sa, wb, sb, q_out, sx_out, acc_out,
+                                 h_out, y, threads);
+}
 
+void dfssm_oracle_linear_unpacked(const uint16_t* x, int m, int d_in, int d_out, int rank,
+                                  const int8_t* w_pm1, const float* alpha, const int8_t* wa,
+                                  const float* sa, const int8_t* wb, const float* sb,
+                                  int8_t* q_out, float* sx_out, int32_t* acc_out, int32_t* h_out,
+                                  double* y, int threads) {
+    const int8_t* w = w_pm1;
     std::vector<int8_t> q((size_t)m * d_in);
     std::vector<float> sx((size_t)m);
     dfssm_oracle_quantize(x, m, d_in, q.data(), sx.data());
@@ -204,7 +220,7 @@ void dfssm_oracle_linear(const uint16_t* x, int m, int d_in, int d_out, int rank
     for (int t = 0; t < m; ++t) {
         for (int o = 0; o < d_out; ++o) {
             int32_t acc = 0;
-            const int8_t* wr = w.data() + (int64_t)o * d_in;
+            const int8_t* wr = w + (int64_t)o * d_in;
             const int8_t* qt = q.data() + (int64_t)t * d_in;
             for (int j = 0; j < d_in; ++j) acc += (int32_t)wr[j] * (int32_t)qt[j];
             if (acc_out) acc_out[(int64_t)t * d_out + o] = acc;

@@ -301,6 +301,15 @@ def test_sampled_matches_full():
     np.testing.assert_array_equal(s["y"], full["y"][t, o])
 
 
+def test_unpacked_entry_matches_the_layer():
+    # the forward pass from the unpacked +-1 matrix (the CPU baseline times the unpack apart)
+    x, w = rand_case(21, 3, 384, 50)
+    full = oracle.linear(x, w, 3, 384, 50)
+    wpm = oracle.unpack_sign(w["sign"], 50, 384)
+    np.testing.assert_array_equal(oracle.linear_unpacked(x, wpm, w, 3, 384, 50), full["y"])
+    np.testing.assert_array_equal(oracle.linear_unpacked(x, wpm, w, 3, 384, 50, threads=1), full["y"])
+
+
 def test_threads_do_not_change_results():
     m, d_in, d_out = 3, 512, 64
     x, w = rand_case(66, m, d_in, d_out)
