@@ -69,7 +69,6 @@ constexpr int kThreads = kWarps * 32;
 #define DFSSM_DECODE_STAGES 3
 #endif
 constexpr int kChunkBytes = DFSSM_DECODE_CHUNK_BYTES;   // sign bytes per row per k-chunk (8 columns per byte)
-constexpr int kChunkJ = kChunkBytes / 16;                // 16-byte pieces per row per chunk
 constexpr int kGroups = kChunkBytes / 32;                // 256-column groups per chunk
 constexpr int kTokPad = 64;        // q row stride = round_up(d_in, 256) + 64 (= 64 mod 128: conflict-free B reads)
 

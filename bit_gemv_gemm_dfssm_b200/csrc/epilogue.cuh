@@ -33,6 +33,29 @@ __device__ __forceinline__ float quant_sx(float amax) { return amax == 0.0f ? 0.
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// 4 bf16 (8 bytes) -> 4 int8 packed little-endian
+__device__ __forceinline__ uint32_t quant4(uint2 raw, float inv, bool zero, int& sum) {
+    const int q0 = quant1(bf16_lo(raw.x), inv, zero);
+    const int q1 = quant1(bf16_hi(raw.x), inv, zero);
+    const int q2 = quant1(bf16_lo(raw.y), inv, zero);
+    const int q3 = quant1(bf16_hi(raw.y), inv, zero);
+    sum += q0 + q1 + q2 + q3;
+    return (uint32_t)(q0 & 0xFF) | ((uint32_t)(q1 & 0xFF) << 8) | ((uint32_t)(q2 & 0xFF) << 16) |
+           ((uint32_t)(q3 & 0xFF) << 24);
+}
+
+// running max of |x| over 8 bf16 values, as fp32 bit patterns: for |x| the unsigned order is
+// the numeric order, and a NaN (bits above Inf) wins, so a non-finite row is still seen
+__device__ __forceinline__ uint32_t absmax8_bits(uint4 v, uint32_t m) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        m = max(m, (w[i] << 16) & 0x7FFFFFFFu);
+        m = max(m, w[i] & 0x7FFF0000u);
+    }
+    return m;
+}
+
 // round-to-nearest-even fp32 -> bf16 bits (NaN kept quiet)
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
     const uint32_t u = __float_as_uint(f);

@@ -43,29 +43,6 @@ struct QuantRed {
     float sx[kTok];
 };
 
-// 4 bf16 (8 bytes) -> 4 int8 packed little-endian
-__device__ __forceinline__ uint32_t quant4(uint2 raw, float inv, bool zero, int& sum) {
-    const int q0 = quant1(bf16_bits_to_float(raw.x & 0xFFFFu), inv, zero);
-    const int q1 = quant1(bf16_bits_to_float(raw.x >> 16), inv, zero);
-    const int q2 = quant1(bf16_bits_to_float(raw.y & 0xFFFFu), inv, zero);
-    const int q3 = quant1(bf16_bits_to_float(raw.y >> 16), inv, zero);
-    sum += q0 + q1 + q2 + q3;
-    return (uint32_t)(q0 & 0xFF) | ((uint32_t)(q1 & 0xFF) << 8) | ((uint32_t)(q2 & 0xFF) << 16) |
-           ((uint32_t)(q3 & 0xFF) << 24);
-}
-
-// running max of |x| over 8 bf16 values, as fp32 bit patterns: for |x| the unsigned order is
-// the numeric order, and a NaN (bits above Inf) wins, so a non-finite row is still seen
-__device__ __forceinline__ uint32_t absmax8_bits(uint4 v, uint32_t m) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        m = max(m, (w[i] << 16) & 0x7FFFFFFFu);
-        m = max(m, w[i] & 0x7FFF0000u);
-    }
-    return m;
-}
-
 __device__ __forceinline__ void mma_s8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -93,7 +70,7 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(const __grid_constant__
     const DevDesc* descs = qa.descs;
     const int m = qa.m;
     uint32_t* err = qa.err;
-    extern __shared__ __align__(16) uint8_t smem_raw[];
+    extern __shared__ __align__(128) uint8_t smem_raw[];
     // let the dependent scaffold kernel start streaming weights right away;
     // it waits for this grid's results before reading them
     ptx::pdl_launch_dependents();

@@ -286,7 +286,8 @@ def test_single_projection_full(workload):
 
 
 @pytest.mark.parametrize("workload,samples", [("stack48_m1", 0), ("stack48_m4", 400), ("stack48_m16", 400),
-                                              ("stack48_m64", 300), ("stack48_m2048", 200)])
+                                              ("stack48_m64", 300), ("stack48_m512", 200),
+                                              ("stack48_m2048", 200)])
 def test_stack_full_size(workload, samples):
     # First the call exactly as bench.py makes it (bf16 y, no debug exports: for M = 2048 this
     # is the 16-byte row-piece store path of the tcgen05 epilogue), y checked against the
