@@ -68,6 +68,8 @@ PREFILL_CASES = [
     # items of 10 and of 5 tokens in the quantiser (32768 / d_in not a power of two), a final
     # half segment, a last row tile of 8 rows, ragged 192-token tiles
     (3200, 520, 300, BF16), (6144, 136, 70, BF16),
+    # 241 and 480 tokens: a second tile of 49 tokens; two whole tiles and half a third
+    (1024, 200, 241, F32), (512, 130, 480, BF16),
 ]
 
 
@@ -316,7 +318,9 @@ def test_stack_full_size(workload, samples):
 
 # bf16 output without debug exports and d_out % 8 == 0: the tcgen05 epilogue stores 16-byte row
 # pieces for whole 32-row groups and single elements for a last partial group; ragged token tiles
-BENCH_STORE_CASES = [(2048, 136, 200), (4096, 520, 400), (1024, 256, 385), (384, 40, 17), (8192, 64, 193)]
+# (192 tokens per tile, 96 per epilogue half; 241 and 480 reach a second and a third tile)
+BENCH_STORE_CASES = [(2048, 136, 200), (4096, 520, 400), (1024, 256, 385), (384, 40, 17), (8192, 64, 193),
+                     (2048, 256, 241), (1024, 128, 480)]
 
 
 @pytest.mark.parametrize("d_in,d_out,m", BENCH_STORE_CASES)
