@@ -66,7 +66,7 @@ constexpr int kThreads = kWarps * 32;
 #define DFSSM_DECODE_CHUNK_BYTES 128
 #endif
 #ifndef DFSSM_DECODE_STAGES
-#define DFSSM_DECODE_STAGES 3
+#define DFSSM_DECODE_STAGES 2
 #endif
 constexpr int kChunkBytes = DFSSM_DECODE_CHUNK_BYTES;   // sign bytes per row per k-chunk (8 columns per byte)
 constexpr int kGroups = kChunkBytes / 32;                // 256-column groups per chunk
@@ -715,8 +715,12 @@ bool encode_sign_map(CUtensorMap* map, const void* sign, int d_in, int d_out, in
 int decode_map_slots_per_sm() { return kMapSlots * kMaxCtasPerSm; }
 int decode_block_rows(int m) { return m <= 8 ? 128 : 64; }
 
-// The largest shared-memory carveout: three decode CTAs take about 196 KB, and the one-token slice
-// kernel's CTA (34 KB) fits beside them only if the SM is configured for 228 KB.
+// The largest shared-memory carveout. Registers allow three decode CTAs per SM; with two ring
+// slots three CTAs also fit in shared memory up to about 8 tokens (about 58 KB each at 4 tokens),
+// beside the one-token slice kernel's CTA (34 KB) at one token. A third slot would leave two CTAs
+// (8 warps) per SM from 2 tokens on, and the kernel is bound by issue latency, not by bytes in
+// flight: measured on the 48-layer stack, 2 slots take 4 tokens from 90.5 to 77.7 us and 16
+// tokens from 210 to 191 us, with one token unchanged (59.5 us).
 cudaError_t set_decode_attr(int optin) {
     cudaError_t e = allow_dyn_smem(decode_kernel<2, 1>, optin);
     if (e == cudaSuccess) e = allow_dyn_smem(decode_kernel<1, 2>, optin);
