@@ -7,8 +7,11 @@
 // the layer is bound by that weight stream. Here the bits never exist as int8
 // bytes in memory:
 //
-//  * Work: blocks of R = 64 * RT output rows (4 warps, RT 16-row tiles per
-//    warp), flattened over all linears of the call. Each CTA is persistent and
+//  * Work: blocks of R = 16 * RT * W output rows (W warps, RT 16-row tiles per
+//    warp): up to 8 tokens 4 warps x 2 tiles (128 rows, three CTAs per SM);
+//    9 to 16 tokens 12 warps x 1 tile (192 rows, one CTA per SM, so the 16
+//    tokens' activations are held once per SM), flattened over all linears of
+//    the call. Each CTA is persistent and
 //    owns a contiguous range of blocks holding an equal share of the work units
 //    (per k-chunk, per block epilogue and for entering a linear; dfssm_internal.cuh):
 //    CTA durations follow these units, not bytes (a partial last block costs
@@ -60,8 +63,7 @@ namespace dfssm {
 
 namespace {
 
-constexpr int kWarps = 4;
-constexpr int kThreads = kWarps * 32;
+constexpr int kMaxWarps = 12;      // warps per CTA: 4 (up to 8 tokens) or 12 (9 to 16 tokens)
 #ifndef DFSSM_DECODE_CHUNK_BYTES
 #define DFSSM_DECODE_CHUNK_BYTES 128
 #endif
@@ -97,7 +99,7 @@ struct DecodeArgs {
     int splits;
     int slices;              // 1: one token, partial h per kLoraSliceCols-column slice (lora_slice_kernel)
     int64_t total_units;     // decode work units of the n linears (dfssm_internal.cuh)
-    int ri;                  // which work_begin: 0 for 128-row blocks, 1 for 64-row blocks
+    int ri;                  // which work_begin: 0 for 128-row blocks, 1 for 192-row blocks
     int slot_bytes;          // bytes of one ring slot
     int q_region;            // bytes of the staged-q region
     // first (linear, block) of each CTA, found on the host (linear << 16 | block), so a CTA
@@ -208,9 +210,10 @@ struct DecCtl {
 // Fill a ring slot with k-chunk kc of block b: R rows x 128 sign bytes by one TMA load (thread 0),
 // plus alpha, s_A and W_A of the block (cp.async, all threads) when kc is its last chunk. Every
 // thread then arrives on the slot's barrier once its own copies have landed.
-template <int R>
+template <int R, int W>
 __device__ __forceinline__ void issue_step(const Cursor& c, const Lin& L, uint32_t slot_s, const CUtensorMap* map,
                                            uint64_t* full) {
+    constexpr int kThreads = W * 32;
     const int row0 = c.b * R;
     if (L.ok) {
         if (threadIdx.x == 0) {
@@ -267,15 +270,17 @@ __device__ __forceinline__ int q_pos(int gg, int i, int p) {
 struct TokShared {
     float sx[kMaxTok];
     int sumq[kMaxTok];
-    float red_f[kWarps][kMaxTok];
-    int red_i[kWarps][kMaxTok];
+    float red_f[kMaxWarps][kMaxTok];
+    int red_i[kMaxWarps][kMaxTok];
     float u[kMaxTok][kRank];
 };
 
 // Quantise the m x d_in activations of linear L into the permuted int8 layout
 // (token stride d_in + kTokPad), with per-token s_x and sum q. Same arithmetic
 // as the quantisation kernel (epilogue.cuh), so the same bytes.
+template <int W>
 __device__ void quantise_into_smem(const Lin& L, int m, uint8_t* q_s, TokShared& ts) {
+    constexpr int kWarps = W, kThreads = W * 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int n8 = L.d_in >> 3;                      // 8-column chunks per row
     const int qstride = q_stride(L.d_in);
@@ -327,9 +332,10 @@ __device__ void quantise_into_smem(const Lin& L, int m, uint8_t* q_s, TokShared&
     // (the caller synchronises before sumq is read)
 }
 
-template <int RT, int NT>
-__global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant__ DecodeArgs a) {
-    constexpr int R = 16 * RT * kWarps;
+template <int RT, int NT, int W>
+__global__ void __launch_bounds__(W * 32) decode_kernel(const __grid_constant__ DecodeArgs a) {
+    constexpr int kThreads = W * 32;
+    constexpr int R = 16 * RT * W;
     extern __shared__ __align__(1024) uint8_t smem[];
     // 1024-byte aligned ring first (the 128-byte swizzle of the TMA boxes repeats every 1 KB)
     uint8_t* ring = smem + ((1024u - (ptx::smem_u32(smem) & 1023u)) & 1023u);
@@ -382,7 +388,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
             map = linear_map(a, lw.L, lw.c.l, nmap, dc);
             map_lin = lw.c.l;
         }
-        issue_step<R>(lw.c, lw.L, ptx::smem_u32(ring + slot * a.slot_bytes), map, &dc.full[slot]);
+        issue_step<R, W>(lw.c, lw.L, ptx::smem_u32(ring + slot * a.slot_bytes), map, &dc.full[slot]);
         lw.advance(a);
     };
     int issued = 0;
@@ -407,7 +413,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
         const Lin& L = cw.L;
         if (cw.c.l != q_lin) {
             // a new linear: quantise its activations (its weights are already streaming)
-            if (L.ok) quantise_into_smem(L, m, q_s, ts);
+            if (L.ok) quantise_into_smem<W>(L, m, q_s, ts);
             q_lin = cw.c.l;
             __syncthreads();
         }
@@ -598,9 +604,9 @@ struct Geometry {
 // Ring slots of R x 128 sign bytes + the block's alpha, s_A, W_A, each a multiple of 1 KB (the
 // TMA swizzle pattern repeats every 1 KB); then the staged q, the per-token values and the
 // control block; 1 KB for aligning the base.
-template <int RT>
+template <int RT, int W>
 Geometry geometry(int m, int max_d_in) {
-    constexpr int R = 16 * RT * kWarps;
+    constexpr int R = 16 * RT * W;
     Geometry g;
     g.slot_bytes = (R * kChunkBytes + R * (4 + 4 + kRank) + 1023) & ~1023;
     g.q_region = (m * q_stride(max_d_in) + 127) & ~127;
@@ -609,11 +615,12 @@ Geometry geometry(int m, int max_d_in) {
     return g;
 }
 
-template <int RT, int NT>
+template <int RT, int NT, int W>
 cudaError_t launch_cfg(const LaunchCtx& c) {
-    constexpr int R = 16 * RT * kWarps;
-    const Geometry geo = geometry<RT>(c.m, c.max_d_in);
-    static_assert(R == 128 || R == 64, "work units exist for 128- and 64-row blocks");
+    constexpr int R = 16 * RT * W;
+    constexpr int kThreads = W * 32;
+    const Geometry geo = geometry<RT, W>(c.m, c.max_d_in);
+    static_assert(R == 128 || R == 192, "work units exist for 128- and 192-row blocks");
     static_assert(kChunkBytes * 8 == kDecodeChunkCols, "kUnitChunk work units per k-chunk");
     int64_t total_units = 0;
     int blocks = 0;
@@ -623,7 +630,7 @@ cudaError_t launch_cfg(const LaunchCtx& c) {
     }
     int per_sm = 0;
     cudaError_t err =
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<RT, NT>, kThreads, geo.smem);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<RT, NT, W>, kThreads, geo.smem);
     if (err != cudaSuccess) return err;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     if (per_sm > kMaxCtasPerSm) per_sm = kMaxCtasPerSm;     // the plan's map slots
@@ -687,14 +694,14 @@ cudaError_t launch_cfg(const LaunchCtx& c) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_kernel<RT, NT>, a);
+    return cudaLaunchKernelEx(&cfg, decode_kernel<RT, NT, W>, a);
 }
 
 }  // namespace
 
 cudaError_t launch_decode(const LaunchCtx& c) {
-    if (c.m <= 8) return launch_cfg<2, 1>(c);
-    return launch_cfg<1, 2>(c);
+    if (c.m <= 8) return launch_cfg<2, 1, 4>(c);
+    return launch_cfg<1, 2, 12>(c);
 }
 
 // The decode kernel's tensor map over a linear's sign rows: d_out rows of d_in / 8 bytes, boxes of
@@ -713,7 +720,7 @@ bool encode_sign_map(CUtensorMap* map, const void* sign, int d_in, int d_out, in
 }
 
 int decode_map_slots_per_sm() { return kMapSlots * kMaxCtasPerSm; }
-int decode_block_rows(int m) { return m <= 8 ? 128 : 64; }
+int decode_block_rows(int m) { return m <= 8 ? 128 : 192; }
 
 // The largest shared-memory carveout. Registers allow three decode CTAs per SM; with two ring
 // slots three CTAs also fit in shared memory up to about 8 tokens (about 58 KB each at 4 tokens),
@@ -722,13 +729,13 @@ int decode_block_rows(int m) { return m <= 8 ? 128 : 64; }
 // flight: measured on the 48-layer stack, 2 slots take 4 tokens from 90.5 to 77.7 us and 16
 // tokens from 210 to 191 us, with one token unchanged (59.5 us).
 cudaError_t set_decode_attr(int optin) {
-    cudaError_t e = allow_dyn_smem(decode_kernel<2, 1>, optin);
-    if (e == cudaSuccess) e = allow_dyn_smem(decode_kernel<1, 2>, optin);
+    cudaError_t e = allow_dyn_smem(decode_kernel<2, 1, 4>, optin);
+    if (e == cudaSuccess) e = allow_dyn_smem(decode_kernel<1, 2, 12>, optin);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(decode_kernel<2, 1>, cudaFuncAttributePreferredSharedMemoryCarveout,
+        e = cudaFuncSetAttribute(decode_kernel<2, 1, 4>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  cudaSharedmemCarveoutMaxShared);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(decode_kernel<1, 2>, cudaFuncAttributePreferredSharedMemoryCarveout,
+        e = cudaFuncSetAttribute(decode_kernel<1, 2, 12>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  cudaSharedmemCarveoutMaxShared);
     return e;
 }

@@ -50,7 +50,7 @@ struct dfssm_plan_s {
     uint32_t* err = nullptr;
     int* part = nullptr;
     CUtensorMap* tmaps = nullptr;       // prefill: activation rows of each linear
-    CUtensorMap* sign_tmpl = nullptr;   // decode: sign rows of each linear (placeholder address), 128- then 64-row boxes
+    CUtensorMap* sign_tmpl = nullptr;   // decode: sign rows of each linear (placeholder address), 128- then 192-row boxes
     CUtensorMap* map_slots = nullptr;   // decode: per-CTA slots for the device-edited sign maps
     uint64_t wait_limit_ns = kWaitLimitNs;
     int stall_test = 0;
@@ -158,7 +158,7 @@ dfssm_status dfssm_linear_plan(const dfssm_linear_desc* descs, int n_descs, dfss
     }
     p->n = n_descs;
     p->hdesc.resize(n_descs);
-    int64_t q_bytes = 0, st_count = 0, units128 = 0, units64 = 0;
+    int64_t q_bytes = 0, st_count = 0, units128 = 0, units192 = 0;
     int32_t rt = 0;
     for (int i = 0; i < n_descs; ++i) {
         DevDesc& d = p->hdesc[i];
@@ -174,9 +174,9 @@ dfssm_status dfssm_linear_plan(const dfssm_linear_desc* descs, int n_descs, dfss
         d.st_off = st_count;
         d.rt_begin = rt;
         d.work_begin[0] = units128;
-        d.work_begin[1] = units64;
+        d.work_begin[1] = units192;
         units128 += decode_units(d.d_in, d.d_out, 128);
-        units64 += decode_units(d.d_in, d.d_out, 64);
+        units192 += decode_units(d.d_in, d.d_out, 192);
         st_count += d.max_m;
         rt += (d.d_out + 127) / 128;
     }

@@ -33,7 +33,7 @@ struct DevDesc {
     int64_t st_off;     // index of its first TokStats record
     int32_t qrow;       // activation bytes per token: d_in rounded up to a whole 256-column segment
     int32_t rt_begin;   // first 128-row tile of this linear in the flattened stack order
-    int64_t work_begin[2]; // decode work units of all preceding linears, for 128- and 64-row blocks
+    int64_t work_begin[2]; // decode work units of all preceding linears, for 128- and 192-row blocks
 };
 
 // Per-token values the main kernels need after quantisation.
