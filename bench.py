@@ -63,24 +63,37 @@ def load_peaks():
     return dict(hbm=FALLBACK_HBM_GBS, bf16=FALLBACK_BF16_TFLOPS, bf16_sustained=1400.0, src="fallback")
 
 
-def kernel_source_hash():
+# The source files each measured kernel is built from (its .cu, the shared device headers and the
+# host code that fixes its launch); a traffic record stays valid while these files are unchanged.
+KERNEL_SOURCES = {
+    "decode_kernel": ["decode.cu", "quant.cu", "epilogue.cuh", "ptx.cuh", "dfssm_internal.cuh", "dfssm_api.cu"],
+    "prefill_kernel": ["prefill.cu", "quant_rows.cu", "epilogue.cuh", "ptx.cuh", "dfssm_internal.cuh",
+                       "dfssm_api.cu"],
+    "lm_head_kernel": ["int8_table.cu", "epilogue.cuh", "ptx.cuh", "dfssm_internal.cuh", "dfssm_api.cu"],
+}
+
+
+def kernel_source_hash(names=None):
+    """sha256 (16 hex digits) over the named files of the library's csrc/ (all of them by default)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_gemv_gemm_dfssm_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(names if names is not None else os.listdir(csrc)):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(workload):
-    """DRAM bytes per call from the committed ncu summary, if taken on the current kernels."""
+    """DRAM bytes per call from the committed ncu summary, if its kernel's sources are unchanged."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         j = json.load(f)
     rec = j.get(workload)
-    if not rec or rec.get("kernel_source_hash") != kernel_source_hash():
+    if not rec or rec.get("kernel") not in KERNEL_SOURCES:
+        return None
+    if rec.get("kernel_source_hash") != kernel_source_hash(KERNEL_SOURCES[rec["kernel"]]):
         return None
     return rec.get("dram_bytes_per_call")
 
@@ -456,7 +469,8 @@ def lm_head_block(torch, seed, peaks, dev, m=1, steps=200):
     nb = vocab * d + 4 * vocab + 2 * m * d + 2 * m * vocab
     return {"workload": f"lm_head_m{m}", "vocab": vocab, "d": d, "m": m, "us_per_call": us,
             "GB/s": nb / (us * 1e-6) / 1e9, "hbm_frac": nb / (us * 1e-6) / 1e9 / peaks["hbm"],
-            "bytes_per_call": nb, "l2": "two 103 MB tables alternated"}
+            "bytes_per_call": nb, "l2": "two 103 MB tables alternated",
+            "traffic": recorded_traffic(f"lm_head_m{m}")}
 
 
 def timed_device(torch, run_step, steps, warmup, dist, dev):

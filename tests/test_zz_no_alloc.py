@@ -52,6 +52,18 @@ def test_noalloc_matches_plan_entry_point_twice():
         check_linear_full(lin)          # lin.dy holds the no-allocation call's output
 
 
+def test_noalloc_allocates_no_device_memory():
+    # after the first call (the per-device set-up), repeated calls leave the device's free memory
+    # unchanged
+    lin = Linear(0x5EED, 9, 600, 2048, 640, 3, dfssm.DFSSM_BF16, dbg=False)
+    run_noalloc(lin)
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(5):
+        run_noalloc(lin)
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+
+
 def test_noalloc_refuses_sizes_beyond_its_limits():
     lin = Linear(7, 9, 1, 256, 64, 1, dfssm.DFSSM_F32, dbg=False)
     too_many = dfssm.LinearDesc(256, 64, dfssm.RANK, 32, dfssm.DFSSM_F32, 0)
