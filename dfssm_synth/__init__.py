@@ -31,6 +31,8 @@ N_LAYERS = 48
 
 # tensor ids inside a stream
 T_X, T_COLS, T_SIGN, T_ALPHA, T_WA, T_SA, T_WB, T_SB, T_TABLE, T_TSCALE, T_IDS = range(11)
+(T_ZXBCDT, T_CONV_STATE, T_SSM_STATE, T_CONV_W, T_CONV_B, T_DT_BIAS, T_A_LOG, T_D_SKIP,
+ T_NORM_W) = range(11, 20)
 KIND_WEIGHTS, KIND_ACT = 1, 2
 # the tied int8 embedding / LM-head table of Mamba-2 1.3B: its 50,277-token vocabulary padded to
 # a multiple of 16, d_model columns
@@ -64,6 +66,7 @@ def _L():
         lib.dfssm_synth_bits.argtypes = [u64, i64, vp]
         lib.dfssm_synth_uniform_f32.argtypes = [u64, i64, dbl, dbl, vp]
         lib.dfssm_synth_int8_sym127.argtypes = [u64, i64, vp]
+        lib.dfssm_synth_normal.argtypes = [u64, i64, dbl, ctypes.c_int, vp]
         lib.dfssm_synth_f64_to_bf16.restype = ctypes.c_uint16
         lib.dfssm_synth_f64_to_bf16.argtypes = [dbl]
         _lib = lib
@@ -152,6 +155,48 @@ def token_ids(seed: int, cfg: int, m: int, vocab: int) -> np.ndarray:
     """m token ids drawn uniformly from [0, vocab)."""
     r = raw(seed, stream_id(KIND_ACT, cfg, m, 0, T_IDS), 0, m)
     return (r % np.uint64(vocab)).astype(np.int32)
+
+
+# The Mamba-2 1.3B state operations between in_proj and out_proj: d_inner = 2 d_model, 64 heads of
+# 64 channels, d_state 128 (one group of B and C), a 4-tap causal convolution, RMS-norm eps 1e-5.
+SSM_DIMS = dict(d_inner=4096, headdim=64, d_state=128, d_conv=4, eps=1e-5)
+
+
+def ssm_layer_inputs(seed: int, cfg: int, index: int, m: int, dims=None) -> dict:
+    """One layer's decode-step inputs for m tokens (inputs only; the state operations themselves
+    are in the oracle and the library). zxbcdt ~ N(0,1) and conv_state ~ N(0,1) as bf16 bits,
+    ssm_state ~ N(0, 0.5^2) fp32; conv_w ~ U(-0.5, 0.5), conv_b ~ U(-0.1, 0.1); the step size at
+    initialisation dt0 ~ U(0.001, 0.1) gives dt_bias = log(expm1(dt0)) (so softplus(dt_bias) = dt0);
+    a_log = log(U(1, 16)); d_skip, norm_w ~ U(0.5, 1.5) (all fp32)."""
+    d = dims or SSM_DIMS
+    d_inner, headdim, d_state, d_conv = d["d_inner"], d["headdim"], d["d_state"], d["d_conv"]
+    nheads = d_inner // headdim
+    conv_dim = d_inner + 2 * d_state
+    row = 2 * d_inner + 2 * d_state + nheads
+    L = _L()
+
+    def k_(kind, t):
+        return key(seed, stream_id(kind, cfg, m if kind == KIND_ACT else 0, index, t))
+
+    out = dict(zxbcdt=np.empty((m, row), np.uint16), conv_state=np.empty((m, conv_dim, d_conv), np.uint16),
+               ssm_state=np.empty((m, nheads, headdim, d_state), np.float32),
+               conv_w=np.empty((conv_dim, d_conv), np.float32), conv_b=np.empty(conv_dim, np.float32),
+               dt_bias=np.empty(nheads, np.float32), a_log=np.empty(nheads, np.float32),
+               d_skip=np.empty(nheads, np.float32), norm_w=np.empty(d_inner, np.float32))
+    L.dfssm_synth_normal(k_(KIND_ACT, T_ZXBCDT), out["zxbcdt"].size, 1.0, 1, _ptr(out["zxbcdt"]))
+    L.dfssm_synth_normal(k_(KIND_ACT, T_CONV_STATE), out["conv_state"].size, 1.0, 1, _ptr(out["conv_state"]))
+    L.dfssm_synth_normal(k_(KIND_ACT, T_SSM_STATE), out["ssm_state"].size, 0.5, 0, _ptr(out["ssm_state"]))
+    L.dfssm_synth_uniform_f32(k_(KIND_WEIGHTS, T_CONV_W), out["conv_w"].size, -0.5, 0.5, _ptr(out["conv_w"]))
+    L.dfssm_synth_uniform_f32(k_(KIND_WEIGHTS, T_CONV_B), conv_dim, -0.1, 0.1, _ptr(out["conv_b"]))
+    dt0 = np.empty(nheads, np.float32)
+    L.dfssm_synth_uniform_f32(k_(KIND_WEIGHTS, T_DT_BIAS), nheads, 0.001, 0.1, _ptr(dt0))
+    out["dt_bias"][:] = np.log(np.expm1(dt0.astype(np.float64))).astype(np.float32)
+    a = np.empty(nheads, np.float32)
+    L.dfssm_synth_uniform_f32(k_(KIND_WEIGHTS, T_A_LOG), nheads, 1.0, 16.0, _ptr(a))
+    out["a_log"][:] = np.log(a.astype(np.float64)).astype(np.float32)
+    L.dfssm_synth_uniform_f32(k_(KIND_WEIGHTS, T_D_SKIP), nheads, 0.5, 1.5, _ptr(out["d_skip"]))
+    L.dfssm_synth_uniform_f32(k_(KIND_WEIGHTS, T_NORM_W), d_inner, 0.5, 1.5, _ptr(out["norm_w"]))
+    return out
 
 
 def stack_shapes(n_layers: int = N_LAYERS):

@@ -129,5 +129,18 @@ void dfssm_synth_int8_sym127(uint64_t key, int64_t n, int8_t* out) {
     }
 }
 
+/* n normals z ~ N(0,1) (Box-Muller in f64, two draws each) times `scale`, rounded once to fp32
+   (bf16 = 0) or to bf16 bits (bf16 = 1). */
+void dfssm_synth_normal(uint64_t key, int64_t n, double scale, int bf16, void* out) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        double u1 = ((double)(draw(key, 2 * (uint64_t)i) >> 11) + 1.0) * 0x1.0p-53; /* (0,1] */
+        double u2 = u01(draw(key, 2 * (uint64_t)i + 1));
+        double z = scale * sqrt(-2.0 * log(u1)) * cos(6.283185307179586 * u2);
+        if (bf16) ((uint16_t*)out)[i] = f64_to_bf16_rne(z);
+        else ((float*)out)[i] = (float)z;
+    }
+}
+
 /* Exposed for the generator's own tests (bf16 rounding of the x draws). */
 uint16_t dfssm_synth_f64_to_bf16(double v) { return f64_to_bf16_rne(v); }

@@ -20,15 +20,17 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "dfssm_oracle.cpp")
+_SRCS = [_SRC, os.path.join(_HERE, "ssm_oracle.cpp")]
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 
 
 def build(force: bool = False) -> str:
     """Compile the oracle with g++ (no fast-math, no FMA contraction, OpenMP)."""
-    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+    if force or not os.path.exists(_LIB_PATH) or any(os.path.getmtime(_LIB_PATH) < os.path.getmtime(f)
+                                                     for f in _SRCS):
         tmp = _LIB_PATH + f".tmp{os.getpid()}"
         subprocess.check_call(["g++", "-O2", "-fPIC", "-shared", "-fopenmp", "-std=c++17",
-                               "-ffp-contract=off", "-fno-fast-math", "-o", tmp, _SRC])
+                               "-ffp-contract=off", "-fno-fast-math", "-o", tmp, *_SRCS])
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
 
@@ -58,6 +60,8 @@ def _L():
         lib.dfssm_oracle_embed.restype = i32
         lib.dfssm_oracle_embed.argtypes = [vp, vp, i32, i32, vp, i32, vp]
         lib.dfssm_oracle_lm_head.argtypes = [vp, vp, i32, i32, vp, i32, vp, vp, i32]
+        lib.dfssm_oracle_ssm_step.argtypes = [i32, i32, i32, i32, dbl, i32, vp, vp, vp, vp, vp, vp, vp, vp,
+                                              vp, vp, vp, vp, vp, vp, vp, vp]
         lib.dfssm_oracle_lm_head_sampled.argtypes = [vp, vp, i32, i32, vp, i32, vp, vp, i64, vp, vp]
         _lib = lib
     return _lib
@@ -199,3 +203,35 @@ def lm_head_sampled(table, scale, h_bf16_bits, m: int, t_idx, v_idx):
     _L().dfssm_oracle_lm_head_sampled(ptb, psc, vocab, d, ph, m, pt, pv, t.size, acc.ctypes.data,
                                       logits.ctypes.data)
     return dict(acc=acc, logits=logits)
+
+
+def ssm_step(dims, inp):
+    """One decode step of the Mamba-2 state operations for one layer (ssm_oracle.cpp).
+
+    dims: dict(d_inner, headdim, d_state, d_conv, eps). inp: dict with zxbcdt (m x row, bf16
+    bits), conv_state (m x conv_dim x d_conv, bf16 bits), ssm_state (m x nheads x headdim x
+    d_state, float32), conv_w (conv_dim x d_conv), conv_b, dt_bias, a_log, d_skip, norm_w
+    (float32). The inputs are not modified. Returns float64 ssm_state and out, the new
+    conv_state (bf16 bits) and the intermediates xc, dt, dA, y (before the gate) and r."""
+    d_inner, headdim, d_state, d_conv = dims["d_inner"], dims["headdim"], dims["d_state"], dims["d_conv"]
+    nheads = d_inner // headdim
+    conv_dim = d_inner + 2 * d_state
+    z, pz = _c(inp["zxbcdt"], np.uint16)
+    m = z.shape[0]
+    assert z.shape == (m, 2 * d_inner + 2 * d_state + nheads)
+    cs = np.array(inp["conv_state"], dtype=np.uint16, copy=True, order="C")
+    assert cs.shape == (m, conv_dim, d_conv)
+    s_in, ps = _c(inp["ssm_state"], np.float32)
+    assert s_in.shape == (m, nheads, headdim, d_state)
+    par = [_c(inp[k], np.float32) for k in ("conv_w", "conv_b", "dt_bias", "a_log", "d_skip", "norm_w")]
+    s_out = np.empty(s_in.shape, np.float64)
+    out = np.empty((m, d_inner), np.float64)
+    xc = np.empty((m, conv_dim), np.float64)
+    dt = np.empty((m, nheads), np.float64)
+    dA = np.empty((m, nheads), np.float64)
+    y = np.empty((m, d_inner), np.float64)
+    r = np.empty(m, np.float64)
+    _L().dfssm_oracle_ssm_step(d_inner, headdim, d_state, d_conv, float(dims["eps"]), m, pz, cs.ctypes.data, ps,
+                               s_out.ctypes.data, *[p for _, p in par], out.ctypes.data, xc.ctypes.data,
+                               dt.ctypes.data, dA.ctypes.data, y.ctypes.data, r.ctypes.data)
+    return dict(ssm_state=s_out, out=out, conv_state=cs, xc=xc, dt=dt, dA=dA, y=y, r=r)
