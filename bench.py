@@ -70,6 +70,7 @@ KERNEL_SOURCES = {
     "prefill_kernel": ["prefill.cu", "quant_rows.cu", "epilogue.cuh", "ptx.cuh", "dfssm_internal.cuh",
                        "dfssm_api.cu"],
     "lm_head_kernel": ["int8_table.cu", "epilogue.cuh", "ptx.cuh", "dfssm_internal.cuh", "dfssm_api.cu"],
+    "ssm_scan_kernel": ["ssm_step.cu", "epilogue.cuh", "dfssm_internal.cuh"],
 }
 
 
@@ -473,6 +474,57 @@ def lm_head_block(torch, seed, peaks, dev, m=1, steps=200):
             "traffic": recorded_traffic(f"lm_head_m{m}")}
 
 
+def ssm_block(torch, seed, peaks, dev, n_layers=48, m=1, steps=200):
+    """The decode step of the state operations (shift register + SSM recurrence) for the 48 layers
+    of Mamba-2 1.3B at m tokens: two full sets of inputs and states alternated (2 x 208 MB > L2),
+    one CUDA graph per call."""
+    import bit_gemv_gemm_dfssm_b200 as dfssm
+    dims = synth.SSM_DIMS
+    d_inner, N, conv = dims["d_inner"], dims["d_state"], dims["d_conv"]
+    nheads = d_inner // dims["headdim"]
+    conv_dim = d_inner + 2 * N
+    c = dfssm.SsmDims(d_inner, dims["headdim"], N, conv, dims["eps"], dfssm.DFSSM_BF16)
+    keep, ldevs = [], []
+    for s in range(2):
+        layers = []
+        for i in range(n_layers):
+            inp = synth.ssm_layer_inputs(seed + s, 10, i, m, dims)
+            d = {k: (torch.from_numpy(v.view(np.int16).copy()) if v.dtype == np.uint16 else torch.from_numpy(v)).cuda()
+                 for k, v in inp.items()}
+            d["out"] = torch.empty((m, d_inner), dtype=torch.bfloat16, device="cuda")
+            keep.append(d)
+            layers.append(dfssm.SsmLayer(*[d[k].data_ptr() for k in ("zxbcdt", "conv_state", "ssm_state", "conv_w",
+                                                                       "conv_b", "dt_bias", "a_log", "d_skip",
+                                                                       "norm_w", "out")]))
+        ldevs.append(torch.frombuffer(bytearray(dfssm.ssm_layers_bytes(layers)), dtype=torch.uint8).cuda())
+    wsb = dfssm.dfssm_ssm_workspace_bytes(c, n_layers, m)
+    ws = torch.zeros(wsb // 4 + 64, dtype=torch.int32, device="cuda")
+    side = torch.cuda.Stream()
+    gs = []
+    for ld in ldevs:
+        side.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            dfssm.dfssm_ssm_step(c, ld.data_ptr(), n_layers, m, ws.data_ptr(), wsb, torch.cuda.current_stream().cuda_stream)
+        gs.append(g)
+    torch.cuda.synchronize()
+    ms = timed_device(torch, lambda i: gs[i % 2].replay(), steps, 3, None, dev)
+    st, bits = dfssm.dfssm_ssm_read_error(ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    assert st == dfssm.DFSSM_OK, hex(bits)
+    del gs
+    us = ms * 1e3 / steps
+    per_layer = m * (2 * (2 * d_inner + 2 * N + nheads)        # zxbcdt (bf16) in
+                     + 2 * 2 * conv_dim * conv                  # shift register (bf16) in and out
+                     + 2 * 4 * nheads * dims["headdim"] * N     # SSM state (fp32) in and out
+                     + 2 * d_inner) \
+        + 4 * (conv_dim * conv + conv_dim + 3 * nheads + d_inner)   # parameters (fp32)
+    nb = n_layers * per_layer
+    return {"workload": f"ssm_step{n_layers}_m{m}", "m": m, "layers": n_layers, "us_per_step": us,
+            "GB/s": nb / (us * 1e-6) / 1e9, "hbm_frac": nb / (us * 1e-6) / 1e9 / peaks["hbm"],
+            "bytes_per_step": nb, "tokens_per_s": m / (us * 1e-6), "gpu_launches_per_step": 3,
+            "l2": "two sets of inputs and states alternated", "traffic": recorded_traffic(f"ssm_step{n_layers}_m{m}")}
+
+
 def timed_device(torch, run_step, steps, warmup, dist, dev):
     for i in range(warmup):
         run_step(i)
@@ -576,10 +628,10 @@ def run_gpu(args, wl_name):
         del pgraphs
 
     # the other configurations: single projections (cold L2), the stack at M = 4 / 16 / 64 / 512,
-    # the int8 LM head (every rank runs the same blocks; rank 0 reports them)
+    # the int8 LM head, the decode step of the state operations (every rank runs the same blocks; rank 0
     extras = None
     if not args.no_extras:
-        extras = {"single": [], "stacks": [], "lm_head": None}
+        extras = {"single": [], "stacks": [], "lm_head": None, "ssm_step": None}
         for wn in ("out_proj_m1", "in_proj_m1"):
             extras["single"].append(single_block(torch, wn, seed, peaks, dev))
         sets = device_weight_sets(synth.stack_shapes(), 2, seed)
@@ -588,6 +640,8 @@ def run_gpu(args, wl_name):
         del sets
         torch.cuda.empty_cache()
         extras["lm_head"] = lm_head_block(torch, seed, peaks, dev)
+        torch.cuda.empty_cache()
+        extras["ssm_step"] = ssm_block(torch, seed, peaks, dev)
 
     if rank != 0:
         if dist is not None:

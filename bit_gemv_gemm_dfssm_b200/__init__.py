@@ -42,6 +42,7 @@ EXPORTS = (
     "dfssm_linear_plan", "dfssm_plan_destroy", "dfssm_pack_sign", "dfssm_linear_fwd",
     "dfssm_linear_stack_fwd", "dfssm_plan_check", "dfssm_plan_workspace_bytes", "dfssm_status_string",
     "dfssm_linear_fwd_noalloc", "dfssm_plan_set_test_hooks", "dfssm_embed_fwd", "dfssm_lm_head_fwd",
+    "dfssm_ssm_workspace_bytes", "dfssm_ssm_step", "dfssm_ssm_read_error",
 )
 DFSSM_DEVERR_TOKEN_ID = 0x10
 DFSSM_TEST_STALL = 0x1
@@ -82,6 +83,18 @@ class Int8Table(ctypes.Structure):
                 ("d", ctypes.c_int32)]
 
 
+class SsmDims(ctypes.Structure):
+    _fields_ = [("d_inner", ctypes.c_int32), ("headdim", ctypes.c_int32), ("d_state", ctypes.c_int32),
+                ("d_conv", ctypes.c_int32), ("eps", ctypes.c_float), ("out_dtype", ctypes.c_int32)]
+
+
+class SsmLayer(ctypes.Structure):
+    _fields_ = [("zxbcdt", ctypes.c_void_p), ("conv_state", ctypes.c_void_p), ("ssm_state", ctypes.c_void_p),
+                ("conv_w", ctypes.c_void_p), ("conv_b", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p),
+                ("a_log", ctypes.c_void_p), ("d_skip", ctypes.c_void_p), ("norm_w", ctypes.c_void_p),
+                ("out", ctypes.c_void_p)]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"libdfssm.so is not built ({LIB_PATH}); run "
@@ -101,6 +114,9 @@ def _load():
     lib.dfssm_plan_set_test_hooks.argtypes = [vp, ctypes.c_uint64, ctypes.c_uint32]
     lib.dfssm_embed_fwd.argtypes = [ctypes.POINTER(Int8Table), vp, i32, vp, i32, vp, vp]
     lib.dfssm_lm_head_fwd.argtypes = [ctypes.POINTER(Int8Table), vp, i32, vp, i32, vp, vp]
+    lib.dfssm_ssm_workspace_bytes.argtypes = [ctypes.POINTER(SsmDims), i32, i32, ctypes.POINTER(ctypes.c_size_t)]
+    lib.dfssm_ssm_step.argtypes = [ctypes.POINTER(SsmDims), vp, i32, i32, vp, ctypes.c_size_t, vp]
+    lib.dfssm_ssm_read_error.argtypes = [vp, u32p, vp]
     lib.dfssm_status_string.restype = ctypes.c_char_p
     lib.dfssm_status_string.argtypes = [ctypes.c_int]
     for name in EXPORTS:
@@ -212,4 +228,33 @@ def weights_struct(sign, alpha, wa, sa, wb, sb) -> LinearWeights:
 def stack_entries_bytes(entries) -> bytes:
     """Pack a list of StackEntry into the byte image the device array must hold."""
     arr = (StackEntry * len(entries))(*entries)
+    return ctypes.string_at(ctypes.addressof(arr), ctypes.sizeof(arr))
+
+
+def dfssm_ssm_workspace_bytes(dims: SsmDims, n_layers: int, m: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().dfssm_ssm_workspace_bytes(ctypes.byref(dims), n_layers, m, ctypes.byref(n)),
+           "dfssm_ssm_workspace_bytes")
+    return n.value
+
+
+def dfssm_ssm_step(dims: SsmDims, layers_dev_ptr: int, n_layers: int, m: int, workspace_ptr: int,
+                   workspace_bytes: int, stream: int = 0) -> None:
+    """One decode step of the state operations for n_layers layers (see include/dfssm.h)."""
+    _check(lib().dfssm_ssm_step(ctypes.byref(dims), layers_dev_ptr, n_layers, m, workspace_ptr, workspace_bytes,
+                                stream), "dfssm_ssm_step")
+
+
+def dfssm_ssm_read_error(workspace_ptr: int, stream: int = 0):
+    """(status, bits) of the workspace's device error word, which is cleared."""
+    bits = ctypes.c_uint32(0)
+    st = lib().dfssm_ssm_read_error(workspace_ptr, ctypes.byref(bits), stream)
+    if st not in (DFSSM_OK, DFSSM_ERR_DEVICE_CHECK):
+        raise DfssmError(st, "dfssm_ssm_read_error")
+    return st, bits.value
+
+
+def ssm_layers_bytes(layers) -> bytes:
+    """Pack a list of SsmLayer into the byte image the device array must hold."""
+    arr = (SsmLayer * len(layers))(*layers)
     return ctypes.string_at(ctypes.addressof(arr), ctypes.sizeof(arr))

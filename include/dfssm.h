@@ -220,6 +220,66 @@ dfssm_status dfssm_embed_fwd(const dfssm_int8_table* table, const int32_t* ids, 
 dfssm_status dfssm_lm_head_fwd(const dfssm_int8_table* table, const void* h, int32_t m, void* logits,
                                int32_t out_dtype, int32_t* acc, void* stream);
 
+/* ---- decode step of the state operations between in_proj and out_proj -------------------
+ * "Density Field State Space Models" (gist.science technical summary), §2.C, state
+ * operations: the state shift register (causal convolution) and the SSM recurrence. The
+ * step is Mamba-2's, for one group of B and C:
+ *   in_proj output per token: [ z (d_inner) | xBC (conv_dim) | dt_raw (nheads) ],
+ *     conv_dim = d_inner + 2 d_state, nheads = d_inner / headdim;
+ *   shift register: window = (state[c][1..d_conv-1], xBC[c]) becomes the new state[c];
+ *   xc[c] = silu(conv_b[c] + sum_k conv_w[c][k] window[k]); x, B, C = xc split;
+ *   dt = softplus(dt_raw + dt_bias) (v itself above 20), dA = exp(-exp(a_log) dt);
+ *   S[h][p][n] = S[h][p][n] dA_h + dt_h x[h headdim + p] B[n];
+ *   y = sum_n S C[n] + d_skip_h x;  g = y silu(z);  out = g / sqrt(mean(g^2) + eps) norm_w.
+ * Supported: headdim 64, d_state 128, d_conv 4, d_inner a multiple of 64 up to 16384. */
+typedef struct {
+    int32_t d_inner;
+    int32_t headdim;    /* 64 */
+    int32_t d_state;    /* 128 */
+    int32_t d_conv;     /* 4 */
+    float eps;          /* RMS-norm epsilon (Mamba-2: 1e-5) */
+    int32_t out_dtype;  /* DFSSM_BF16 or DFSSM_F32 */
+} dfssm_ssm_dims;
+
+/* One layer (this struct lives in DEVICE memory for dfssm_ssm_step). Device pointers,
+ * 16-byte aligned (zxbcdt: 2-byte aligned), caller-owned:
+ *   zxbcdt     m x (2 d_inner + 2 d_state + nheads) bf16, row-major: the in_proj output;
+ *   conv_state m x conv_dim x d_conv bf16, updated in place;
+ *   ssm_state  m x nheads x headdim x d_state fp32, updated in place;
+ *   conv_w     conv_dim x d_conv fp32; conv_b conv_dim fp32;
+ *   dt_bias, a_log, d_skip  nheads fp32 each; norm_w d_inner fp32;
+ *   out        m x d_inner of out_dtype: the out_proj input. */
+typedef struct {
+    const void* zxbcdt;
+    void* conv_state;
+    float* ssm_state;
+    const float* conv_w;
+    const float* conv_b;
+    const float* dt_bias;
+    const float* a_log;
+    const float* d_skip;
+    const float* norm_w;
+    void* out;
+} dfssm_ssm_layer;
+
+/* Bytes of caller-owned device workspace one dfssm_ssm_step call of this shape needs. */
+dfssm_status dfssm_ssm_workspace_bytes(const dfssm_ssm_dims* dims, int32_t n_layers, int32_t m, size_t* bytes);
+
+/* One decode step for n_layers independent layers (layers_dev: DEVICE array of n_layers
+ * dfssm_ssm_layer) and m tokens each, on `stream`: three kernels (shift register and
+ * convolution; recurrence, readout and gate; RMS norm). workspace: 256-byte aligned, at
+ * least dfssm_ssm_workspace_bytes; its first 4 bytes are a device error word (zero it once
+ * before the first call) that gets DFSSM_DEVERR_ENTRY_PTR when a layer holds a NULL or
+ * misaligned pointer (that layer is skipped); read and clear it with dfssm_ssm_read_error.
+ * Calls sharing a workspace must be ordered. Allocates nothing. Argument errors return
+ * synchronously with no launch. */
+dfssm_status dfssm_ssm_step(const dfssm_ssm_dims* dims, const dfssm_ssm_layer* layers_dev, int32_t n_layers,
+                            int32_t m, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronise `stream`, return the workspace's error word in *bits and clear it;
+ * DFSSM_ERR_DEVICE_CHECK if it was set. */
+dfssm_status dfssm_ssm_read_error(void* workspace, uint32_t* bits, void* stream);
+
 /* Test of the error path of the decode kernel (m <= 16 tokens), which must end with an
  * error status and never hang. With flags & DFSSM_TEST_STALL, the first CTA of that
  * kernel waits on a barrier that nothing arrives on: the wait gives up after

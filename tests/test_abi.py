@@ -42,9 +42,10 @@ def test_struct_layout_matches_c(tmp_path):
 #include <stddef.h>
 #include "{HEADER}"
 int main(void) {{
-  printf("%zu %zu %zu %zu %zu %zu %zu\\n", sizeof(dfssm_linear_desc), sizeof(dfssm_linear_weights),
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\\n", sizeof(dfssm_linear_desc), sizeof(dfssm_linear_weights),
          sizeof(dfssm_debug), sizeof(dfssm_stack_entry), offsetof(dfssm_stack_entry, x),
-         offsetof(dfssm_stack_entry, dbg), offsetof(dfssm_stack_entry, desc_index));
+         offsetof(dfssm_stack_entry, dbg), offsetof(dfssm_stack_entry, desc_index), sizeof(dfssm_ssm_dims),
+         sizeof(dfssm_ssm_layer), offsetof(dfssm_ssm_layer, out));
   return 0;
 }}''')
     exe = tmp_path / "layout"
@@ -52,7 +53,8 @@ int main(void) {{
     got = [int(v) for v in subprocess.check_output([str(exe)]).split()]
     S = dfssm.StackEntry
     assert got == [ctypes.sizeof(dfssm.LinearDesc), ctypes.sizeof(dfssm.LinearWeights), ctypes.sizeof(dfssm.Debug),
-                   ctypes.sizeof(S), S.x.offset, S.dbg.offset, S.desc_index.offset]
+                   ctypes.sizeof(S), S.x.offset, S.dbg.offset, S.desc_index.offset, ctypes.sizeof(dfssm.SsmDims),
+                   ctypes.sizeof(dfssm.SsmLayer), dfssm.SsmLayer.out.offset]
 
 
 def test_argument_errors_without_gpu():
@@ -70,6 +72,19 @@ def test_argument_errors_without_gpu():
     assert lib.dfssm_linear_stack_fwd(None, None, 1, 1, None) == dfssm.DFSSM_ERR_INVALID_ARG
     assert lib.dfssm_pack_sign(None, dfssm.DFSSM_I8, 1, 128, None, None) == dfssm.DFSSM_ERR_INVALID_ARG
     assert lib.dfssm_plan_destroy(None) == dfssm.DFSSM_OK
+    # the state step: unsupported shapes and missing buffers return before any CUDA call
+    dims = dfssm.SsmDims(4096, 64, 128, 4, 1e-5, dfssm.DFSSM_BF16)
+    assert dfssm.dfssm_ssm_workspace_bytes(dims, 48, 1) > 48 * 4352 * 4
+    for bad in (dfssm.SsmDims(4096, 32, 128, 4, 1e-5, 0), dfssm.SsmDims(4096, 64, 64, 4, 1e-5, 0),
+                dfssm.SsmDims(4096, 64, 128, 3, 1e-5, 0), dfssm.SsmDims(4100, 64, 128, 4, 1e-5, 0)):
+        n = ctypes.c_size_t(0)
+        assert lib.dfssm_ssm_workspace_bytes(ctypes.byref(bad), 1, 1, ctypes.byref(n)) == \
+            dfssm.DFSSM_ERR_UNSUPPORTED_SHAPE
+    nan_eps = dfssm.SsmDims(4096, 64, 128, 4, float("nan"), 0)
+    n = ctypes.c_size_t(0)
+    assert lib.dfssm_ssm_workspace_bytes(ctypes.byref(nan_eps), 1, 1, ctypes.byref(n)) == dfssm.DFSSM_ERR_INVALID_ARG
+    assert lib.dfssm_ssm_step(ctypes.byref(dims), None, 1, 1, None, 0, None) == dfssm.DFSSM_ERR_INVALID_ARG
+    assert lib.dfssm_ssm_step(ctypes.byref(dims), 256, 1, 1, 4096, 16, None) == dfssm.DFSSM_ERR_INVALID_ARG
     assert dfssm.dfssm_status_string(dfssm.DFSSM_ERR_CUDA) == "CUDA error"
     with pytest.raises(dfssm.DfssmError):
         dfssm.dfssm_linear_plan([(100, 10, 1, 0)])
