@@ -70,7 +70,7 @@ KERNEL_SOURCES = {
     "prefill_kernel": ["prefill.cu", "quant_rows.cu", "epilogue.cuh", "ptx.cuh", "dfssm_internal.cuh",
                        "dfssm_api.cu"],
     "lm_head_kernel": ["int8_table.cu", "epilogue.cuh", "ptx.cuh", "dfssm_internal.cuh", "dfssm_api.cu"],
-    "ssm_scan_kernel": ["ssm_step.cu", "epilogue.cuh", "dfssm_internal.cuh"],
+    "ssm_step_kernel": ["ssm_step.cu", "epilogue.cuh", "dfssm_internal.cuh"],
 }
 
 
@@ -521,7 +521,7 @@ def ssm_block(torch, seed, peaks, dev, n_layers=48, m=1, steps=200):
     nb = n_layers * per_layer
     return {"workload": f"ssm_step{n_layers}_m{m}", "m": m, "layers": n_layers, "us_per_step": us,
             "GB/s": nb / (us * 1e-6) / 1e9, "hbm_frac": nb / (us * 1e-6) / 1e9 / peaks["hbm"],
-            "bytes_per_step": nb, "tokens_per_s": m / (us * 1e-6), "gpu_launches_per_step": 3,
+            "bytes_per_step": nb, "tokens_per_s": m / (us * 1e-6), "gpu_launches_per_step": 2,
             "l2": "two sets of inputs and states alternated", "traffic": recorded_traffic(f"ssm_step{n_layers}_m{m}")}
 
 

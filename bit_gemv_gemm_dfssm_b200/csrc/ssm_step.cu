@@ -6,25 +6,28 @@
 // state operations: custom kernels handle the state shift register (the causal
 // convolution) and the SSM recurrence (a warp-level reduction). The arithmetic is
 // the Mamba-2 decode step (one group of B and C, 64-channel heads, d_state 128,
-// 4 taps):
+// 4 taps). Two kernels:
 //
-//   ssm_conv_kernel   per channel c: window = (state[c][1..3], xBC[c]) is written
-//                     back as the new shift register (bf16, exact), and
-//                     xc[c] = silu(conv_b[c] + sum_k conv_w[c][k] window[k]) (fp32 fmaf
-//                     chain in k order); per head h: dt = softplus(dt_raw + dt_bias)
-//                     (v itself above 20), dA = exp(-exp(a_log) dt)
-//   ssm_scan_kernel   per (head, token, layer), 256 threads: thread (p, q) owns state row
-//                     p of the head and columns [32 q, 32 q + 32): it streams them with
-//                     16-byte loads and stores, S = fmaf(S, dA, dt x_p B[n]), sums
-//                     S C[n] for its columns, and the four threads of a row add their
-//                     sums with warp shuffles; y = sum + D x_p, g = y silu(z_p), and
-//                     the head's sum of g^2 (warp shuffles, then in warp order)
-//   ssm_norm_kernel   per token: r = 1 / sqrt(mean(g^2) + eps) from the heads' sums in
-//                     head order, out = g r norm_w (bf16 round-to-nearest-even or fp32)
+//   ssm_step_kernel, one CTA of 8 warps per (head, token, layer):
+//   1. the head's 64 x channels and the 256 B and C channels of the convolution:
+//      window = (state[c][1..3], xBC[c]), xc[c] = silu(conv_b[c] + sum_k conv_w[c][k]
+//      window[k]) (fp32 fmaf chain in k order); the window is written back as the new
+//      shift register of the head's own x channels (bf16, exact); dt = softplus(dt_raw +
+//      dt_bias) (v itself above 20), dA = exp(-exp(a_log) dt);
+//   2. the recurrence: lane i owns columns [4 i, 4 i + 4) of the head's state rows, warp
+//      w rows w, w + 8, ..., so one warp instruction loads or stores a whole 512-byte row;
+//      S = fmaf(S, dA, dt x_p B[n]), and y of the row is the warp-level reduction of the
+//      lanes' sums of S C[n] (shuffle tree); y += D x_p, g = y silu(z_p), and the head's
+//      sum of g^2 (per warp over its rows, then in warp order);
+//   ssm_norm_kernel, one CTA per (token, layer), after every head has read the B and C
+//   registers: shifts them, and applies the RMS norm: r = 1 / sqrt(mean(g^2) + eps) from
+//   the heads' sums (lane i adds heads i, i + 32, ..., then a shuffle tree),
+//   out = g r norm_w (bf16 round-to-nearest-even or fp32).
+// (One kernel with a last-CTA ticket for the norm measured slower: the fence before the
+// ticket holds every CTA until its 32 KB of state stores are visible.)
 //
 // The state stream (2 MB of fp32 per layer and token, read and written) bounds the
-// step; the conv and norm kernels move a few tens of KB per layer. Every order of
-// summation is fixed, so results repeat bit for bit.
+// step. Every order of summation is fixed, so results repeat bit for bit.
 #include <cstdint>
 
 #include "dfssm_internal.cuh"
@@ -37,9 +40,7 @@ namespace {
 constexpr int kHeadDim = 64;
 constexpr int kDState = 128;
 constexpr int kDConv = 4;
-constexpr int kConvThreads = 256;
-constexpr int kScanThreads = 256;          // 64 rows x 4 column quarters
-constexpr int kNormThreads = 256;
+constexpr int kThreads = 256;              // 8 warps, 8 state rows each
 constexpr int kMaxDInner = 16384;
 
 struct SsmShape {
@@ -48,25 +49,18 @@ struct SsmShape {
     int out_dtype;
 };
 
-// workspace pieces (byte offsets, 256-aligned): error word, xc, (dt, dA), g, per-head sum of g^2
+// workspace pieces (byte offsets, 256-aligned): error word, g, per-head sum of g^2
 struct SsmWs {
     uint32_t* err;
-    float* xc;
-    float2* dta;
     float* g;
     float* ssq;
 };
 
 __host__ __device__ inline size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-__host__ __device__ inline size_t ws_layout(const SsmShape& s, size_t* off_xc, size_t* off_dta, size_t* off_g,
-                                            size_t* off_ssq) {
+__host__ __device__ inline size_t ws_layout(const SsmShape& s, size_t* off_g, size_t* off_ssq) {
     const size_t lt = (size_t)s.n_layers * s.m;
     size_t o = 256;                                          // error word
-    *off_xc = o;
-    o = align256(o + lt * s.conv_dim * sizeof(float));
-    *off_dta = o;
-    o = align256(o + lt * s.nheads * sizeof(float2));
     *off_g = o;
     o = align256(o + lt * s.d_inner * sizeof(float));
     *off_ssq = o;
@@ -84,115 +78,132 @@ __device__ __forceinline__ float bf16f(uint16_t b) { return __uint_as_float((uin
 
 __device__ __forceinline__ float silu_f(float v) { return __fdiv_rn(v, __fadd_rn(1.0f, expf(-v))); }
 
-__global__ void __launch_bounds__(kConvThreads) ssm_conv_kernel(const dfssm_ssm_layer* __restrict__ layers,
-                                                                const SsmShape s, SsmWs ws) {
-    const int l = blockIdx.z, t = blockIdx.y;
+// The shift register of channel c of token t: its window (old state[1..3], the new input) as
+// packed bf16, and the convolution output silu(conv_b + sum_k conv_w window[k]).
+struct ConvOut {
+    float xc;
+    uint2 window;
+};
+__device__ __forceinline__ ConvOut conv_channel(const dfssm_ssm_layer& L, const SsmShape& s, const uint16_t* zr,
+                                                int t, int c) {
+    const uint2 old = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(L.conv_state) +
+                                                      ((int64_t)t * s.conv_dim + c) * kDConv);
+    const uint16_t win[kDConv] = {(uint16_t)(old.x >> 16), (uint16_t)(old.y & 0xFFFFu), (uint16_t)(old.y >> 16),
+                                  zr[s.d_inner + c]};
+    const float4 w = *reinterpret_cast<const float4*>(L.conv_w + (int64_t)c * kDConv);
+    const float wk[kDConv] = {w.x, w.y, w.z, w.w};
+    float pre = L.conv_b[c];
+#pragma unroll
+    for (int k = 0; k < kDConv; ++k) pre = __fmaf_rn(wk[k], bf16f(win[k]), pre);
+    return ConvOut{silu_f(pre), make_uint2((uint32_t)win[0] | ((uint32_t)win[1] << 16),
+                                           (uint32_t)win[2] | ((uint32_t)win[3] << 16))};
+}
+
+__device__ __forceinline__ uint2* state_slot(const dfssm_ssm_layer& L, const SsmShape& s, int t, int c) {
+    return reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(L.conv_state) + ((int64_t)t * s.conv_dim + c) * kDConv);
+}
+
+__global__ void __launch_bounds__(kThreads, 4) ssm_step_kernel(const dfssm_ssm_layer* __restrict__ layers,
+                                                            const SsmShape s, SsmWs ws) {
+    constexpr int kWarps = kThreads / 32;
+    constexpr int kRows = kHeadDim / kWarps;        // state rows per warp
+    __shared__ __align__(16) float xs[kHeadDim];
+    __shared__ __align__(16) float bc[2 * kDState];  // B then C
+    __shared__ float red[kWarps];
+    __shared__ float2 dta_s;
+    const int h = blockIdx.x, t = blockIdx.y, l = blockIdx.z;
     const dfssm_ssm_layer L = layers[l];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (!layer_ok(L)) {
-        if (blockIdx.x == 0 && t == 0 && threadIdx.x == 0) atomicOr(ws.err, DFSSM_DEVERR_ENTRY_PTR);
+        if (h == 0 && t == 0 && tid == 0) atomicOr(ws.err, DFSSM_DEVERR_ENTRY_PTR);
         return;
     }
     const uint16_t* zr = reinterpret_cast<const uint16_t*>(L.zxbcdt) + (int64_t)t * s.row;
     const int64_t lt = (int64_t)l * s.m + t;
-    const int c = blockIdx.x * kConvThreads + threadIdx.x;
-    if (c < s.conv_dim) {
-        uint2* stp = reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(L.conv_state) +
-                                              ((int64_t)t * s.conv_dim + c) * kDConv);
-        const uint2 old = *stp;
-        const uint16_t nv = zr[s.d_inner + c];
-        // window = (state[1], state[2], state[3], new)
-        const uint16_t win[kDConv] = {(uint16_t)(old.x >> 16), (uint16_t)(old.y & 0xFFFFu), (uint16_t)(old.y >> 16),
-                                      nv};
-        const float4 w = *reinterpret_cast<const float4*>(L.conv_w + (int64_t)c * kDConv);
-        const float wk[kDConv] = {w.x, w.y, w.z, w.w};
-        float pre = L.conv_b[c];
+    // the head's state rows warp + kWarps r (r < kRows), loaded first: their latency overlaps the
+    // convolution below
+    float4* S = reinterpret_cast<float4*>(L.ssm_state + ((int64_t)t * s.nheads + h) * kHeadDim * kDState) + lane;
+    float4 sv[kRows];
 #pragma unroll
-        for (int k = 0; k < kDConv; ++k) pre = __fmaf_rn(wk[k], bf16f(win[k]), pre);
-        ws.xc[lt * s.conv_dim + c] = silu_f(pre);
-        *stp = make_uint2((uint32_t)win[0] | ((uint32_t)win[1] << 16), (uint32_t)win[2] | ((uint32_t)win[3] << 16));
-    }
-    if (blockIdx.x == 0 && threadIdx.x < s.nheads) {
-        const int h = threadIdx.x;
-        const float v = __fadd_rn(bf16f(zr[s.d_inner + s.conv_dim + h]), L.dt_bias[h]);
-        const float dt = v > 20.0f ? v : log1pf(expf(v));
-        const float A = -expf(L.a_log[h]);
-        ws.dta[lt * s.nheads + h] = make_float2(dt, expf(__fmul_rn(dt, A)));
-    }
-}
+    for (int r = 0; r < kRows; ++r) sv[r] = S[(warp + kWarps * r) * (kDState / 4)];
 
-__global__ void __launch_bounds__(kScanThreads) ssm_scan_kernel(const dfssm_ssm_layer* __restrict__ layers,
-                                                                const SsmShape s, SsmWs ws) {
-    __shared__ float red[kScanThreads / 32];
-    const int h = blockIdx.x, t = blockIdx.y, l = blockIdx.z;
-    const dfssm_ssm_layer L = layers[l];
-    if (!layer_ok(L)) return;                       // reported by the conv kernel
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int p = tid >> 2, q = tid & 3;
-    const int64_t lt = (int64_t)l * s.m + t;
-    const float* xc = ws.xc + lt * s.conv_dim;
-    const int ch = h * kHeadDim + p;
-    const float2 dta = ws.dta[lt * s.nheads + h];
-    const float dtx = __fmul_rn(dta.x, xc[ch]);
-    const float4* Bv = reinterpret_cast<const float4*>(xc + s.d_inner + 32 * q);
-    const float4* Cv = reinterpret_cast<const float4*>(xc + s.d_inner + kDState + 32 * q);
-    float4* S = reinterpret_cast<float4*>(L.ssm_state + (((int64_t)t * s.nheads + h) * kHeadDim + p) * kDState + 32 * q);
-    float4 sv[8];
+    // ---- 1. convolution of the B and C channels (read only here) and of the head's x channels
+    {
+        bc[tid] = conv_channel(L, s, zr, t, s.d_inner + tid).xc;
+        if (tid < kHeadDim) {
+            const int c = h * kHeadDim + tid;
+            const ConvOut co = conv_channel(L, s, zr, t, c);
+            xs[tid] = co.xc;
+            *state_slot(L, s, t, c) = co.window;     // only this CTA reads the head's x registers
+        }
+        if (tid == kThreads - 1) {
+            const float v = __fadd_rn(bf16f(zr[s.d_inner + s.conv_dim + h]), L.dt_bias[h]);
+            const float dt = v > 20.0f ? v : log1pf(expf(v));
+            const float A = -expf(L.a_log[h]);
+            dta_s = make_float2(dt, expf(__fmul_rn(dt, A)));
+        }
+    }
+    __syncthreads();
+
+    // ---- 2. the recurrence and the readout
+    const float2 dta = dta_s;
+    const float4 b = reinterpret_cast<const float4*>(bc)[lane];
+    const float4 c = reinterpret_cast<const float4*>(bc + kDState)[lane];
+    float g2 = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) sv[i] = S[i];
-    float acc = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const float4 b = Bv[i], c = Cv[i];
-        float4 v = sv[i];
+    for (int r = 0; r < kRows; ++r) {
+        const int p = warp + kWarps * r, ch = h * kHeadDim + p;
+        const float xp = xs[p];
+        const float dtx = __fmul_rn(dta.x, xp);
+        float4 v = sv[r];
         v.x = __fmaf_rn(v.x, dta.y, __fmul_rn(dtx, b.x));
         v.y = __fmaf_rn(v.y, dta.y, __fmul_rn(dtx, b.y));
         v.z = __fmaf_rn(v.z, dta.y, __fmul_rn(dtx, b.z));
         v.w = __fmaf_rn(v.w, dta.y, __fmul_rn(dtx, b.w));
-        acc = __fmaf_rn(v.x, c.x, acc);
-        acc = __fmaf_rn(v.y, c.y, acc);
-        acc = __fmaf_rn(v.z, c.z, acc);
-        acc = __fmaf_rn(v.w, c.w, acc);
-        sv[i] = v;
+        S[p * (kDState / 4)] = v;
+        float acc = __fmaf_rn(v.x, c.x, __fmaf_rn(v.y, c.y, __fmaf_rn(v.z, c.z, __fmul_rn(v.w, c.w))));
+        // y of row p: the warp-level reduction over the 32 lanes' column groups
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, o));
+        const float y = __fmaf_rn(L.d_skip[h], xp, acc);
+        const float g = __fmul_rn(y, silu_f(bf16f(zr[ch])));
+        if (lane == 0) ws.g[lt * s.d_inner + ch] = g;
+        g2 = __fmaf_rn(g, g, g2);                   // every lane holds the same g
     }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) S[i] = sv[i];
-    // the four column quarters of row p are lanes 4 (p % 8) .. + 3 of this warp
-    acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 1));
-    acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, 2));
-    const float y = __fmaf_rn(L.d_skip[h], xc[ch], acc);
-    const uint16_t* zr = reinterpret_cast<const uint16_t*>(L.zxbcdt) + (int64_t)t * s.row;
-    const float g = __fmul_rn(y, silu_f(bf16f(zr[ch])));
-    if (q == 0) ws.g[lt * s.d_inner + ch] = g;
-    float g2 = q == 0 ? __fmul_rn(g, g) : 0.0f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) g2 = __fadd_rn(g2, __shfl_xor_sync(0xffffffffu, g2, o));
     if (lane == 0) red[warp] = g2;
     __syncthreads();
     if (tid == 0) {
         float sum = 0.0f;
 #pragma unroll
-        for (int w = 0; w < kScanThreads / 32; ++w) sum = __fadd_rn(sum, red[w]);
+        for (int w = 0; w < kWarps; ++w) sum = __fadd_rn(sum, red[w]);
         ws.ssq[lt * s.nheads + h] = sum;
     }
 }
 
-__global__ void __launch_bounds__(kNormThreads) ssm_norm_kernel(const dfssm_ssm_layer* __restrict__ layers,
-                                                                const SsmShape s, SsmWs ws) {
+__global__ void __launch_bounds__(kThreads) ssm_norm_kernel(const dfssm_ssm_layer* __restrict__ layers,
+                                                            const SsmShape s, SsmWs ws) {
     __shared__ float r_s;
-    const int t = blockIdx.y, l = blockIdx.z;
+    const int t = blockIdx.y, l = blockIdx.z, tid = threadIdx.x;
     const dfssm_ssm_layer L = layers[l];
-    if (!layer_ok(L)) return;
+    if (!layer_ok(L)) return;                        // reported by the step kernel
+    const uint16_t* zr = reinterpret_cast<const uint16_t*>(L.zxbcdt) + (int64_t)t * s.row;
     const int64_t lt = (int64_t)l * s.m + t;
-    if (threadIdx.x == 0) {
+    {
+        const int cch = s.d_inner + tid;             // every head has read these registers
+        *state_slot(L, s, t, cch) = conv_channel(L, s, zr, t, cch).window;
+    }
+    if (tid < 32) {
         float sum = 0.0f;
-        for (int h = 0; h < s.nheads; ++h) sum = __fadd_rn(sum, ws.ssq[lt * s.nheads + h]);
-        r_s = __frsqrt_rn(__fadd_rn(__fdiv_rn(sum, (float)s.d_inner), s.eps));
+        for (int hh = tid; hh < s.nheads; hh += 32) sum = __fadd_rn(sum, ws.ssq[lt * s.nheads + hh]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, o));
+        if (tid == 0) r_s = __frsqrt_rn(__fadd_rn(__fdiv_rn(sum, (float)s.d_inner), s.eps));
     }
     __syncthreads();
     const float r = r_s;
-    for (int c = blockIdx.x * kNormThreads + threadIdx.x; c < s.d_inner; c += gridDim.x * kNormThreads) {
-        const float o = __fmul_rn(__fmul_rn(ws.g[lt * s.d_inner + c], r), L.norm_w[c]);
-        const int64_t idx = (int64_t)t * s.d_inner + c;
+    for (int cc = tid; cc < s.d_inner; cc += kThreads) {
+        const float o = __fmul_rn(__fmul_rn(ws.g[lt * s.d_inner + cc], r), L.norm_w[cc]);
+        const int64_t idx = (int64_t)t * s.d_inner + cc;
         if (s.out_dtype == DFSSM_BF16) reinterpret_cast<uint16_t*>(L.out)[idx] = f32_to_bf16_bits(o);
         else reinterpret_cast<float*>(L.out)[idx] = o;
     }
@@ -229,8 +240,8 @@ extern "C" dfssm_status dfssm_ssm_workspace_bytes(const dfssm_ssm_dims* dims, in
     const dfssm_status st = shape_of(dims, n_layers, m, &s);
     if (st != DFSSM_OK) return st;
     if (!bytes) return DFSSM_ERR_INVALID_ARG;
-    size_t a, b, c, d;
-    *bytes = ws_layout(s, &a, &b, &c, &d);
+    size_t a, b;
+    *bytes = ws_layout(s, &a, &b);
     return DFSSM_OK;
 }
 
@@ -241,19 +252,15 @@ extern "C" dfssm_status dfssm_ssm_step(const dfssm_ssm_dims* dims, const dfssm_s
     const dfssm_status st = shape_of(dims, n_layers, m, &s);
     if (st != DFSSM_OK) return st;
     if (!layers_dev || (reinterpret_cast<uintptr_t>(layers_dev) & 7u)) return DFSSM_ERR_INVALID_ARG;
-    size_t o_xc, o_dta, o_g, o_ssq;
-    const size_t need = ws_layout(s, &o_xc, &o_dta, &o_g, &o_ssq);
+    size_t o_g, o_ssq;
+    const size_t need = ws_layout(s, &o_g, &o_ssq);
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
         return DFSSM_ERR_INVALID_ARG;
     uint8_t* w = static_cast<uint8_t*>(workspace);
-    SsmWs ws{reinterpret_cast<uint32_t*>(w), reinterpret_cast<float*>(w + o_xc), reinterpret_cast<float2*>(w + o_dta),
-             reinterpret_cast<float*>(w + o_g), reinterpret_cast<float*>(w + o_ssq)};
+    SsmWs ws{reinterpret_cast<uint32_t*>(w), reinterpret_cast<float*>(w + o_g), reinterpret_cast<float*>(w + o_ssq)};
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    ssm_conv_kernel<<<dim3((s.conv_dim + kConvThreads - 1) / kConvThreads, m, n_layers), kConvThreads, 0, cs>>>(
-        layers_dev, s, ws);
-    ssm_scan_kernel<<<dim3(s.nheads, m, n_layers), kScanThreads, 0, cs>>>(layers_dev, s, ws);
-    ssm_norm_kernel<<<dim3((s.d_inner + 4 * kNormThreads - 1) / (4 * kNormThreads), m, n_layers), kNormThreads, 0,
-                      cs>>>(layers_dev, s, ws);
+    ssm_step_kernel<<<dim3(s.nheads, m, n_layers), kThreads, 0, cs>>>(layers_dev, s, ws);
+    ssm_norm_kernel<<<dim3(1, m, n_layers), kThreads, 0, cs>>>(layers_dev, s, ws);
     return cudaGetLastError() == cudaSuccess ? DFSSM_OK : DFSSM_ERR_CUDA;
 }
 

@@ -266,13 +266,13 @@ typedef struct {
 dfssm_status dfssm_ssm_workspace_bytes(const dfssm_ssm_dims* dims, int32_t n_layers, int32_t m, size_t* bytes);
 
 /* One decode step for n_layers independent layers (layers_dev: DEVICE array of n_layers
- * dfssm_ssm_layer) and m tokens each, on `stream`: three kernels (shift register and
- * convolution; recurrence, readout and gate; RMS norm). workspace: 256-byte aligned, at
- * least dfssm_ssm_workspace_bytes; its first 4 bytes are a device error word (zero it once
- * before the first call) that gets DFSSM_DEVERR_ENTRY_PTR when a layer holds a NULL or
- * misaligned pointer (that layer is skipped); read and clear it with dfssm_ssm_read_error.
- * Calls sharing a workspace must be ordered. Allocates nothing. Argument errors return
- * synchronously with no launch. */
+ * dfssm_ssm_layer) and m tokens each, on `stream`, as two kernels (convolution, recurrence
+ * and gate, one CTA per head, token and layer; then the B and C registers and the RMS norm
+ * per token and layer). workspace: 256-byte aligned, at least dfssm_ssm_workspace_bytes,
+ * zeroed once before its first use. Its first 4 bytes are a device error word that
+ * gets DFSSM_DEVERR_ENTRY_PTR when a layer holds a NULL or misaligned pointer (that layer
+ * is skipped); read and clear it with dfssm_ssm_read_error. Calls sharing a workspace must
+ * be ordered. Allocates nothing. Argument errors return synchronously with no launch. */
 dfssm_status dfssm_ssm_step(const dfssm_ssm_dims* dims, const dfssm_ssm_layer* layers_dev, int32_t n_layers,
                             int32_t m, void* workspace, size_t workspace_bytes, void* stream);
 

@@ -74,7 +74,7 @@ def test_argument_errors_without_gpu():
     assert lib.dfssm_plan_destroy(None) == dfssm.DFSSM_OK
     # the state step: unsupported shapes and missing buffers return before any CUDA call
     dims = dfssm.SsmDims(4096, 64, 128, 4, 1e-5, dfssm.DFSSM_BF16)
-    assert dfssm.dfssm_ssm_workspace_bytes(dims, 48, 1) > 48 * 4352 * 4
+    assert dfssm.dfssm_ssm_workspace_bytes(dims, 48, 1) >= 48 * 4096 * 4       # g of every layer
     for bad in (dfssm.SsmDims(4096, 32, 128, 4, 1e-5, 0), dfssm.SsmDims(4096, 64, 64, 4, 1e-5, 0),
                 dfssm.SsmDims(4096, 64, 128, 3, 1e-5, 0), dfssm.SsmDims(4100, 64, 128, 4, 1e-5, 0)):
         n = ctypes.c_size_t(0)
