@@ -19,8 +19,9 @@
 //      S = fmaf(S, dA, dt x_p B[n]), and y of the row is the warp-level reduction of the
 //      lanes' sums of S C[n] (shuffle tree); y += D x_p, g = y silu(z_p), and the head's
 //      sum of g^2 (per warp over its rows, then in warp order);
-//   ssm_norm_kernel, one CTA per (token, layer), after every head has read the B and C
-//   registers: shifts them, and applies the RMS norm: r = 1 / sqrt(mean(g^2) + eps) from
+//   ssm_norm_kernel, 1024 channels per CTA, after every head has read the B and C
+//   registers: the first CTA of a (token, layer) shifts them, and each applies the RMS
+//   norm to its channels: r = 1 / sqrt(mean(g^2) + eps) from
 //   the heads' sums (lane i adds heads i, i + 32, ..., then a shuffle tree),
 //   out = g r norm_w (bf16 round-to-nearest-even or fp32).
 // (One kernel with a last-CTA ticket for the norm measured slower: the fence before the
@@ -42,6 +43,7 @@ constexpr int kDState = 128;
 constexpr int kDConv = 4;
 constexpr int kThreads = 256;              // 8 warps, 8 state rows each
 constexpr int kMaxDInner = 16384;
+constexpr int kNormCols = 1024;            // channels per CTA of the norm kernel
 
 struct SsmShape {
     int d_inner, nheads, conv_dim, row, m, n_layers;
@@ -188,7 +190,7 @@ __global__ void __launch_bounds__(kThreads) ssm_norm_kernel(const dfssm_ssm_laye
     if (!layer_ok(L)) return;                        // reported by the step kernel
     const uint16_t* zr = reinterpret_cast<const uint16_t*>(L.zxbcdt) + (int64_t)t * s.row;
     const int64_t lt = (int64_t)l * s.m + t;
-    {
+    if (blockIdx.x == 0) {
         const int cch = s.d_inner + tid;             // every head has read these registers
         *state_slot(L, s, t, cch) = conv_channel(L, s, zr, t, cch).window;
     }
@@ -201,8 +203,21 @@ __global__ void __launch_bounds__(kThreads) ssm_norm_kernel(const dfssm_ssm_laye
     }
     __syncthreads();
     const float r = r_s;
-    for (int cc = tid; cc < s.d_inner; cc += kThreads) {
-        const float o = __fmul_rn(__fmul_rn(ws.g[lt * s.d_inner + cc], r), L.norm_w[cc]);
+    // this CTA's kNormCols channels, kNormCols / kThreads per thread, loads first
+    constexpr int kPer = kNormCols / kThreads;
+    const int c0 = blockIdx.x * kNormCols + tid;
+    float gv[kPer], wv[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        const int cc = c0 + i * kThreads;
+        gv[i] = cc < s.d_inner ? ws.g[lt * s.d_inner + cc] : 0.0f;
+        wv[i] = cc < s.d_inner ? L.norm_w[cc] : 0.0f;
+    }
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        const int cc = c0 + i * kThreads;
+        if (cc >= s.d_inner) break;
+        const float o = __fmul_rn(__fmul_rn(gv[i], r), wv[i]);
         const int64_t idx = (int64_t)t * s.d_inner + cc;
         if (s.out_dtype == DFSSM_BF16) reinterpret_cast<uint16_t*>(L.out)[idx] = f32_to_bf16_bits(o);
         else reinterpret_cast<float*>(L.out)[idx] = o;
@@ -260,7 +275,8 @@ extern "C" dfssm_status dfssm_ssm_step(const dfssm_ssm_dims* dims, const dfssm_s
     SsmWs ws{reinterpret_cast<uint32_t*>(w), reinterpret_cast<float*>(w + o_g), reinterpret_cast<float*>(w + o_ssq)};
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
     ssm_step_kernel<<<dim3(s.nheads, m, n_layers), kThreads, 0, cs>>>(layers_dev, s, ws);
-    ssm_norm_kernel<<<dim3(1, m, n_layers), kThreads, 0, cs>>>(layers_dev, s, ws);
+    ssm_norm_kernel<<<dim3((s.d_inner + kNormCols - 1) / kNormCols, m, n_layers), kThreads, 0, cs>>>(layers_dev, s,
+                                                                                                        ws);
     return cudaGetLastError() == cudaSuccess ? DFSSM_OK : DFSSM_ERR_CUDA;
 }
 
