@@ -337,8 +337,15 @@ __global__ void __launch_bounds__(kSliceThreads, 65536 / (kSliceThreads * kSlice
                                       &sh.bar);
                 }
             }
-            if (!ptx::mbar_wait(&sh.bar, phase)) {
-                if (tid == 0) atomicOr(sa.err, DFSSM_DEVERR_TIMEOUT);
+            // a wait that gave up stops the CTA: it reports the error, lets the copies in flight
+            // into its shared memory land (bounded) and issues nothing more
+            const bool got = ptx::mbar_wait(&sh.bar, phase);
+            if (__syncthreads_or(!got)) {
+                if (tid == 0) {
+                    atomicOr(sa.err, DFSSM_DEVERR_TIMEOUT);
+                    ptx::mbar_wait(&sh.bar, phase);
+                }
+                return;
             }
             phase ^= 1u;
             int h[kWbRows];
