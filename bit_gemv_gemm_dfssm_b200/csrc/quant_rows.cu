@@ -99,6 +99,8 @@ __host__ __device__ inline int tokens_per_item(int d_in) {
     return t < kMaxT ? t : kMaxT;
 }
 
+constexpr int kStartTable = 256;            // blocks whose first item's linear the host supplies
+
 struct RowsArgs {
     const dfssm_stack_entry* entries;
     dfssm_stack_entry single;
@@ -109,6 +111,11 @@ struct RowsArgs {
     int8_t* q_ws;
     TokStats* st_ws;
     uint32_t* err;
+    // the linear of each block's first item and that linear's first item index, found on the host,
+    // so a block does not walk the descriptors from the first linear (has_start = 0: it does)
+    int has_start;
+    int start_lin[kStartTable];
+    int start_item[kStartTable];
 };
 
 __device__ __forceinline__ void consumer_sync() { ptx::named_barrier(kBarConsumers, kConsumers); }
@@ -194,9 +201,9 @@ __device__ __forceinline__ void item_range(const RowsArgs& a, int& lo, int& hi) 
 
 // ------------------------------------------------------------------ item issue (warp 0)
 __device__ __forceinline__ void cursor_start(const RowsArgs& a, Cursor& cur) {
-    cur.lin = 0;
-    cur.begin = 0;
-    cur.tpi = tokens_per_item(a.descs[0].d_in);
+    cur.lin = a.has_start ? a.start_lin[blockIdx.x] : 0;
+    cur.begin = a.has_start ? a.start_item[blockIdx.x] : 0;
+    cur.tpi = tokens_per_item(a.descs[cur.lin].d_in);
     cur.count = (a.m + cur.tpi - 1) / cur.tpi;
     cur.info_lin = -1;
     cur.x = nullptr;
@@ -544,7 +551,24 @@ cudaError_t launch_quant_rows(const LaunchCtx& c) {
     }
     if (total == 0) return cudaSuccess;
     const int grid = min(total, c.sm_count);
-    RowsArgs ra{c.entries, c.single, c.desc, c.n, c.m, total, c.q_ws, c.st_ws, c.err};
+    RowsArgs ra{c.entries, c.single, c.desc, c.n, c.m, total, c.q_ws, c.st_ws, c.err, 0, {}, {}};
+    if (grid <= kStartTable) {
+        // block b's items start at b * total / grid (item_range); its linear and that linear's first item
+        int l = 0, begin = 0;
+        for (int b = 0; b < grid; ++b) {
+            const int lo = (int)((int64_t)b * total / grid);
+            for (;;) {
+                const int tpi = tokens_per_item(c.host_desc[l].d_in);
+                const int count = (c.m + tpi - 1) / tpi;
+                if (lo < begin + count || l + 1 == c.n) break;
+                begin += count;
+                ++l;
+            }
+            ra.start_lin[b] = l;
+            ra.start_item[b] = begin;
+        }
+        ra.has_start = 1;
+    }
     quant_rows_kernel<<<grid, kThreads, sizeof(RowsShared), c.stream>>>(ra);
     return cudaGetLastError();
 }
