@@ -270,66 +270,96 @@ __device__ __forceinline__ int q_pos(int gg, int i, int p) {
 struct TokShared {
     float sx[kMaxTok];
     int sumq[kMaxTok];
-    float red_f[kMaxWarps][kMaxTok];
-    int red_i[kMaxWarps][kMaxTok];
+    uint32_t amax_u[kMaxTok];          // max |x| per token as fp32 bit patterns
     float u[kMaxTok][kRank];
 };
 
 // Quantise the m x d_in activations of linear L into the permuted int8 layout
 // (token stride d_in + kTokPad), with per-token s_x and sum q. Same arithmetic
-// as the quantisation kernel (epilogue.cuh), so the same bytes.
+// as the quantisation kernel (epilogue.cuh), so the same bytes. Both passes run over
+// the (token, 8-column chunk) pairs of the whole m x d_in block, kQuantLoads 16-byte loads
+// in flight per thread whatever m is; a thread's per-token max and sum go to shared memory
+// (atomics) when its pairs move on to the next token.
+constexpr int kQuantLoads = 4;
 template <int W>
 __device__ void quantise_into_smem(const Lin& L, int m, uint8_t* q_s, TokShared& ts) {
-    constexpr int kWarps = W, kThreads = W * 32;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int kThreads = W * 32;
+    const int tid = threadIdx.x;
     const int n8 = L.d_in >> 3;                      // 8-column chunks per row
+    const int total = m * n8;
     const int qstride = q_stride(L.d_in);
-    for (int t = 0; t < m; ++t) {
-        float am = 0.0f;
-        for (int ch = tid; ch < n8; ch += kThreads) {
-            const uint4 v = *reinterpret_cast<const uint4*>(L.x + (int64_t)t * L.d_in + 8 * ch);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) am = fmaxf(am, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-        if (lane == 0) ts.red_f[warp][t] = am;
+    const uint4* xv = reinterpret_cast<const uint4*>(L.x);    // pair k = t n8 + ch is xv[k]
+    if (tid < m) {
+        ts.amax_u[tid] = 0u;
+        ts.sumq[tid] = 0;
     }
     __syncthreads();
-    for (int t = 0; t < m; ++t) {
-        float am = ts.red_f[0][t];
+    {
+        uint32_t am = 0u;
+        int tcur = -1;
+        for (int k0 = tid; k0 < total; k0 += kQuantLoads * kThreads) {
+            uint4 v[kQuantLoads];
 #pragma unroll
-        for (int w = 1; w < kWarps; ++w) am = fmaxf(am, ts.red_f[w][t]);
-        const float inv = quant_inv(am);
-        const bool zero = am == 0.0f;
-        int sum = 0;
-        for (int ch = tid; ch < n8; ch += kThreads) {
-            const uint4 v = *reinterpret_cast<const uint4*>(L.x + (int64_t)t * L.d_in + 8 * ch);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            // columns 8 ch + p (p = 0..7) of 32-column group gg = ch / 4 (i = ch % 4)
-            uint8_t* row = q_s + t * qstride;
+            for (int j = 0; j < kQuantLoads; ++j) {
+                const int k = k0 + j * kThreads;
+                v[j] = k < total ? xv[k] : make_uint4(0u, 0u, 0u, 0u);
+            }
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int q0 = quant1(bf16_lo(w[i]), inv, zero), q1 = quant1(bf16_hi(w[i]), inv, zero);
-                sum += q0 + q1;
-                row[q_pos(ch >> 2, ch & 3, 2 * i)] = (uint8_t)q0;
-                row[q_pos(ch >> 2, ch & 3, 2 * i + 1)] = (uint8_t)q1;
+            for (int j = 0; j < kQuantLoads; ++j) {
+                const int k = k0 + j * kThreads;
+                if (k >= total) break;
+                const int t = k / n8;
+                if (t != tcur) {
+                    if (tcur >= 0) atomicMax(&ts.amax_u[tcur], am);
+                    am = 0u;
+                    tcur = t;
+                }
+                am = absmax8_bits(v[j], am);
             }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        if (lane == 0) ts.red_i[warp][t] = sum;
-        if (tid == 0) ts.sx[t] = quant_sx(am);
+        if (tcur >= 0) atomicMax(&ts.amax_u[tcur], am);
     }
     __syncthreads();
-    if (tid < m) {
-        int s = 0;
+    {
+        int sum = 0, tcur = -1;
+        float inv = 0.0f;
+        bool zero = true;
+        for (int k0 = tid; k0 < total; k0 += kQuantLoads * kThreads) {
+            uint4 v[kQuantLoads];
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) s += ts.red_i[w][tid];
-        ts.sumq[tid] = s;
+            for (int j = 0; j < kQuantLoads; ++j) {
+                const int k = k0 + j * kThreads;
+                v[j] = k < total ? xv[k] : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int j = 0; j < kQuantLoads; ++j) {
+                const int k = k0 + j * kThreads;
+                if (k >= total) break;
+                const int t = k / n8, ch = k - t * n8;
+                if (t != tcur) {
+                    if (tcur >= 0) atomicAdd(&ts.sumq[tcur], sum);
+                    sum = 0;
+                    tcur = t;
+                    const float am = __uint_as_float(ts.amax_u[t]);
+                    inv = quant_inv(am);
+                    zero = am == 0.0f;
+                }
+                const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+                // columns 8 ch + p (p = 0..7) of 32-column group gg = ch / 4 (i = ch % 4)
+                uint8_t* row = q_s + t * qstride;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int q0 = quant1(bf16_lo(w[i]), inv, zero), q1 = quant1(bf16_hi(w[i]), inv, zero);
+                    sum += q0 + q1;
+                    row[q_pos(ch >> 2, ch & 3, 2 * i)] = (uint8_t)q0;
+                    row[q_pos(ch >> 2, ch & 3, 2 * i + 1)] = (uint8_t)q1;
+                }
+            }
+        }
+        if (tcur >= 0) atomicAdd(&ts.sumq[tcur], sum);
     }
-    // (the caller synchronises before sumq is read)
+    if (tid < m) ts.sx[tid] = quant_sx(__uint_as_float(ts.amax_u[tid]));
+    // (the caller synchronises before sumq and sx are read)
 }
 
 template <int RT, int NT, int W>
