@@ -304,6 +304,16 @@ def device_weight_sets(shapes, cfg, seed, n_sets=2):
     return sets
 
 
+def mapped_address(host_ptr):
+    """The device address of pinned host memory (under unified addressing the same number);
+    raises, before anything is launched, if the memory is not mapped for the device."""
+    from cuda.bindings import runtime as rt
+    err, attr = rt.cudaPointerGetAttributes(host_ptr)
+    if err != rt.cudaError_t.cudaSuccess or attr.type != rt.cudaMemoryType.cudaMemoryTypeHost or not attr.devicePointer:
+        raise RuntimeError(f"host buffer {host_ptr:#x} is not pinned and mapped for the device ({err})")
+    return int(attr.devicePointer)
+
+
 class StackRunner:
     """Device buffers, plan and stack entries for one workload, two weight sets."""
 
@@ -330,22 +340,20 @@ class StackRunner:
         self.x = self.x_host.cuda()
         self.y = torch.empty(yo, dtype=torch.bfloat16, device="cuda")
         self.y_host = torch.empty(yo, dtype=torch.int16).pin_memory()
-        self.sets = []
         if weight_sets is None:
             weight_sets = device_weight_sets(shapes, cfg, seed, n_sets)
-        for s in range(n_sets):
-            ws = weight_sets[s]
-            ents = []
-            for i, w in enumerate(ws):
-                ents.append(dfssm.StackEntry(
-                    dfssm.weights_struct(w["sign"], w["alpha"], w["wa"], w["sa"], w["wb"], w["sb"]),
-                    self.x.data_ptr() + 2 * self.x_off[i], self.y.data_ptr() + 2 * self.y_off[i],
-                    dfssm.Debug(0, 0, 0, 0), i, 0))
-            raw = dfssm.stack_entries_bytes(ents)
-            edev = torch.frombuffer(bytearray(raw), dtype=torch.uint8).cuda()
-            self.sets.append((ws, edev))
+        self.sets = [(ws, self.entries(ws, self.y.data_ptr())) for ws in weight_sets[:n_sets]]
         self.n = n
         torch.cuda.synchronize()
+
+    def entries(self, ws, y_base):
+        """The device array of stack entries for the weight set ws, entry i's y at y_base plus its
+        offset in the contiguous output (y_base: any address the GPU can write)."""
+        dfssm = self.dfssm
+        ents = [dfssm.StackEntry(dfssm.weights_struct(w["sign"], w["alpha"], w["wa"], w["sa"], w["wb"], w["sb"]),
+                                 self.x.data_ptr() + 2 * self.x_off[i], y_base + 2 * self.y_off[i],
+                                 dfssm.Debug(0, 0, 0, 0), i, 0) for i, w in enumerate(ws)]
+        return self.torch.frombuffer(bytearray(dfssm.stack_entries_bytes(ents)), dtype=self.torch.uint8).cuda()
 
     def weights_of(self, s):
         return self.sets[s][0]
@@ -582,20 +590,29 @@ def run_gpu(args, wl_name):
     tok_s = total_units / (ms * 1e-3)
     achieved = nb / (ms_step * 1e-3) / 1e9
 
-    # end to end through the C ABI: pinned host x -> device, stack call, y -> pinned host
-    stream = torch.cuda.current_stream()
-
-    def e2e_step(i):
-        r.x.copy_(r.x_host, non_blocking=True)
-        r.call(i % 2, stream.cuda_stream)
-        r.y_host.copy_(r.y.view(torch.int16), non_blocking=True)
-
+    # end to end through the C ABI with host buffers, every step: pinned host x -> device (one
+    # copy), then the stack call with each entry's y in pinned host memory, which the kernels
+    # write over PCIe as they finish each row (the device -> host transfer overlaps the compute).
     e2e = None
     if not args.no_e2e:
+        y_host_dev = mapped_address(r.y_host.data_ptr())
+        host_sets = [r.entries(ws, y_host_dev) for ws, _ in r.sets]
+        stream = torch.cuda.current_stream()
+
+        def e2e_step(i):
+            r.x.copy_(r.x_host, non_blocking=True)
+            r.dfssm.dfssm_linear_stack_fwd(r.plan, host_sets[i % 2].data_ptr(), r.n, r.m, stream.cuda_stream)
+
         e2e_ms = timed_device(torch, e2e_step, args.steps, args.warmup, dist, dev)
+        # the host outputs equal those of the same call writing device memory
+        last = r.y_host.clone()
+        r.call((args.steps - 1) % 2, stream.cuda_stream)
+        torch.cuda.synchronize()
+        if not torch.equal(r.y.view(torch.int16).cpu(), last):
+            raise RuntimeError("outputs written to host memory differ from those written to device memory")
         e2e = {"value": sum_over_ranks(float(nb * args.steps), dist, dev) / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                "ms_per_step": e2e_ms / args.steps, "h2d_bytes_per_step": r.x_elems * 2,
-               "d2h_bytes_per_step": r.y_elems * 2}
+               "d2h_bytes_per_step": r.y_elems * 2, "y": "pinned host memory, written by the kernels"}
     r.check()
     r.close()
     del graphs

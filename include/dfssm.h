@@ -112,7 +112,11 @@ typedef struct {
 
 /* One linear of a stack (this struct lives in DEVICE memory for
  * dfssm_linear_stack_fwd). x: m x d_in bf16 row-major; y: m x d_out of the
- * desc's y_dtype, row-major. desc_index must equal the entry's position. */
+ * desc's y_dtype, row-major. desc_index must equal the entry's position.
+ * y may be pinned host memory mapped for the device (its device address): the
+ * kernels then write each output over the bus as they finish it, so the copy
+ * back overlaps the compute. x is read several times and belongs in device
+ * memory. */
 typedef struct {
     dfssm_linear_weights w;
     const void* x;

@@ -69,6 +69,15 @@ class Linear:
         return self.dy.cpu().numpy()
 
 
+def mapped_address(host_ptr: int) -> int:
+    """The device address of pinned host memory; raises before any launch if it is not mapped."""
+    from cuda.bindings import runtime as rt
+    err, attr = rt.cudaPointerGetAttributes(host_ptr)
+    assert err == rt.cudaError_t.cudaSuccess and attr.type == rt.cudaMemoryType.cudaMemoryTypeHost, err
+    assert attr.devicePointer
+    return int(attr.devicePointer)
+
+
 def entries_device(entries) -> torch.Tensor:
     raw = dfssm.stack_entries_bytes(entries)
     return torch.frombuffer(bytearray(raw), dtype=torch.uint8).cuda()

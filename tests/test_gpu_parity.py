@@ -13,7 +13,8 @@ import torch
 import bit_gemv_gemm_dfssm_b200 as dfssm
 import dfssm_synth as synth
 import oracle
-from gpu_util import Linear, check_linear_full, check_linear_sampled, check_y, dev, entries_device, term_bound
+from gpu_util import (Linear, check_linear_full, check_linear_sampled, check_y, dev, entries_device, mapped_address,
+                      term_bound)
 
 pytestmark = pytest.mark.gpu
 
@@ -274,6 +275,29 @@ def test_repeated_calls_are_deterministic():
                     assert torch.equal(a, b)
         finally:
             dfssm.dfssm_plan_destroy(plan)
+
+
+@pytest.mark.parametrize("m", [1, 5, 40])
+def test_stack_output_in_pinned_host_memory(m):
+    # y may be any memory the GPU can write: outputs in pinned host buffers (written by the kernels
+    # over the bus) are byte-identical to outputs in device memory, on the slice, quant and prefill paths
+    shapes = [(2048, 1000), (4096, 512), (256, 100)]
+    lins, plan, ent = build_stack(shapes, m, F32 if m % 2 else BF16, dbg=False)
+    try:
+        stream = torch.cuda.current_stream().cuda_stream
+        dfssm.dfssm_linear_stack_fwd(plan, ent.data_ptr(), len(lins), m, stream)
+        torch.cuda.synchronize()
+        hosts = [torch.full_like(l.dy, float("nan"), device="cpu").pin_memory() for l in lins]
+        hent = entries_device([dfssm.StackEntry(l.weights(), l.dx.data_ptr(), mapped_address(h.data_ptr()),
+                                                dfssm.Debug(0, 0, 0, 0), i, 0) for i, (l, h) in enumerate(zip(lins, hosts))])
+        dfssm.dfssm_linear_stack_fwd(plan, hent.data_ptr(), len(lins), m, stream)
+        st, bits = dfssm.dfssm_plan_check(plan)
+        assert st == dfssm.DFSSM_OK, hex(bits)
+        for l, h in zip(lins, hosts):
+            assert torch.equal(h.view(torch.uint8), l.dy.cpu().view(torch.uint8))
+            check_linear_full(l)
+    finally:
+        dfssm.dfssm_plan_destroy(plan)
 
 
 # ------------------------------------------------------------------ full-size workloads
