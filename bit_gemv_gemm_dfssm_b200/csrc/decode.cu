@@ -53,6 +53,7 @@
 //  * Epilogue (epilogue.cuh): lane i of a warp takes output row i, gathers its
 //    sums with warp shuffles, and applies the LoRA up-projection and the
 //    dequantisation in the same fp32 order as the prefill path.
+#include <algorithm>
 #include <cstring>
 
 #include "dfssm_internal.cuh"
@@ -79,7 +80,7 @@ __host__ __device__ __forceinline__ int q_stride(int d_in) { return ((d_in + 255
 constexpr int kStages = DFSSM_DECODE_STAGES;
 constexpr int kMaxTok = 16;
 
-constexpr int kStartTable = 700;   // CTAs whose start the host supplies (keeps the arguments under 4 KB)
+constexpr int kStartTable = 600;   // CTAs whose start the host supplies (keeps the arguments under 4 KB)
 constexpr int kMapSlots = 4;       // device-edited maps per CTA; >= kStages, so a slot's old loads are done
 constexpr int kMaxCtasPerSm = 8;   // map slots are allocated for this many CTAs per SM
 static_assert(kMapSlots >= kStages, "map slot reuse");
@@ -102,13 +103,16 @@ struct DecodeArgs {
     int ri;                  // which work_begin: 0 for 128-row blocks, 1 for 192-row blocks
     int slot_bytes;          // bytes of one ring slot
     int q_region;            // bytes of the staged-q region
-    // first (linear, block) of each CTA, found on the host (linear << 16 | block), so a CTA
-    // needs no search through the descriptors before its first loads; has_start = 0 when the
-    // grid is larger than the table (the CTAs then search themselves)
+    // the grid's contiguous work ranges, found on the host: range r runs from start[r] (linear
+    // << 16 | block) up to start[r + 1], so a CTA needs no search through the descriptors before
+    // its first loads; CTA i runs range perm[i]. has_start = 0 when the grid is larger than the
+    // table (CTA i then finds range i itself).
     int has_start;
     uint32_t* err;           // the plan's device error word
     uint32_t start[kStartTable];
+    uint16_t perm[kStartTable];
 };
+static_assert(sizeof(DecodeArgs) <= 4096, "decode kernel arguments");
 
 // Fields of one linear, cached in registers while a cursor is on it.
 // (kStartTable is defined before DecodeArgs.)
@@ -396,9 +400,10 @@ __global__ void __launch_bounds__(W * 32) decode_kernel(const __grid_constant__ 
 
     const int64_t lo = a.total_units * blockIdx.x / gridDim.x;
     const int64_t hi = a.total_units * (blockIdx.x + 1) / gridDim.x;
-    const uint32_t end = a.has_start && blockIdx.x + 1 < gridDim.x ? a.start[blockIdx.x + 1] : ((uint32_t)a.n << 16);
+    const int range = a.has_start ? (int)a.perm[blockIdx.x] : (int)blockIdx.x;
+    const uint32_t end = a.has_start && range + 1 < (int)gridDim.x ? a.start[range + 1] : ((uint32_t)a.n << 16);
     Walk<R> cw, lw;
-    if (a.has_start) cw.start_at(a, (int)(a.start[blockIdx.x] >> 16), (int)(a.start[blockIdx.x] & 0xFFFFu));
+    if (a.has_start) cw.start_at(a, (int)(a.start[range] >> 16), (int)(a.start[range] & 0xFFFFu));
     else cw.start(a, lo);
     lw = cw;
     // the first linear's activations into L2 ahead of the weight stream (quantised below)
@@ -692,12 +697,13 @@ cudaError_t launch_cfg(const LaunchCtx& c) {
     a.q_region = geo.q_region;
     a.has_start = 0;
     a.err = c.err;
-    // each CTA's first block, as Walk::start finds it on the device; a CTA runs up to the next
-    // CTA's first block
+    // the grid's work ranges: range i starts at the first block at or after work unit
+    // total_units * i / grid (as Walk::start finds it on the device) and runs up to range i + 1
     if (grid <= kStartTable && c.n < 65536) {
         bool fits = true;
         const int ri = R == 128 ? 0 : 1;
         const int64_t base = c.host_desc[0].work_begin[ri];
+        int64_t pos[kStartTable + 1];      // first work unit of each range (its entry included)
         int l = 0;
         for (int i = 0; i < grid && fits; ++i) {
             const int64_t lo = total_units * i / grid;
@@ -711,8 +717,36 @@ cudaError_t launch_cfg(const LaunchCtx& c) {
             if (b >= nblocks) { b = 0; ++sl; }
             if (b > 0xFFFF) fits = false;
             a.start[i] = ((uint32_t)sl << 16) | (uint32_t)b;
+            pos[i] = sl >= c.n ? total_units
+                               : c.host_desc[sl].work_begin[ri] - base + (b > 0 ? kDecodeLinStart + (int64_t)b * bu : 0);
         }
+        pos[grid] = total_units;
         a.has_start = fits ? 1 : 0;
+        // Which CTA runs which range. Ranges end on block boundaries, so their costs differ by up
+        // to a block (2 or 4 k-chunks in about 21 for the one-token stack), and a stack whose
+        // linears repeat with the grid's period gives the CTAs that share an SM (CTAs i, i + S,
+        // i + 2S, ... for S SMs when all are resident) equal ranges, so some SMs carry a whole
+        // block per CTA more than others. Ranges are therefore dealt by cost, largest first, in
+        // passes over the SMs that alternate direction; pass w goes to the CTAs i = w S + g, so
+        // the first-launched CTA of an SM (the fastest of its CTAs in a per-CTA timing trace)
+        // takes the largest.
+        // The placement of CTAs on SMs is the hardware's: this only decides which range each CTA
+        // index runs, so the results never depend on it.
+        int order[kStartTable];
+        for (int i = 0; i < grid; ++i) order[i] = i;
+        const int S = c.sm_count;
+        if (fits && grid == S * per_sm && per_sm > 1) {
+            int64_t cost[kStartTable];
+            for (int i = 0; i < grid; ++i) {
+                const bool mid = (a.start[i] & 0xFFFFu) != 0;   // a CTA entering mid-linear quantises too
+                cost[i] = pos[i + 1] - pos[i] + (mid ? kDecodeLinStart : 0);
+            }
+            std::stable_sort(order, order + grid, [&](int x, int y) { return cost[x] > cost[y]; });
+            for (int w = 0; w < per_sm; ++w)
+                for (int g = 0; g < S; ++g) a.perm[w * S + g] = (uint16_t)order[w * S + ((w & 1) ? S - 1 - g : g)];
+        } else {
+            for (int i = 0; i < grid; ++i) a.perm[i] = (uint16_t)i;
+        }
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
