@@ -2,11 +2,14 @@
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package. The library (``bit_gemv_gemm_dfssm_b200``)
-never imports it, and the two share no code. ``dfssm_oracle.cpp`` holds the
-arithmetic, written as plain loops; this file only loads it and marshals numpy
-arrays.
+never imports it, and the two share no code. ``dfssm_oracle.cpp`` (the layer,
+the int8 table), ``ssm_oracle.cpp`` (the state operations) and
+``block_oracle.cpp`` (the block frame: residual add and RMS norm) hold the
+arithmetic, written as plain loops; this file only loads them and marshals
+numpy arrays.
 
-Every function is pinned by ``tests/test_oracle_pins.py`` against brute force,
+Every function is pinned (``tests/test_oracle_pins.py``,
+``tests/test_ssm_oracle_pins.py``, ``tests/test_block_oracle_pins.py``) against brute force,
 closed forms, invariants and hand-computed fixtures; no function here is
 "parity unpinned".
 """
@@ -20,7 +23,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "dfssm_oracle.cpp")
-_SRCS = [_SRC, os.path.join(_HERE, "ssm_oracle.cpp")]
+_SRCS = [_SRC, os.path.join(_HERE, "ssm_oracle.cpp"), os.path.join(_HERE, "block_oracle.cpp")]
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 
 
@@ -63,6 +66,7 @@ def _L():
         lib.dfssm_oracle_ssm_step.argtypes = [i32, i32, i32, i32, dbl, i32, vp, vp, vp, vp, vp, vp, vp, vp,
                                               vp, vp, vp, vp, vp, vp, vp, vp]
         lib.dfssm_oracle_lm_head_sampled.argtypes = [vp, vp, i32, i32, vp, i32, vp, vp, i64, vp, vp]
+        lib.dfssm_oracle_add_rmsnorm.argtypes = [i32, dbl, i32, vp, vp, i32, vp, vp, vp, vp]
         _lib = lib
     return _lib
 
@@ -235,3 +239,27 @@ def ssm_step(dims, inp):
                                s_out.ctypes.data, *[p for _, p in par], out.ctypes.data, xc.ctypes.data,
                                dt.ctypes.data, dA.ctypes.data, y.ctypes.data, r.ctypes.data)
     return dict(ssm_state=s_out, out=out, conv_state=cs, xc=xc, dt=dt, dA=dA, y=y, r=r)
+
+
+def add_rmsnorm(resid, delta, w, eps):
+    """The residual add and RMS norm of the Mamba-2 block frame (block_oracle.cpp).
+
+    resid: m x d float32; delta: m x d bf16 bits (uint16) or float32, or None; w: d float32.
+    Returns the new residual (float32: the fp32 sum), the normed output (float64) and the
+    per-token factor 1/sqrt(mean(r^2) + eps) (float64)."""
+    r_in, pr = _c(resid, np.float32)
+    m, d = r_in.shape
+    wv, pw = _c(w, np.float32)
+    assert wv.shape == (d,)
+    pd, bf = None, 0
+    if delta is not None:
+        dl = np.ascontiguousarray(delta)
+        assert dl.shape == (m, d) and dl.dtype in (np.uint16, np.float32)
+        bf = 1 if dl.dtype == np.uint16 else 0
+        pd = dl.ctypes.data
+    r_out = np.empty((m, d), np.float32)
+    out = np.empty((m, d), np.float64)
+    r = np.empty(m, np.float64)
+    _L().dfssm_oracle_add_rmsnorm(d, float(eps), m, pr, pd, bf, pw, r_out.ctypes.data, out.ctypes.data,
+                                  r.ctypes.data)
+    return dict(resid=r_out, out=out, r=r)
