@@ -9,7 +9,8 @@ The entry points keep the C names: ``dfssm_linear_plan``, ``dfssm_plan_destroy``
 ``dfssm_pack_sign``, ``dfssm_linear_fwd``, ``dfssm_linear_stack_fwd``,
 ``dfssm_plan_check``, ``dfssm_plan_workspace_bytes``, ``dfssm_status_string``,
 ``dfssm_linear_fwd_noalloc``, ``dfssm_plan_set_test_hooks``, ``dfssm_embed_fwd``,
-``dfssm_lm_head_fwd``.
+``dfssm_lm_head_fwd``, ``dfssm_ssm_workspace_bytes``, ``dfssm_ssm_step``,
+``dfssm_ssm_read_error``, ``dfssm_add_rmsnorm``.
 """
 from __future__ import annotations
 
@@ -42,7 +43,7 @@ EXPORTS = (
     "dfssm_linear_plan", "dfssm_plan_destroy", "dfssm_pack_sign", "dfssm_linear_fwd",
     "dfssm_linear_stack_fwd", "dfssm_plan_check", "dfssm_plan_workspace_bytes", "dfssm_status_string",
     "dfssm_linear_fwd_noalloc", "dfssm_plan_set_test_hooks", "dfssm_embed_fwd", "dfssm_lm_head_fwd",
-    "dfssm_ssm_workspace_bytes", "dfssm_ssm_step", "dfssm_ssm_read_error",
+    "dfssm_ssm_workspace_bytes", "dfssm_ssm_step", "dfssm_ssm_read_error", "dfssm_add_rmsnorm",
 )
 DFSSM_DEVERR_TOKEN_ID = 0x10
 DFSSM_TEST_STALL = 0x1
@@ -117,6 +118,7 @@ def _load():
     lib.dfssm_ssm_workspace_bytes.argtypes = [ctypes.POINTER(SsmDims), i32, i32, ctypes.POINTER(ctypes.c_size_t)]
     lib.dfssm_ssm_step.argtypes = [ctypes.POINTER(SsmDims), vp, i32, i32, vp, ctypes.c_size_t, vp]
     lib.dfssm_ssm_read_error.argtypes = [vp, u32p, vp]
+    lib.dfssm_add_rmsnorm.argtypes = [vp, i32, ctypes.c_float, vp, vp, i32, i32, vp, vp, i32, vp]
     lib.dfssm_status_string.restype = ctypes.c_char_p
     lib.dfssm_status_string.argtypes = [ctypes.c_int]
     for name in EXPORTS:
@@ -258,3 +260,10 @@ def ssm_layers_bytes(layers) -> bytes:
     """Pack a list of SsmLayer into the byte image the device array must hold."""
     arr = (SsmLayer * len(layers))(*layers)
     return ctypes.string_at(ctypes.addressof(arr), ctypes.sizeof(arr))
+
+
+def dfssm_add_rmsnorm(norm_w_ptr: int, d: int, eps: float, resid_in_ptr: int, delta_ptr: int, delta_dtype: int,
+                      m: int, resid_out_ptr: int, out_ptr: int, out_dtype: int, stream: int = 0) -> None:
+    """Residual add and RMS norm of the Mamba-2 block frame (see include/dfssm.h)."""
+    _check(lib().dfssm_add_rmsnorm(norm_w_ptr, d, eps, resid_in_ptr, delta_ptr or None, delta_dtype, m,
+                                   resid_out_ptr, out_ptr, out_dtype, stream), "dfssm_add_rmsnorm")

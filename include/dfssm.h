@@ -284,6 +284,25 @@ dfssm_status dfssm_ssm_step(const dfssm_ssm_dims* dims, const dfssm_ssm_layer* l
  * DFSSM_ERR_DEVICE_CHECK if it was set. */
 dfssm_status dfssm_ssm_read_error(void* workspace, uint32_t* bits, void* stream);
 
+/* ---- the frame of a Mamba-2 block: residual add and RMS norm ------------------------------
+ * "Density Field State Space Models" (gist.science technical summary), §2.B and §3: the
+ * model is Mamba-2 1.3B (48 layers, d_model 2048) with in_proj / out_proj replaced by the
+ * layer above. Around the layer each block keeps Mamba-2's frame: an fp32 residual stream r,
+ *   r_new = r + delta            (delta: the previous block's out_proj output; NULL: none)
+ *   out   = r_new / sqrt(mean(r_new^2) + eps) * norm_w      (the next in_proj's input,
+ *                                                           or the LM head's after the last block)
+ * per token, over d channels. r_new is one fp32 addition per element; the mean square is
+ * summed in fp32 in a fixed order and the output rounded once (bf16 nearest even, or fp32).
+ * Device pointers, caller-owned, 16-byte aligned: norm_w d fp32; resid_in, resid_out m x d
+ * fp32 (resid_out may equal resid_in: in place); delta m x d of delta_dtype (DFSSM_BF16 or
+ * DFSSM_F32) or NULL; out m x d of out_dtype (DFSSM_BF16 or DFSSM_F32). 8 <= d <= 8192,
+ * d % 8 == 0, 1 <= m <= 65536 (else DFSSM_ERR_UNSUPPORTED_SHAPE); eps finite and >= 0.
+ * One kernel (one CTA per token) on `stream`; allocates nothing; argument errors return
+ * synchronously with no launch. */
+dfssm_status dfssm_add_rmsnorm(const float* norm_w, int32_t d, float eps, const float* resid_in,
+                               const void* delta, int32_t delta_dtype, int32_t m, float* resid_out,
+                               void* out, int32_t out_dtype, void* stream);
+
 /* Test of the error path of the decode kernel (m <= 16 tokens), which must end with an
  * error status and never hang. With flags & DFSSM_TEST_STALL, the first CTA of that
  * kernel waits on a barrier that nothing arrives on: the wait gives up after

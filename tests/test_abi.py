@@ -85,6 +85,21 @@ def test_argument_errors_without_gpu():
     assert lib.dfssm_ssm_workspace_bytes(ctypes.byref(nan_eps), 1, 1, ctypes.byref(n)) == dfssm.DFSSM_ERR_INVALID_ARG
     assert lib.dfssm_ssm_step(ctypes.byref(dims), None, 1, 1, None, 0, None) == dfssm.DFSSM_ERR_INVALID_ARG
     assert lib.dfssm_ssm_step(ctypes.byref(dims), 256, 1, 1, 4096, 16, None) == dfssm.DFSSM_ERR_INVALID_ARG
+    # the block frame: shapes, alignment, eps and dtypes are checked before any launch
+    A = 1 << 12                                              # 16-byte aligned dummy addresses
+    args = dict(w=A, d=2048, eps=1e-5, rin=A, delta=A, ddt=dfssm.DFSSM_BF16, m=1, rout=A, out=A,
+                odt=dfssm.DFSSM_BF16)
+
+    def norm(**kw):
+        a = dict(args, **kw)
+        return lib.dfssm_add_rmsnorm(a["w"], a["d"], a["eps"], a["rin"], a["delta"], a["ddt"], a["m"], a["rout"],
+                                     a["out"], a["odt"], None)
+
+    for bad in (dict(d=2044), dict(d=0), dict(d=8200), dict(m=0), dict(m=65537)):
+        assert norm(**bad) == dfssm.DFSSM_ERR_UNSUPPORTED_SHAPE, bad
+    for bad in (dict(w=None), dict(rin=A + 4), dict(delta=A + 8), dict(out=None), dict(eps=-1.0),
+                dict(eps=float("inf")), dict(ddt=dfssm.DFSSM_I8), dict(odt=7)):
+        assert norm(**bad) == dfssm.DFSSM_ERR_INVALID_ARG, bad
     assert dfssm.dfssm_status_string(dfssm.DFSSM_ERR_CUDA) == "CUDA error"
     with pytest.raises(dfssm.DfssmError):
         dfssm.dfssm_linear_plan([(100, 10, 1, 0)])
