@@ -482,6 +482,19 @@ def lm_head_block(torch, seed, peaks, dev, m=1, steps=200):
             "traffic": recorded_traffic(f"lm_head_m{m}")}
 
 
+def ssm_layer_bytes(dims, m):
+    """Algorithmic bytes of one layer's state step at m tokens: zxbcdt in, shift register and
+    SSM state in and out, out (bf16), parameters."""
+    d_inner, N, conv = dims["d_inner"], dims["d_state"], dims["d_conv"]
+    nheads = d_inner // dims["headdim"]
+    conv_dim = d_inner + 2 * N
+    return m * (2 * (2 * d_inner + 2 * N + nheads)             # zxbcdt (bf16) in
+                + 2 * 2 * conv_dim * conv                       # shift register (bf16) in and out
+                + 2 * 4 * nheads * dims["headdim"] * N          # SSM state (fp32) in and out
+                + 2 * d_inner) \
+        + 4 * (conv_dim * conv + conv_dim + 3 * nheads + d_inner)   # parameters (fp32)
+
+
 def ssm_block(torch, seed, peaks, dev, n_layers=48, m=1, steps=200):
     """The decode step of the state operations (shift register + SSM recurrence) for the 48 layers
     of Mamba-2 1.3B at m tokens: two full sets of inputs and states alternated (2 x 208 MB > L2),
@@ -521,16 +534,156 @@ def ssm_block(torch, seed, peaks, dev, n_layers=48, m=1, steps=200):
     assert st == dfssm.DFSSM_OK, hex(bits)
     del gs
     us = ms * 1e3 / steps
-    per_layer = m * (2 * (2 * d_inner + 2 * N + nheads)        # zxbcdt (bf16) in
-                     + 2 * 2 * conv_dim * conv                  # shift register (bf16) in and out
-                     + 2 * 4 * nheads * dims["headdim"] * N     # SSM state (fp32) in and out
-                     + 2 * d_inner) \
-        + 4 * (conv_dim * conv + conv_dim + 3 * nheads + d_inner)   # parameters (fp32)
-    nb = n_layers * per_layer
+    nb = n_layers * ssm_layer_bytes(dims, m)
     return {"workload": f"ssm_step{n_layers}_m{m}", "m": m, "layers": n_layers, "us_per_step": us,
             "GB/s": nb / (us * 1e-6) / 1e9, "hbm_frac": nb / (us * 1e-6) / 1e9 / peaks["hbm"],
             "bytes_per_step": nb, "tokens_per_s": m / (us * 1e-6), "gpu_launches_per_step": 2,
             "l2": "two sets of inputs and states alternated", "traffic": recorded_traffic(f"ssm_step{n_layers}_m{m}")}
+
+
+class ChainRunner:
+    """The model's whole decode step for m tokens as one CUDA graph of the library's calls:
+    the int8 embedding, then per block the residual add + RMS norm, in_proj, the state step and
+    out_proj, then the last residual add + RMS norm and the int8 LM head. Every block has its own
+    output buffers, so each stage's input and output can be read back after a step; the
+    shift-register and SSM states are updated in place, so each replay decodes the next token."""
+
+    def __init__(self, m, seed, n_layers=synth.N_LAYERS, d_model=synth.D_MODEL, dims=None, vocab=synth.VOCAB,
+                 cfg=2):
+        import torch
+        import bit_gemv_gemm_dfssm_b200 as dfssm
+        self.torch, self.dfssm = torch, dfssm
+        dims = dict(dims or synth.SSM_DIMS)
+        self.m, self.n, self.d, self.dims, self.vocab = m, n_layers, d_model, dims, vocab
+        d_inner, N = dims["d_inner"], dims["d_state"]
+        self.nheads = d_inner // dims["headdim"]
+        self.zx_w = 2 * d_inner + 2 * N + self.nheads
+        self.shapes = [(d_model, self.zx_w), (d_inner, d_model)]
+
+        def dev(a):
+            a = np.ascontiguousarray(a)
+            return torch.from_numpy(a.view(np.int16).copy() if a.dtype == np.uint16 else a.copy()).cuda()
+
+        wc = synth.weight_cfg(cfg)
+        self.w_host, self.w = [], []
+        for i in range(2 * n_layers):
+            d_in, d_out = self.shapes[i % 2]
+            w = synth.linear_weights(seed, wc, i, d_in, d_out)
+            self.w_host.append(w)
+            self.w.append({k: dev(v) for k, v in w.items()})
+        self.ssm_host = [synth.ssm_layer_inputs(seed, cfg, i, m, dims) for i in range(n_layers)]
+        self.ssm = [{k: dev(v) for k, v in x.items() if k != "zxbcdt"} for x in self.ssm_host]
+        self.nw_host = [synth.block_norm_weights(seed, cfg, i, d_model) for i in range(n_layers + 1)]
+        self.nw = [dev(v) for v in self.nw_host]
+        self.table_host = synth.int8_table(seed, cfg, vocab, d_model)
+        self.table = {k: dev(v) for k, v in self.table_host.items()}
+        self.tc = dfssm.Int8Table(self.table["table"].data_ptr(), self.table["scale"].data_ptr(), vocab, d_model)
+        self.ids_host = synth.token_ids(seed, cfg, m, vocab)
+        self.ids = dev(self.ids_host)
+        f32, bf16 = torch.float32, torch.bfloat16
+        e = dict(device="cuda")
+        self.emb = torch.empty((m, d_model), dtype=f32, **e)
+        self.resid = [torch.empty((m, d_model), dtype=f32, **e) for _ in range(n_layers + 1)]
+        self.xn = [torch.empty((m, d_model), dtype=bf16, **e) for _ in range(n_layers + 1)]
+        self.zx = [torch.empty((m, self.zx_w), dtype=bf16, **e) for _ in range(n_layers)]
+        self.so = [torch.empty((m, d_inner), dtype=bf16, **e) for _ in range(n_layers)]
+        self.yo = [torch.empty((m, d_model), dtype=bf16, **e) for _ in range(n_layers)]
+        self.logits = torch.empty((m, vocab), dtype=f32, **e)
+        self.plan = dfssm.dfssm_linear_plan([(d_in, d_out, m, dfssm.DFSSM_BF16) for d_in, d_out in self.shapes])
+        self.c = dfssm.SsmDims(d_inner, dims["headdim"], N, dims["d_conv"], dims["eps"], dfssm.DFSSM_BF16)
+        layers = [dfssm.SsmLayer(self.zx[i].data_ptr(), *[self.ssm[i][k].data_ptr() for k in (
+            "conv_state", "ssm_state", "conv_w", "conv_b", "dt_bias", "a_log", "d_skip", "norm_w")],
+            self.so[i].data_ptr()) for i in range(n_layers)]
+        self.layer_bytes = len(dfssm.ssm_layers_bytes(layers[:1]))
+        self.ldev = torch.frombuffer(bytearray(dfssm.ssm_layers_bytes(layers)), dtype=torch.uint8).cuda()
+        self.wsb = dfssm.dfssm_ssm_workspace_bytes(self.c, 1, m)
+        self.ws = torch.zeros(self.wsb // 4 + 64, dtype=torch.int32, **e)
+        self.ws_ptr = (self.ws.data_ptr() + 255) // 256 * 256
+        self.ws_ptr_bytes = self.wsb
+        # the per-device set-up of the table calls, before any capture
+        stream = torch.cuda.current_stream().cuda_stream
+        dfssm.dfssm_embed_fwd(self.tc, self.ids.data_ptr(), m, self.emb.data_ptr(), dfssm.DFSSM_F32, 0, stream)
+        torch.cuda.synchronize()
+
+    def weights(self, i):
+        w = self.w[i]
+        return self.dfssm.weights_struct(w["sign"], w["alpha"], w["wa"], w["sa"], w["wb"], w["sb"])
+
+    def step(self, stream):
+        """Enqueue one decode step (1 + 7 n + 2 kernel launches)."""
+        dfssm, m, d = self.dfssm, self.m, self.d
+        BF16, F32 = dfssm.DFSSM_BF16, dfssm.DFSSM_F32
+        eps = self.dims["eps"]
+        dfssm.dfssm_embed_fwd(self.tc, self.ids.data_ptr(), m, self.emb.data_ptr(), F32, 0, stream)
+        for i in range(self.n):
+            r_in = self.emb if i == 0 else self.resid[i - 1]
+            delta = 0 if i == 0 else self.yo[i - 1].data_ptr()
+            dfssm.dfssm_add_rmsnorm(self.nw[i].data_ptr(), d, eps, r_in.data_ptr(), delta, BF16, m,
+                                    self.resid[i].data_ptr(), self.xn[i].data_ptr(), BF16, stream)
+            dfssm.dfssm_linear_fwd(self.plan, 0, self.weights(2 * i), self.xn[i].data_ptr(), m, self.zx[i].data_ptr(),
+                                   None, stream)
+            dfssm.dfssm_ssm_step(self.c, self.ldev.data_ptr() + i * self.layer_bytes, 1, m, self.ws_ptr,
+                                 self.ws_ptr_bytes, stream)
+            dfssm.dfssm_linear_fwd(self.plan, 1, self.weights(2 * i + 1), self.so[i].data_ptr(), m,
+                                   self.yo[i].data_ptr(), None, stream)
+        n = self.n
+        dfssm.dfssm_add_rmsnorm(self.nw[n].data_ptr(), d, eps, self.resid[n - 1].data_ptr(), self.yo[n - 1].data_ptr(),
+                                BF16, m, self.resid[n].data_ptr(), self.xn[n].data_ptr(), BF16, stream)
+        dfssm.dfssm_lm_head_fwd(self.tc, self.xn[n].data_ptr(), m, self.logits.data_ptr(), F32, 0, stream)
+
+    def launches(self):
+        return 1 + 7 * self.n + 2
+
+    def graph(self):
+        torch = self.torch
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            self.step(torch.cuda.current_stream().cuda_stream)
+        torch.cuda.synchronize()
+        return g
+
+    def bytes_per_step(self):
+        """Algorithmic bytes of one step: every weight once (scaffold + LoRA + scales, the int8
+        table and its scales, the state parameters, the norm weights), the shift-register and
+        SSM states in and out, and the activations between the stages."""
+        m, d, V = self.m, self.d, self.vocab
+        lin = stack_bytes(self.shapes * self.n, m)
+        ssm = self.n * ssm_layer_bytes(self.dims, m)
+        norms = (self.n + 1) * (4 * d + m * (4 * d + 2 * d + 4 * d + 2 * d))   # w; r in, delta in, r out, out
+        head = V * d + 4 * V + 2 * m * d + 4 * m * V
+        embed = m * (d + 4 + 4 * d + 4)
+        return lin + ssm + norms + head + embed
+
+    def check(self):
+        st, bits = self.dfssm.dfssm_ssm_read_error(self.ws_ptr, self.torch.cuda.current_stream().cuda_stream)
+        if st != self.dfssm.DFSSM_OK:
+            raise RuntimeError(f"state step error word set: {bits:#x}")
+        st, bits = self.dfssm.dfssm_plan_check(self.plan)
+        if st != self.dfssm.DFSSM_OK:
+            raise RuntimeError(f"linear error word set: {bits:#x}")
+
+    def close(self):
+        self.dfssm.dfssm_plan_destroy(self.plan)
+
+
+def chain_block(torch, seed, peaks, dev, m=1, steps=100):
+    """The model's whole decode step (48 blocks of Mamba-2 1.3B with the layer in every in_proj
+    and out_proj, embedding and LM head in int8) at m tokens, one CUDA graph per step; each step
+    decodes the next token (the states carry over). Reads about 480 MB per token, well above L2."""
+    r = ChainRunner(m, seed)
+    g = r.graph()
+    ms = timed_device(torch, lambda i: g.replay(), steps, 3, None, dev)
+    r.check()
+    del g
+    r.close()
+    us = ms * 1e3 / steps
+    nb = r.bytes_per_step()
+    return {"workload": f"decode_step48_m{m}", "m": m, "layers": r.n, "us_per_step": us,
+            "tokens_per_s": m / (us * 1e-6), "GB/s": nb / (us * 1e-6) / 1e9,
+            "hbm_frac": nb / (us * 1e-6) / 1e9 / peaks["hbm"], "bytes_per_step": nb,
+            "gpu_launches_per_step": r.launches(), "l2": "one step reads every weight and state once (~480 MB)"}
 
 
 def timed_device(torch, run_step, steps, warmup, dist, dev):
@@ -645,10 +798,11 @@ def run_gpu(args, wl_name):
         del pgraphs
 
     # the other configurations: single projections (cold L2), the stack at M = 4 / 16 / 64 / 512,
-    # the int8 LM head, the decode step of the state operations (every rank runs the same blocks; rank 0
+    # the int8 LM head, the decode step of the state operations, the model's whole chained decode
+    # step (every rank runs the same blocks; rank 0 reports them)
     extras = None
     if not args.no_extras:
-        extras = {"single": [], "stacks": [], "lm_head": None, "ssm_step": None}
+        extras = {"single": [], "stacks": [], "lm_head": None, "ssm_step": None, "decode_step": None}
         for wn in ("out_proj_m1", "in_proj_m1"):
             extras["single"].append(single_block(torch, wn, seed, peaks, dev))
         sets = device_weight_sets(synth.stack_shapes(), 2, seed)
@@ -659,6 +813,8 @@ def run_gpu(args, wl_name):
         extras["lm_head"] = lm_head_block(torch, seed, peaks, dev)
         torch.cuda.empty_cache()
         extras["ssm_step"] = ssm_block(torch, seed, peaks, dev)
+        torch.cuda.empty_cache()
+        extras["decode_step"] = chain_block(torch, seed, peaks, dev)
 
     if rank != 0:
         if dist is not None:

@@ -33,6 +33,7 @@ N_LAYERS = 48
 T_X, T_COLS, T_SIGN, T_ALPHA, T_WA, T_SA, T_WB, T_SB, T_TABLE, T_TSCALE, T_IDS = range(11)
 (T_ZXBCDT, T_CONV_STATE, T_SSM_STATE, T_CONV_W, T_CONV_B, T_DT_BIAS, T_A_LOG, T_D_SKIP,
  T_NORM_W) = range(11, 20)
+T_BLOCK_NORM = 20
 KIND_WEIGHTS, KIND_ACT = 1, 2
 # the tied int8 embedding / LM-head table of Mamba-2 1.3B: its 50,277-token vocabulary padded to
 # a multiple of 16, d_model columns
@@ -197,6 +198,15 @@ def ssm_layer_inputs(seed: int, cfg: int, index: int, m: int, dims=None) -> dict
     L.dfssm_synth_uniform_f32(k_(KIND_WEIGHTS, T_D_SKIP), nheads, 0.5, 1.5, _ptr(out["d_skip"]))
     L.dfssm_synth_uniform_f32(k_(KIND_WEIGHTS, T_NORM_W), d_inner, 0.5, 1.5, _ptr(out["norm_w"]))
     return out
+
+
+def block_norm_weights(seed: int, cfg: int, index: int, d: int) -> np.ndarray:
+    """The RMS-norm weight in front of block `index` (index = the number of blocks: the final
+    norm before the LM head), U(0.5, 1.5) fp32."""
+    w = np.empty(d, np.float32)
+    _L().dfssm_synth_uniform_f32(key(seed, stream_id(KIND_WEIGHTS, cfg, 0, index, T_BLOCK_NORM)), d, 0.5, 1.5,
+                                 _ptr(w))
+    return w
 
 
 def stack_shapes(n_layers: int = N_LAYERS):
