@@ -4,12 +4,13 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package. The library (``bit_gemv_gemm_dfssm_b200``)
 never imports it, and the two share no code. ``dfssm_oracle.cpp`` (the layer,
 the int8 table), ``ssm_oracle.cpp`` (the state operations) and
-``block_oracle.cpp`` (the block frame: residual add and RMS norm) hold the
-arithmetic, written as plain loops; this file only loads them and marshals
+``block_oracle.cpp`` (the block frame: residual add and RMS norm) and
+``density_oracle.cpp`` (the state density field) hold the arithmetic, written as plain loops; this file only loads them and marshals
 numpy arrays.
 
 Every function is pinned (``tests/test_oracle_pins.py``,
-``tests/test_ssm_oracle_pins.py``, ``tests/test_block_oracle_pins.py``) against brute force,
+``tests/test_ssm_oracle_pins.py``, ``tests/test_block_oracle_pins.py``,
+``tests/test_density_oracle_pins.py``) against brute force,
 closed forms, invariants and hand-computed fixtures; no function here is
 "parity unpinned".
 """
@@ -23,7 +24,8 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "dfssm_oracle.cpp")
-_SRCS = [_SRC, os.path.join(_HERE, "ssm_oracle.cpp"), os.path.join(_HERE, "block_oracle.cpp")]
+_SRCS = [_SRC, os.path.join(_HERE, "ssm_oracle.cpp"), os.path.join(_HERE, "block_oracle.cpp"),
+         os.path.join(_HERE, "density_oracle.cpp")]
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 
 
@@ -67,6 +69,8 @@ def _L():
                                               vp, vp, vp, vp, vp, vp, vp, vp]
         lib.dfssm_oracle_lm_head_sampled.argtypes = [vp, vp, i32, i32, vp, i32, vp, vp, i64, vp, vp]
         lib.dfssm_oracle_add_rmsnorm.argtypes = [i32, dbl, i32, vp, vp, i32, vp, vp, vp, vp]
+        lib.dfssm_oracle_density_encode.argtypes = [i32, i32, i32, vp, vp, vp]
+        lib.dfssm_oracle_density_decode.argtypes = [i32, i32, i32, vp, vp, vp]
         _lib = lib
     return _lib
 
@@ -263,3 +267,26 @@ def add_rmsnorm(resid, delta, w, eps):
     _L().dfssm_oracle_add_rmsnorm(d, float(eps), m, pr, pd, bf, pw, r_out.ctypes.data, out.ctypes.data,
                                   r.ctypes.data)
     return dict(resid=r_out, out=out, r=r)
+
+
+def density_encode(state, K: int):
+    """The state density field of each row (density_oracle.cpp): state rows x d_state float32.
+    Returns (scale: rows float32, bits: rows x ceil(K*K/8) uint8, LSB-first cells)."""
+    st, ps = _c(state, np.float32)
+    rows, d = st.shape
+    assert K * K >= d, "every value needs at least one cell"
+    scale = np.empty(rows, np.float32)
+    bits = np.empty((rows, (K * K + 7) // 8), np.uint8)
+    _L().dfssm_oracle_density_encode(rows, d, K, ps, scale.ctypes.data, bits.ctypes.data)
+    return scale, bits
+
+
+def density_decode(scale, bits, d_state: int, K: int):
+    """The popcount readout: rows x d_state float64 values from the scales and fields."""
+    sc, psc = _c(scale, np.float32)
+    b, pb = _c(bits, np.uint8)
+    rows = sc.size
+    assert K * K >= d_state and b.shape == (rows, (K * K + 7) // 8)
+    out = np.empty((rows, d_state), np.float64)
+    _L().dfssm_oracle_density_decode(rows, d_state, K, psc, pb, out.ctypes.data)
+    return out
