@@ -1,6 +1,8 @@
 /*
  * dfssm.h - C ABI of libdfssm: the DF-SSM 1-bit scaffold + int8 LoRA linear on
- * NVIDIA B200 (sm_100a).
+ * NVIDIA B200 (sm_100a), and the parts of the model's decode step around it (the
+ * int8 embedding / LM head, the Mamba-2 state step, the block frame), each
+ * declared in its own section below.
  *
  * The layer ("Density Field State Space Models", gist.science technical
  * summary, §2.B "frozen scaffold with LoRA correction" and §2.C "optimised
@@ -24,8 +26,10 @@
  *   - alpha, s_A: one fp32 per output row; s_B: one fp32 per LoRA row.
  *   - s_x multiplies both terms; s_B * h stays in fp32 (not re-quantised).
  *
- * Memory: every tensor pointer is a DEVICE pointer owned by the caller; the
- * library never frees it. Tensor pointers must be 16-byte aligned. A plan owns
+ * Memory: every tensor pointer is a DEVICE pointer owned by the caller (a
+ * stack entry's y may also be the device address of mapped pinned host memory,
+ * see dfssm_stack_entry); the library never frees it. Tensor pointers must be
+ * 16-byte aligned. A plan owns
  * its workspace (device memory allocated by dfssm_linear_plan, freed by
  * dfssm_plan_destroy) and is tied to the device current at plan time.
  *
