@@ -541,6 +541,22 @@ def ssm_block(torch, seed, peaks, dev, n_layers=48, m=1, steps=200):
             "l2": "two sets of inputs and states alternated", "traffic": recorded_traffic(f"ssm_step{n_layers}_m{m}")}
 
 
+def chain_bytes(n_layers, d_model, dims, vocab, m):
+    """Algorithmic bytes of one chained decode step: every weight once (scaffold + LoRA + scales,
+    the int8 table and its scales, the state parameters, the norm weights), the shift-register and
+    SSM states in and out, and the activations between the stages (fp32 residual, bf16 between
+    the kernels, fp32 logits)."""
+    d_inner, N = dims["d_inner"], dims["d_state"]
+    zx_w = 2 * d_inner + 2 * N + d_inner // dims["headdim"]
+    lin = stack_bytes([(d_model, zx_w), (d_inner, d_model)] * n_layers, m)
+    ssm = n_layers * ssm_layer_bytes(dims, m)
+    d, V = d_model, vocab
+    norms = (n_layers + 1) * (4 * d + m * (4 * d + 2 * d + 4 * d + 2 * d))   # w; r in, delta in, r out, out
+    head = V * d + 4 * V + 2 * m * d + 4 * m * V
+    embed = m * (d + 4 + 4 * d + 4)                                            # row, scale, out, id
+    return lin + ssm + norms + head + embed
+
+
 class ChainRunner:
     """The model's whole decode step for m tokens as one CUDA graph of the library's calls:
     the int8 embedding, then per block the residual add + RMS norm, in_proj, the state step and
@@ -645,16 +661,7 @@ class ChainRunner:
         return g
 
     def bytes_per_step(self):
-        """Algorithmic bytes of one step: every weight once (scaffold + LoRA + scales, the int8
-        table and its scales, the state parameters, the norm weights), the shift-register and
-        SSM states in and out, and the activations between the stages."""
-        m, d, V = self.m, self.d, self.vocab
-        lin = stack_bytes(self.shapes * self.n, m)
-        ssm = self.n * ssm_layer_bytes(self.dims, m)
-        norms = (self.n + 1) * (4 * d + m * (4 * d + 2 * d + 4 * d + 2 * d))   # w; r in, delta in, r out, out
-        head = V * d + 4 * V + 2 * m * d + 4 * m * V
-        embed = m * (d + 4 + 4 * d + 4)
-        return lin + ssm + norms + head + embed
+        return chain_bytes(self.n, self.d, self.dims, self.vocab, self.m)
 
     def check(self):
         st, bits = self.dfssm.dfssm_ssm_read_error(self.ws_ptr, self.torch.cuda.current_stream().cuda_stream)
