@@ -22,7 +22,8 @@
  *     bit 1 -> +1, bit 0 -> -1.
  *   - quantiser, in IEEE fp32 with round-to-nearest: amax = max_j |x[t,j]|;
  *     amax == 0 -> q = 0, s_x = 0; otherwise inv = 127/amax,
- *     q = clamp(round_half_even(x * inv), -127, 127), s_x = amax/127.
+ *     q = clamp(round_half_even(x * inv), -127, 127), s_x = amax/127
+ *     (amax below 127/FLT_MAX overflows inv: nonzero entries give +-127, zeros 0).
  *   - alpha, s_A: one fp32 per output row; s_B: one fp32 per LoRA row.
  *   - s_x multiplies both terms; s_B * h stays in fp32 (not re-quantised).
  *

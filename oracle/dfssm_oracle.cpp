@@ -150,6 +150,9 @@ static void quantize_token(const uint16_t* x, int d_in, int8_t* q, float* sx) {
     for (int j = 0; j < d_in; ++j) {
         volatile float v = bf16_to_float(x[j]) * inv;   // one fp32 product, RN
         float r = std::nearbyintf(v);                   // ties to even
+        // amax below 127 / FLT_MAX makes inv = +inf: a zero entry gives 0 * inf = NaN, taken as 0
+        // (x = 0 quantises to 0); a nonzero entry gives +-inf, clamped to +-127 below
+        if (std::isnan(r)) r = 0.0f;
         if (r > 127.0f) r = 127.0f;
         if (r < -127.0f) r = -127.0f;
         q[j] = (int8_t)r;

@@ -162,6 +162,23 @@ def test_quantizer_one_nonzero_channel():
         assert sx[0] == np.float32(abs(vv)) / np.float32(127)
 
 
+def test_quantizer_tiny_amax_saturates():
+    # amax below 127 / FLT_MAX (about 3.7e-37): inv = 127 / amax overflows to +inf in fp32, so
+    # every nonzero entry maps to +-127 and a zero entry (0 * inf) to 0; s_x stays amax / 127
+    for amax_bits in (0x0080, 0x0100, 0x01F0):          # bf16 2^-126, 2^-125, about 1.8e-37
+        x = np.zeros((1, 16), np.uint16)
+        x[0, 0] = amax_bits
+        x[0, 3] = amax_bits ^ 0x8000                     # -amax
+        x[0, 7] = 0x0001                                 # the smallest bf16 subnormal
+        q, sx = oracle.quantize(x, 1, 16)
+        a = oracle.bf16_bits_to_f64(x)[0, 0]
+        assert np.float32(127) / np.float32(a) == np.inf
+        expect = np.zeros(16, np.int8)
+        expect[[0, 7]], expect[3] = 127, -127
+        np.testing.assert_array_equal(q[0], expect)
+        assert sx[0] == np.float32(a) / np.float32(127)
+
+
 # ---------------------------------------------------------------- the linear
 
 def test_linear_golden_hand_worked():
