@@ -23,7 +23,9 @@
  *   - quantiser, in IEEE fp32 with round-to-nearest: amax = max_j |x[t,j]|;
  *     amax == 0 -> q = 0, s_x = 0; otherwise inv = 127/amax,
  *     q = clamp(round_half_even(x * inv), -127, 127), s_x = amax/127
- *     (amax below 127/FLT_MAX overflows inv: nonzero entries give +-127, zeros 0).
+ *     (amax below 127/FLT_MAX overflows inv: nonzero entries give +-127, zeros 0;
+ *     known issue: for m > 16 tokens the quantiser does not yet follow this case and
+ *     gives 0 for nonzero entries and -1 for zeros of such a token).
  *   - alpha, s_A: one fp32 per output row; s_B: one fp32 per LoRA row.
  *   - s_x multiplies both terms; s_B * h stays in fp32 (not re-quantised).
  *
